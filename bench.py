@@ -1,0 +1,334 @@
+"""Throughput of the FBNL scoring path: reranked pairs/s on one query of 100 documents (Nano shape).
+
+python bench.py [--gpus N] [--steps K] [--warmup W] [--config nano] [--impl kalm|reference]
+
+One step = one query through the whole path (chunk pooling of every document's
+encoder states, the cross K/V projection of all layers, 18 decoder layers of
+Q|K|V projection + merged attention + output projection, and the yes/no
+readout), replayed as one CUDA graph with every input resident in HBM.  The L2
+is flushed (a 256 MiB write) before every step, outside the step's CUDA-event
+interval.  Rank 0 prints one JSON line.
+
+Multi-GPU (torchrun): every rank scores its own query of the same shape (the
+path shards by documents and queries; nothing crosses GPUs on the data path),
+so per-GPU work is fixed ("weak" scaling).  Timing is the max over ranks.
+
+--impl reference times the fp64 CPU oracle (the only reference this path has)
+on a bounded sample of the same workload on the host cores.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "reranked pairs/s (Nano shape, 1 B200); pool GB/s and attn TFLOP/s vs peak"
+UNIT = "pairs/s"
+L2_FLUSH_BYTES = 256 << 20
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=30)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--config", default="nano", choices=["tiny", "nano", "small", "large"])
+    ap.add_argument("--impl", default="kalm", choices=["kalm", "reference"])
+    ap.add_argument("--cpu-sample-docs", type=int, default=0, help="documents in the oracle sample (0 = auto)")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return dict(hbm=p["hbm_gbs"], bf16=p["bf16_tflops"], bf16_sustained=p["bf16_tflops_sustained"],
+                    source="measured")
+    return dict(hbm=6650.0, bf16=1590.0, bf16_sustained=1400.0, source="fallback")
+
+
+# ---------------------------------------------------------------------------
+# algorithmic work (what the method must do; padding and masked keys not counted)
+# ---------------------------------------------------------------------------
+def workload(q):
+    H, D, nq, nkv, L, lq = q.hidden, q.head_dim, q.n_q, q.n_kv, q.layers, q.lq
+    n = q.n_docs
+    lens = q.doc_len.astype(np.int64)
+    nc = (lens + 3) // 4
+    rows = n * lq
+    w = {}
+    w["pool_bytes"] = int((lens.sum() + nc.sum()) * H * 2 + 8 * n)
+    w["cross_flops"] = int(2 * nc.sum() * H * 2 * nkv * D * L)
+    w["cross_bytes"] = int(nc.sum() * H * 2 + L * H * 2 * nkv * D * 2 + nc.sum() * L * 2 * nkv * D * 2)
+    w["qkv_flops_per_layer"] = int(2 * rows * H * (nq + 2 * nkv) * D)
+    w["o_flops_per_layer"] = int(2 * rows * nq * D * H)
+    w["attn_flops_per_layer"] = int(4 * nq * D * (n * lq * (lq + 1) // 2 + lq * nc.sum()))
+    w["total_flops"] = w["cross_flops"] + L * (w["qkv_flops_per_layer"] + w["o_flops_per_layer"] +
+                                               w["attn_flops_per_layer"])
+    return w
+
+
+class Clocks:
+    """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = max(float(r[2]) for r in rows if r[2].replace(".", "").isdigit())
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+        loaded = [v for v in sm if v > 0.5 * mx] or sm
+        return {"sm_mhz": statistics.median(loaded) if loaded else None, "sm_max_mhz": mx, "reasons": reasons,
+                "samples": len(rows)}
+
+
+def cpu_baseline(q, n_sample: int):
+    """The fp64 oracle (as it stands) on the first n_sample documents of the query."""
+    import oracle
+    from threadpoolctl import threadpool_info
+    t0 = time.perf_counter()
+    oracle.forward_query(q, docs=range(n_sample))
+    dt = time.perf_counter() - t0
+    threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    return {"value": n_sample / dt, "unit": UNIT, "cores": threads, "kind": "oracle",
+            "sample": f"{n_sample} of {q.n_docs} documents of one {q.name} query, all {q.layers} layers, fp64 "
+                      f"numpy (BLAS threads={threads}); {dt:.1f} s"}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import synthetic
+    q = synthetic.make_query(args.config)
+    n_sample = args.cpu_sample_docs or (2 if args.config in ("nano", "tiny") else 1)
+    n_sample = min(n_sample, q.n_docs)
+    for _ in range(args.warmup):
+        cpu_baseline(q, 1)
+    times = []
+    cb = None
+    for _ in range(args.steps):
+        cb = cpu_baseline(q, n_sample)
+        times.append(n_sample / cb["value"])
+    total = sum(times)
+    value = n_sample * args.steps / total
+    cb["value"] = value
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": f"{q.name}: 1 query x {n_sample} sampled documents per step (of {q.n_docs})",
+                       "hidden": q.hidden, "layers": q.layers, "lq": q.lq},
+            "cpu_baseline": cb,
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        run_reference(args)
+        return
+    import torch
+    import torch.distributed as dist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+
+    import synthetic
+    from encoder_decoder_document_b200 import _build, kalm_check_device_errors
+    from encoder_decoder_document_b200.scorer import DeviceWeights, FBNLScorer
+
+    if rank == 0:
+        _build.build()
+    if world > 1:
+        dist.barrier()
+    # each rank scores its own query (its own document shard) of the configured shape
+    base = synthetic.CONFIGS[args.config]["seed"]
+    q = synthetic.make_query(args.config, seed=base if rank == 0 else base + 1000 * rank)
+    w = workload(q)
+    pk = peaks()
+    sc = FBNLScorer(DeviceWeights.from_bits(q.weights), q.n_q, q.n_kv)
+    total_pooled = int(((q.doc_len.astype(np.int64) + 3) // 4).sum())
+    sc.prepare(q.n_docs, int(q.doc_len.sum()), total_pooled, q.lq)
+    enc_h = torch.from_numpy(q.enc.view(np.int16)).view(torch.bfloat16).pin_memory()
+    len_h = torch.from_numpy(q.doc_len).pin_memory()
+    x0_h = torch.from_numpy(q.x0.view(np.int16)).view(torch.bfloat16).pin_memory()
+    out_h = torch.empty(4, q.n_docs, dtype=torch.float32).pin_memory()
+    sc.load_inputs(enc_h, len_h, x0_h)
+    sc.capture(instrument=True)
+    stream = torch.cuda.current_stream()
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device="cuda")
+
+    def step_timed():
+        flush.fill_(1.0)
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        sc.graph.replay()
+        b.record(stream)
+        return a, b
+
+    for _ in range(max(args.warmup, 3)):
+        step_timed()
+    torch.cuda.synchronize()
+    kalm_check_device_errors()
+
+    # ---------------- timed region: K steps, device-timed, per-kernel events inside the graph
+    clocks = Clocks(local)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    step_ms = []
+    per_kernel: dict = {}
+    for _ in range(args.steps):
+        a, b = step_timed()
+        b.synchronize()
+        step_ms.append(a.elapsed_time(b))
+        for label, v in sc.kernel_times().items():
+            per_kernel.setdefault(label, []).extend(v)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clk = clocks.stop()
+    kalm_check_device_errors()
+    total_ms = sum(step_ms)
+    if world > 1:
+        t = torch.tensor([total_ms], device="cuda", dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    value = world * q.n_docs * args.steps / (total_ms / 1e3)
+
+    # ---------------- end to end through the public API: H2D inputs, graph, D2H scores
+    e2e_ms = []
+    for _ in range(max(args.warmup, 3) + args.steps):
+        flush.fill_(1.0)
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        sc.load_inputs(enc_h, len_h, x0_h)
+        sc.graph.replay()
+        sc.scores_to_host(out_h)
+        b.record(stream)
+        b.synchronize()
+        e2e_ms.append(a.elapsed_time(b))
+    e2e_ms = e2e_ms[max(args.warmup, 3):]
+    e2e_total = sum(e2e_ms)
+    if world > 1:
+        t = torch.tensor([e2e_total], device="cuda", dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_total = float(t.item())
+    h2d = enc_h.numel() * 2 + len_h.numel() * 4 + x0_h.numel() * 2
+    d2h = out_h.numel() * 4
+
+    # ---------------- per-kernel summary and roofline of the dominant kernel
+    kern = {}
+    for label, v in per_kernel.items():
+        launches_per_step = len(v) / args.steps
+        kern[label] = {"launches_per_step": launches_per_step, "avg_us": 1e3 * statistics.mean(v),
+                       "share": sum(v) / max(sum(sum(x) for x in per_kernel.values()), 1e-12)}
+    flops_per_launch = {"qkv_proj": w["qkv_flops_per_layer"], "o_proj": w["o_flops_per_layer"],
+                        "merged_attention": w["attn_flops_per_layer"], "cross_kv_proj": w["cross_flops"]}
+    tensor_kernels = [k for k in kern if k in flops_per_launch]
+    dom = max(tensor_kernels, key=lambda k: kern[k]["share"])
+    dom_ach = flops_per_launch[dom] / (kern[dom]["avg_us"] * 1e-6) / 1e12
+    roofline = {"kernel": dom, "bound": "tensor", "achieved": dom_ach, "peak": pk["bf16"], "unit": "TFLOP/s",
+                "frac": dom_ach / pk["bf16"], "traffic": None,
+                "peak_source": f"{pk['source']} dense bf16 burst (cuBLAS)"}
+    pool_gbs = w["pool_bytes"] / (kern["chunk_pool"]["avg_us"] * 1e-6) / 1e9
+    attn_proj_us = sum(kern[k]["avg_us"] * kern[k]["launches_per_step"] for k in
+                       ("merged_attention", "cross_kv_proj") if k in kern)
+    attn_proj_flops = w["cross_flops"] + q.layers * w["attn_flops_per_layer"]
+    step_flops = w["total_flops"]
+    ms_step = total_ms / args.steps
+
+    if rank == 0:
+        cb = None
+        if not args.no_cpu_baseline and world == 1:
+            cb = cpu_baseline(q, args.cpu_sample_docs or 20)
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": f"{q.name}: 1 query x {q.n_docs} documents per GPU, hidden {q.hidden}, "
+                                   f"Lq {q.lq}, {q.n_q}q/{q.n_kv}kv heads x 256, {q.layers} layers",
+                       "docs_per_step": q.n_docs * world, "encoder_tokens": int(q.doc_len.sum()),
+                       "pooled_vectors": total_pooled, "parallelism": f"dp{world} (independent queries)",
+                       "l2": "flushed (256 MiB write) before every step, outside the step's events",
+                       "graph": "one CUDA graph per step with timing events between launches"},
+            "roofline": roofline,
+            "pool": {"bytes": w["pool_bytes"], "avg_us": kern["chunk_pool"]["avg_us"], "achieved_gbs": pool_gbs,
+                     "peak_gbs": pk["hbm"], "frac": pool_gbs / pk["hbm"]},
+            "attn_plus_cross_proj": {"flops": attn_proj_flops, "us": attn_proj_us,
+                                     "tflops": attn_proj_flops / (attn_proj_us * 1e-6) / 1e12,
+                                     "frac": attn_proj_flops / (attn_proj_us * 1e-6) / 1e12 / pk["bf16"]},
+            "step_tflops": step_flops / (ms_step * 1e-3) / 1e12,
+            "kernels": kern,
+            "e2e": {"value": world * q.n_docs * args.steps / (e2e_total / 1e3), "unit": UNIT,
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                    "ms_per_step": e2e_total / args.steps},
+            "gpu_launches": sc.launches * args.steps,
+            "clocks": clk,
+            "cpu_baseline": cb,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        sc.graph = None
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,129 @@
+"""KaLM-Reranker-V1 FBNL scoring hot path on B200: thin PyTorch binding of libkalm.
+
+Every function here marshals torch tensors (device memory owned by the caller)
+into the C ABI of ``include/kalm.h``; all arithmetic runs in the CUDA kernels of
+``libkalm.so``.  Functions keep the C names.  There is no CPU fallback: without
+the built library or an sm_100 device they raise ``KalmError``.
+"""
+from __future__ import annotations
+
+import ctypes
+from typing import Optional
+
+import torch
+
+from ._abi import KalmError, call, load, library_path  # noqa: F401
+
+__all__ = [
+    "KalmError", "load", "library_path", "kalm_version", "kalm_device_check", "kalm_check_device_errors",
+    "kalm_ragged_offsets", "kalm_chunk_pool", "kalm_linear", "kalm_cross_kv_proj", "kalm_merged_attention",
+    "kalm_yes_no_score", "kalm_broadcast_rows", "kalm_selftest_wait_timeout",
+]
+
+HEAD_DIM = 256
+
+
+def _stream(stream: Optional[torch.cuda.Stream]) -> int:
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return s.cuda_stream
+
+
+def _p(t: Optional[torch.Tensor], dtype: Optional[torch.dtype] = None) -> Optional[int]:
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise KalmError(1, "binding", "tensors must live on the CUDA device")
+    if dtype is not None and t.dtype != dtype:
+        raise KalmError(1, "binding", f"expected {dtype}, got {t.dtype}")
+    return t.data_ptr()
+
+
+def _ld(t: torch.Tensor) -> int:
+    """Row stride (elements) of a 2-D view whose last dimension is contiguous."""
+    if t.dim() != 2 or t.stride(1) != 1:
+        raise KalmError(1, "binding", "expected a 2-D tensor with contiguous rows")
+    return t.stride(0)
+
+
+def kalm_version() -> int:
+    return load().kalm_version()
+
+
+def kalm_device_check() -> None:
+    call("kalm_device_check")
+
+
+def kalm_check_device_errors(stream: Optional[torch.cuda.Stream] = None) -> int:
+    """Synchronise the stream and raise if a kernel recorded a device error."""
+    word = ctypes.c_uint32(0)
+    call("kalm_check_device_errors", _stream(stream), ctypes.byref(word))
+    return word.value
+
+
+def kalm_ragged_offsets(length: torch.Tensor, tok_off: Optional[torch.Tensor], pool_off: Optional[torch.Tensor],
+                        chunk: int = 4, stream=None) -> None:
+    call("kalm_ragged_offsets", _p(length, torch.int32), length.numel(), chunk, _p(tok_off, torch.int64),
+         _p(pool_off, torch.int64), _stream(stream))
+
+
+def kalm_chunk_pool(enc: torch.Tensor, tok_off: torch.Tensor, length: torch.Tensor, pooled: torch.Tensor,
+                    pool_off: torch.Tensor, total_pooled: int, chunk: int = 4, stream=None) -> None:
+    call("kalm_chunk_pool", _p(enc, torch.bfloat16), _ld(enc), _p(tok_off, torch.int64), _p(length, torch.int32),
+         length.numel(), enc.shape[1], chunk, _p(pooled, torch.bfloat16), _ld(pooled), _p(pool_off, torch.int64),
+         int(total_pooled), _stream(stream))
+
+
+def kalm_linear(x: torch.Tensor, w: torch.Tensor, y: torch.Tensor, residual: Optional[torch.Tensor] = None,
+                stream=None) -> None:
+    """y = x . w^T (+ residual); w is [out][in]."""
+    m, k = x.shape
+    n = w.shape[0]
+    if w.shape[1] != k or y.shape[0] != m or y.shape[1] != n:
+        raise KalmError(1, "kalm_linear", f"shapes x{tuple(x.shape)} w{tuple(w.shape)} y{tuple(y.shape)}")
+    call("kalm_linear", _p(x, torch.bfloat16), _ld(x), _p(w, torch.bfloat16), _ld(w),
+         _p(residual, torch.bfloat16), _ld(residual) if residual is not None else 0,
+         _p(y, torch.bfloat16), _ld(y), m, n, k, _stream(stream))
+
+
+def kalm_cross_kv_proj(pooled: torch.Tensor, w_kv: torch.Tensor, kv_cross: torch.Tensor, n_kv: int,
+                       head_dim: int = HEAD_DIM, stream=None) -> None:
+    """w_kv: [n_layers][2*n_kv*D][hidden]; kv_cross: [rows][n_layers*2*n_kv*D]."""
+    n_layers = w_kv.shape[0]
+    if not w_kv.is_contiguous() or not kv_cross.is_contiguous():
+        raise KalmError(1, "kalm_cross_kv_proj", "w_kv and kv_cross must be contiguous")
+    call("kalm_cross_kv_proj", _p(pooled, torch.bfloat16), _ld(pooled), pooled.shape[0], pooled.shape[1],
+         _p(w_kv, torch.bfloat16), n_layers, n_kv, head_dim, _p(kv_cross, torch.bfloat16), _stream(stream))
+
+
+def kalm_merged_attention(q: torch.Tensor, k_self: torch.Tensor, v_self: torch.Tensor, k_cross: torch.Tensor,
+                          v_cross: torch.Tensor, q_off: torch.Tensor, pool_off: torch.Tensor, max_q: int,
+                          n_q: int, n_kv: int, out: torch.Tensor, scale: Optional[float] = None,
+                          lse: Optional[torch.Tensor] = None, head_dim: int = HEAD_DIM, stream=None) -> None:
+    """2-D row views: q/out [rows][>= n_q*D], k/v self [rows][>= n_kv*D], k/v cross [pooled rows][>= n_kv*D]."""
+    if scale is None:
+        scale = head_dim ** -0.5
+    if _ld(k_self) != _ld(v_self) or _ld(k_cross) != _ld(v_cross):
+        raise KalmError(1, "kalm_merged_attention", "K and V views must share a row stride")
+    n_docs = q_off.numel() - 1
+    call("kalm_merged_attention", _p(q, torch.bfloat16), _ld(q), _p(k_self, torch.bfloat16),
+         _p(v_self, torch.bfloat16), _ld(k_self), _p(k_cross, torch.bfloat16), _p(v_cross, torch.bfloat16),
+         _ld(k_cross), _p(q_off, torch.int64), _p(pool_off, torch.int64), n_docs, int(max_q), q.shape[0],
+         k_cross.shape[0], n_q, n_kv, head_dim, float(scale), _p(out, torch.bfloat16), _ld(out),
+         _p(lse, torch.float32), _stream(stream))
+
+
+def kalm_yes_no_score(hidden: torch.Tensor, q_off: torch.Tensor, w_yes: torch.Tensor, w_no: torch.Tensor,
+                      yes: torch.Tensor, no: torch.Tensor, score: torch.Tensor,
+                      margin: Optional[torch.Tensor] = None, stream=None) -> None:
+    call("kalm_yes_no_score", _p(hidden, torch.bfloat16), _ld(hidden), _p(q_off, torch.int64), q_off.numel() - 1,
+         hidden.shape[1], _p(w_yes, torch.bfloat16), _p(w_no, torch.bfloat16), _p(yes, torch.float32),
+         _p(no, torch.float32), _p(margin, torch.float32), _p(score, torch.float32), _stream(stream))
+
+
+def kalm_broadcast_rows(src: torch.Tensor, q_off: torch.Tensor, dst: torch.Tensor, stream=None) -> None:
+    call("kalm_broadcast_rows", _p(src, torch.bfloat16), _ld(src), src.shape[0], src.shape[1],
+         _p(q_off, torch.int64), q_off.numel() - 1, _p(dst, torch.bfloat16), _ld(dst), _stream(stream))
+
+
+def kalm_selftest_wait_timeout(wait_ns: int, stream=None) -> None:
+    call("kalm_selftest_wait_timeout", int(wait_ns), _stream(stream))

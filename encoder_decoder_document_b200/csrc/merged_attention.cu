@@ -1,0 +1,432 @@
+// Step 3: merged self + cross attention for a ragged batch of documents.
+//
+// "KaLM-Reranker-V1-Nano - MLX (Apple Silicon)", "What this is": the decoder runs
+// a single scaled-dot-product attention whose keys and values are the
+// concatenation of its own (causal) self-attention K/V and the cross-attention
+// K/V of the document's cached pooled vectors.  One softmax covers both parts.
+//
+// Design (sm_100a), one CTA per (query tile, KV head, document):
+//   * 128 packed rows = (128 / G) decoder positions x G query heads of one KV
+//     head (GQA), so every K/V tile is fetched once for the G heads sharing it.
+//     The Q tile (128 x 256 bf16) is fetched once by a 3-D TMA box.
+//   * The KV loop walks the self segment (64-key tiles up to the tile's last
+//     position, causal mask inside) and then the cross segment (64-key tiles,
+//     only the ragged tail masked).  The concatenation exists only as this
+//     loop order; nothing is materialised in memory.
+//   * S = Q K^T and O += P V run on the tensor cores (tcgen05.mma, fp32
+//     accumulators in tensor memory: O = 256 columns, S double-buffered 2 x 64).
+//   * Softmax: one thread per row reads its S row with tcgen05.ld, keeps an
+//     online (running max / running sum) softmax in fp32 with exp2, and writes P
+//     as bf16 into a 128-byte-swizzled shared tile that is the A operand of PV.
+//     The running max is only raised when it grows by more than 2^8 in the
+//     exponent; otherwise P keeps the stale max (values stay below 256), so the
+//     O accumulator is rescaled in tensor memory only on such rare jumps.  The
+//     final O / l is exact either way.
+//   * Warp roles: warps 0-3 softmax + epilogue, warp 4 TMA producer, warp 5
+//     tensor-memory allocation and MMA issue.  K, V and P are double-buffered.
+#include <cmath>
+
+#include "kalm.h"
+#include "kalm_internal.h"
+#include "kalm_ptx.cuh"
+
+namespace kalm {
+namespace {
+
+constexpr int kD = 256;
+constexpr int kBM = 128;
+constexpr int kBKV = 64;
+constexpr int kThreads = 192;
+constexpr int kQBytes = kBM * kD * 2;          // 4 slabs of 128 rows x 128 B
+constexpr int kQSlab = kBM * 128;              // 16 KB
+constexpr int kKVBytes = kBKV * kD * 2;        // 4 slabs of 64 rows x 128 B
+constexpr int kKVSlab = kBKV * 128;            // 8 KB
+constexpr int kPBytes = kBM * kBKV * 2;        // 1 slab of 128 rows x 128 B
+constexpr int kSmem = 1024 + kQBytes + 2 * kKVBytes + 2 * kKVBytes + 2 * kPBytes + 256;
+constexpr uint32_t kTmemCols = 512;            // O: [0,256), S0: [256,320), S1: [320,384)
+constexpr uint32_t kIdescS = idesc_bf16_f32(kBM, kBKV, false, false);
+constexpr uint32_t kIdescPV = idesc_bf16_f32(kBM, kD, false, true);
+constexpr float kRescaleThreshold = 8.0f;      // log2 units
+
+struct AttnParams {
+  const int64_t* q_off;
+  const int64_t* pool_off;
+  __nv_bfloat16* out;
+  float* lse;
+  int64_t ldo;
+  int n_docs;
+  int n_q;
+  int n_kv;
+  int G;            // query heads per KV head
+  int P;            // decoder positions per tile = 128 / G
+  int tiles_per_doc;
+  float scale_log2;  // scale * log2(e)
+  uint64_t wait_ns;
+  uint32_t* err;
+};
+
+__global__ void __launch_bounds__(kThreads, 1)
+    merged_attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_ks,
+                            const __grid_constant__ CUtensorMap tm_vs, const __grid_constant__ CUtensorMap tm_kc,
+                            const __grid_constant__ CUtensorMap tm_vc, const AttnParams p) {
+  // ---- work item: heaviest query tiles (largest t) first
+  const int per_t = p.n_docs * p.n_kv;
+  const int t = p.tiles_per_doc - 1 - static_cast<int>(blockIdx.x) / per_t;
+  const int rem = static_cast<int>(blockIdx.x) % per_t;
+  const int g = rem % p.n_kv;
+  const int d = rem / p.n_kv;
+  const int64_t q0 = p.q_off[d];
+  const int Lq = static_cast<int>(p.q_off[d + 1] - q0);
+  const int64_t c0 = p.pool_off[d];
+  const int Nc = static_cast<int>(p.pool_off[d + 1] - c0);
+  const int pos0 = t * p.P;
+  if (pos0 >= Lq) return;  // uniform across the CTA, before any set-up
+  const int pos1 = min(pos0 + p.P, Lq);
+  const int n_self = (pos1 + kBKV - 1) / kBKV;
+  const int n_cross = (Nc + kBKV - 1) / kBKV;
+  const int nt = n_self + n_cross;
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sQ = smem;
+  uint8_t* sK = sQ + kQBytes;
+  uint8_t* sV = sK + 2 * kKVBytes;
+  uint8_t* sP = sV + 2 * kKVBytes;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sP + 2 * kPBytes);
+  uint64_t* bar_q = bars;
+  uint64_t* bar_k = bars + 1;   // [2]
+  uint64_t* bar_v = bars + 3;   // [2]
+  uint64_t* bar_s = bars + 5;   // [2]
+  uint64_t* bar_p = bars + 7;   // [2]
+  uint64_t* bar_pv = bars + 9;  // [2]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 11);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    mbar_init(bar_q, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&bar_k[i], 1);
+      mbar_init(&bar_v[i], 1);
+      mbar_init(&bar_s[i], 1);
+      mbar_init(&bar_p[i], 128);
+      mbar_init(&bar_pv[i], 1);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 5) {
+    tmem_alloc(tmem_slot, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 4) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      mbar_arrive_expect_tx(bar_q, kQBytes);
+      for (int j = 0; j < 4; ++j)
+        tma_load_3d(sQ + j * kQSlab, &tm_q, bar_q, j * 64, g * p.G, static_cast<int32_t>(q0 + pos0));
+      for (int j = 0; j < nt && !*abort_flag; ++j) {
+        const int s = j & 1;
+        const bool self = j < n_self;
+        const int32_t row = self ? static_cast<int32_t>(q0 + j * kBKV)
+                                 : static_cast<int32_t>(c0 + (j - n_self) * kBKV);
+        const CUtensorMap* mk = self ? &tm_ks : &tm_kc;
+        const CUtensorMap* mv = self ? &tm_vs : &tm_vc;
+        if (j >= 2 && !mbar_wait(&bar_s[s], ((j - 2) >> 1) & 1, p.wait_ns)) {
+          record_error(p.err, kErrTimeout | kSiteAttention);
+          *abort_flag = 1;
+          break;
+        }
+        mbar_arrive_expect_tx(&bar_k[s], kKVBytes);
+        for (int q = 0; q < 4; ++q)
+          tma_load_2d(sK + s * kKVBytes + q * kKVSlab, mk, &bar_k[s], g * kD + q * 64, row);
+        if (j >= 2 && !mbar_wait(&bar_pv[s], ((j - 2) >> 1) & 1, p.wait_ns)) {
+          record_error(p.err, kErrTimeout | kSiteAttention);
+          *abort_flag = 1;
+          break;
+        }
+        mbar_arrive_expect_tx(&bar_v[s], kKVBytes);
+        for (int q = 0; q < 4; ++q)
+          tma_load_2d(sV + s * kKVBytes + q * kKVSlab, mv, &bar_v[s], g * kD + q * 64, row);
+      }
+    }
+  } else if (warp == 5) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const uint32_t q_base = smem_u32(sQ), k_base = smem_u32(sK), v_base = smem_u32(sV), p_base = smem_u32(sP);
+      bool ok = mbar_wait(bar_q, 0, p.wait_ns);
+      auto issue_s = [&](int j) -> bool {
+        const int s = j & 1;
+        if (!mbar_wait(&bar_k[s], (j >> 1) & 1, p.wait_ns)) return false;
+        tc_fence_after();
+        const uint32_t d_s = tmem + 256u + static_cast<uint32_t>(s * kBKV);
+#pragma unroll
+        for (int kk = 0; kk < kD / 16; ++kk) {
+          const uint32_t off = static_cast<uint32_t>((kk & 3) * 32);  // 16-element step inside a swizzle row
+          const uint64_t ad = sdesc_sw128(q_base + (kk >> 2) * kQSlab + off, 16, 1024);
+          const uint64_t bd = sdesc_sw128(k_base + s * kKVBytes + (kk >> 2) * kKVSlab + off, 16, 1024);
+          umma_bf16_ss(d_s, ad, bd, kIdescS, kk != 0 ? 1u : 0u);
+        }
+        umma_commit(&bar_s[s]);
+        return true;
+      };
+      if (ok) ok = issue_s(0);
+      for (int j = 0; j < nt && ok && !*abort_flag; ++j) {
+        const int s = j & 1;
+        if (j + 1 < nt) {
+          ok = issue_s(j + 1);
+          if (!ok) break;
+        }
+        if (!mbar_wait(&bar_p[s], (j >> 1) & 1, p.wait_ns) || !mbar_wait(&bar_v[s], (j >> 1) & 1, p.wait_ns)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < kBKV / 16; ++kk) {
+          const uint64_t ad = sdesc_sw128(p_base + s * kPBytes + kk * 32, 16, 1024);
+          // V is MN-major: 64-column slabs kKVSlab apart (LBO), 8-key groups 1024 B apart (SBO)
+          const uint64_t bd = sdesc_sw128(v_base + s * kKVBytes + kk * 16 * 128, kKVSlab, 1024);
+          umma_bf16_ss(tmem, ad, bd, kIdescPV, (j | kk) != 0 ? 1u : 0u);
+        }
+        umma_commit(&bar_pv[s]);
+      }
+      if (!ok) {
+        record_error(p.err, kErrTimeout | kSiteAttention);
+        *abort_flag = 1;
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ softmax warps 0..3
+    const int r = warp * 32 + lane;          // packed row = TMEM lane
+    const int pos = pos0 + r / p.G;          // decoder position of this row
+    const int hh = r % p.G;                  // query head within the KV group
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+    float m_run = -INFINITY, l_run = 0.f;
+    bool ok = true;
+    for (int j = 0; j < nt; ++j) {
+      const int s = j & 1;
+      bool w = mbar_wait(&bar_s[s], (j >> 1) & 1, p.wait_ns);
+      if (!__all_sync(0xffffffffu, w) || *abort_flag) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      uint32_t sr[64];
+      tmem_ld32(lane_base + 256u + s * kBKV, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
+      tmem_ld32(lane_base + 256u + s * kBKV + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
+      tmem_ld_wait();
+      // visible keys of this tile: self keys k <= pos (and < pos1 rows exist), cross keys k < Nc
+      int n_vis;
+      if (j < n_self) {
+        n_vis = pos + 1 - j * kBKV;
+      } else {
+        n_vis = Nc - (j - n_self) * kBKV;
+      }
+      n_vis = max(0, min(kBKV, n_vis));
+      float x[64];
+      float mx = -INFINITY;
+#pragma unroll
+      for (int k = 0; k < 64; ++k) {
+        x[k] = k < n_vis ? __uint_as_float(sr[k]) * p.scale_log2 : -INFINITY;
+        mx = fmaxf(mx, x[k]);
+      }
+      float alpha = 1.f;
+      bool rescale = false;
+      if (j == 0) {
+        m_run = mx;  // every row sees self key 0, so mx is finite
+      } else if (mx > m_run + kRescaleThreshold) {
+        alpha = exp2f(m_run - mx);
+        m_run = mx;
+        rescale = true;
+      }
+      float sum = 0.f;
+      uint32_t pk[32];
+#pragma unroll
+      for (int k = 0; k < 64; k += 2) {
+        const float e0 = exp2f(x[k] - m_run);
+        const float e1 = exp2f(x[k + 1] - m_run);
+        sum += e0 + e1;
+        pk[k >> 1] = pack_bf16x2(e0, e1);
+      }
+      l_run = l_run * alpha + sum;
+      // P stage s is free once PV_{j-2} has completed
+      if (j >= 2) {
+        w = mbar_wait(&bar_pv[s], ((j - 2) >> 1) & 1, p.wait_ns);
+        if (!__all_sync(0xffffffffu, w)) {
+          ok = false;
+          break;
+        }
+      }
+      // 128-byte swizzled K-major row: 16-byte chunk c of row r sits at chunk c ^ (r & 7)
+      uint8_t* prow = sP + s * kPBytes + r * 128;
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        uint4 v;
+        v.x = pk[4 * c + 0];
+        v.y = pk[4 * c + 1];
+        v.z = pk[4 * c + 2];
+        v.w = pk[4 * c + 3];
+        *reinterpret_cast<uint4*>(prow + ((c ^ (r & 7)) << 4)) = v;
+      }
+      fence_proxy_async_smem();
+      if (__any_sync(0xffffffffu, rescale)) {
+        // O must hold the result of PV_{j-1} before it is rescaled in place
+        w = mbar_wait(&bar_pv[(j - 1) & 1], ((j - 1) >> 1) & 1, p.wait_ns);
+        if (!__all_sync(0xffffffffu, w)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+#pragma unroll 1
+        for (int c = 0; c < kD; c += 32) {
+          uint32_t o[32];
+          tmem_ld32(lane_base + c, o);
+          tmem_ld_wait();
+#pragma unroll
+          for (int k = 0; k < 32; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * alpha);
+          tmem_st32(lane_base + c, o);
+        }
+        tmem_st_wait();
+      }
+      tc_fence_before();
+      mbar_arrive(&bar_p[s]);
+    }
+    if (!ok) {
+      if (lane == 0) record_error(p.err, kErrTimeout | kSiteAttention);
+      *abort_flag = 1;
+    } else {
+      // ---- epilogue: O / l -> bf16
+      const int jl = nt - 1;
+      bool w = mbar_wait(&bar_pv[jl & 1], (jl >> 1) & 1, p.wait_ns);
+      if (!__all_sync(0xffffffffu, w)) {
+        if (lane == 0) record_error(p.err, kErrTimeout | kSiteAttention);
+        *abort_flag = 1;
+      } else {
+        tc_fence_after();
+        const float inv_l = 1.f / l_run;
+        const bool valid = pos < pos1;
+        const int head = g * p.G + hh;
+        __nv_bfloat16* orow = p.out + (q0 + pos) * p.ldo + static_cast<int64_t>(head) * kD;
+#pragma unroll 1
+        for (int c = 0; c < kD; c += 32) {
+          uint32_t o[32];
+          tmem_ld32(lane_base + c, o);
+          tmem_ld_wait();
+          if (valid) {
+            uint4* dst = reinterpret_cast<uint4*>(orow + c);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              uint4 v;
+              v.x = pack_bf16x2(__uint_as_float(o[8 * q + 0]) * inv_l, __uint_as_float(o[8 * q + 1]) * inv_l);
+              v.y = pack_bf16x2(__uint_as_float(o[8 * q + 2]) * inv_l, __uint_as_float(o[8 * q + 3]) * inv_l);
+              v.z = pack_bf16x2(__uint_as_float(o[8 * q + 4]) * inv_l, __uint_as_float(o[8 * q + 5]) * inv_l);
+              v.w = pack_bf16x2(__uint_as_float(o[8 * q + 6]) * inv_l, __uint_as_float(o[8 * q + 7]) * inv_l);
+              dst[q] = v;
+            }
+          }
+        }
+        if (valid && p.lse) {
+          // natural-log softmax denominator in scaled-logit units
+          p.lse[(q0 + pos) * p.n_q + head] = (m_run + log2f(l_run)) * 0.69314718055994531f;
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 5) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+}  // namespace
+
+kalm_status setup_attention_kernels() {
+  return check_cuda(cudaFuncSetAttribute(merged_attention_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem),
+                    "cudaFuncSetAttribute(merged_attention_kernel)");
+}
+
+}  // namespace kalm
+
+using namespace kalm;
+
+extern "C" kalm_status kalm_merged_attention(const kalm_bf16* q, int64_t ldq, const kalm_bf16* k_self,
+                                             const kalm_bf16* v_self, int64_t ld_self, const kalm_bf16* k_cross,
+                                             const kalm_bf16* v_cross, int64_t ld_cross, const int64_t* q_off,
+                                             const int64_t* pool_off, int32_t n_docs, int32_t max_q,
+                                             int64_t total_q, int64_t total_pool, int32_t n_q, int32_t n_kv,
+                                             int32_t head_dim, float scale, kalm_bf16* out, int64_t ldo, float* lse,
+                                             kalm_stream_t stream) {
+  kalm_status st = ensure_device(nullptr);
+  if (st != KALM_OK) return st;
+  if (head_dim != kD) return fail(KALM_ERR_UNSUPPORTED, "kalm_merged_attention: head_dim=%d (only 256)", head_dim);
+  if (n_docs < 0 || n_q <= 0 || n_kv <= 0 || n_q % n_kv || max_q < 0 || max_q > KALM_MAX_QUERY_TOKENS ||
+      total_q < 0 || total_pool < 0)
+    return fail(KALM_ERR_INVALID_ARG, "kalm_merged_attention: bad sizes (n_docs=%d n_q=%d n_kv=%d max_q=%d)", n_docs,
+                n_q, n_kv, max_q);
+  const int G = n_q / n_kv;
+  if (kBM % G) return fail(KALM_ERR_UNSUPPORTED, "kalm_merged_attention: n_q/n_kv=%d must divide 128", G);
+  if (!(scale > 0.f) || !std::isfinite(scale)) return fail(KALM_ERR_INVALID_ARG, "kalm_merged_attention: bad scale");
+  if (n_docs == 0 || max_q == 0 || total_q == 0) return KALM_OK;
+  if (!q || !k_self || !v_self || !out || !q_off || !pool_off || (total_pool > 0 && (!k_cross || !v_cross)))
+    return fail(KALM_ERR_INVALID_ARG, "kalm_merged_attention: NULL pointer");
+  if (ldq % 8 || ld_self % 8 || ld_cross % 8 || ldo % 8 || ldq < (int64_t)n_q * kD || ld_self < (int64_t)n_kv * kD ||
+      (total_pool > 0 && ld_cross < (int64_t)n_kv * kD) || ldo < (int64_t)n_q * kD)
+    return fail(KALM_ERR_INVALID_ARG, "kalm_merged_attention: strides must be multiples of 8 covering all heads");
+  if (!aligned16(q) || !aligned16(k_self) || !aligned16(v_self) || !aligned16(out) ||
+      (total_pool > 0 && (!aligned16(k_cross) || !aligned16(v_cross))))
+    return fail(KALM_ERR_INVALID_ARG, "kalm_merged_attention: bf16 pointers must be 16-byte aligned");
+  if (total_q > INT32_MAX - 1024 || total_pool > INT32_MAX - 1024)
+    return fail(KALM_ERR_INVALID_ARG, "kalm_merged_attention: too many rows");
+
+  CUtensorMap tq, tks, tvs, tkc, tvc;
+  {
+    const uint64_t dims[3] = {kD, static_cast<uint64_t>(n_q), static_cast<uint64_t>(total_q)};
+    const uint64_t strides[2] = {kD * 2, static_cast<uint64_t>(ldq) * 2};
+    const uint32_t box[3] = {64, static_cast<uint32_t>(G), static_cast<uint32_t>(kBM / G)};
+    if ((st = make_tmap_bf16(&tq, q, 3, dims, strides, box)) != KALM_OK) return st;
+  }
+  auto kv_map = [&](CUtensorMap* m, const kalm_bf16* base, int64_t ld, int64_t rows) -> kalm_status {
+    const uint64_t dims[2] = {static_cast<uint64_t>(n_kv) * kD, static_cast<uint64_t>(rows > 0 ? rows : 1)};
+    const uint64_t strides[1] = {static_cast<uint64_t>(ld) * 2};
+    const uint32_t box[2] = {64, kBKV};
+    return make_tmap_bf16(m, base, 2, dims, strides, box);
+  };
+  if ((st = kv_map(&tks, k_self, ld_self, total_q)) != KALM_OK) return st;
+  if ((st = kv_map(&tvs, v_self, ld_self, total_q)) != KALM_OK) return st;
+  // with no cross rows at all, the cross maps are never read; point them at the self tensors
+  if ((st = kv_map(&tkc, total_pool > 0 ? k_cross : k_self, total_pool > 0 ? ld_cross : ld_self,
+                   total_pool > 0 ? total_pool : total_q)) != KALM_OK)
+    return st;
+  if ((st = kv_map(&tvc, total_pool > 0 ? v_cross : v_self, total_pool > 0 ? ld_cross : ld_self,
+                   total_pool > 0 ? total_pool : total_q)) != KALM_OK)
+    return st;
+
+  AttnParams prm;
+  prm.q_off = q_off;
+  prm.pool_off = pool_off;
+  prm.out = reinterpret_cast<__nv_bfloat16*>(out);
+  prm.lse = lse;
+  prm.ldo = ldo;
+  prm.n_docs = n_docs;
+  prm.n_q = n_q;
+  prm.n_kv = n_kv;
+  prm.G = G;
+  prm.P = kBM / G;
+  prm.tiles_per_doc = (max_q + prm.P - 1) / prm.P;
+  prm.scale_log2 = scale * 1.4426950408889634f;
+  prm.wait_ns = kWaitNs;
+  prm.err = device_error_word();
+  const int64_t grid = static_cast<int64_t>(prm.tiles_per_doc) * n_docs * n_kv;
+  if (grid > INT32_MAX) return fail(KALM_ERR_INVALID_ARG, "kalm_merged_attention: grid too large");
+  merged_attention_kernel<<<static_cast<unsigned>(grid), kThreads, kSmem, static_cast<cudaStream_t>(stream)>>>(
+      tq, tks, tvs, tkc, tvc, prm);
+  return check_cuda(cudaGetLastError(), "launch merged_attention_kernel");
+}

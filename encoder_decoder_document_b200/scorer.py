@@ -1,0 +1,231 @@
+"""One query against a ragged batch of documents: the four scoring steps chained.
+
+``FBNLScorer`` owns the decoder weights (device, bf16) and reusable device
+buffers, and runs, on one stream:
+
+  kalm_ragged_offsets -> kalm_chunk_pool (document cache) -> kalm_cross_kv_proj
+  (all layers at once) -> kalm_broadcast_rows (the query's decoder input for
+  every document) -> per layer: kalm_linear (Q | K_self | V_self),
+  kalm_merged_attention, kalm_linear (output projection + residual) ->
+  kalm_yes_no_score.
+
+Python only sequences the calls and owns the buffers; every step runs in the
+CUDA kernels of libkalm.  ``capture()`` records the whole sequence in a CUDA
+graph so a query costs one graph launch.  ``rerank()`` is the user-facing call:
+host inputs in, the best-first list out ("KaLM-Reranker-V1-Nano - MLX",
+"Usage": rerank returns {index, relevance_score} entries, highest first;
+"KaLM-Reranker-V1-Small-Q4_K_M-GGUF", "Score a pair": larger margins rank first).
+"""
+from __future__ import annotations
+
+import dataclasses
+from typing import Optional
+
+import numpy as np
+import torch
+
+from . import (kalm_broadcast_rows, kalm_chunk_pool, kalm_cross_kv_proj, kalm_device_check, kalm_linear,
+               kalm_merged_attention, kalm_ragged_offsets, kalm_yes_no_score)
+
+HEAD_DIM = 256
+
+
+def bf16_from_bits(bits: np.ndarray, device="cuda") -> torch.Tensor:
+    """uint16 bf16 bit patterns (host) -> bf16 device tensor (bit-exact)."""
+    t = torch.from_numpy(np.ascontiguousarray(bits).view(np.int16))
+    return t.to(device).view(torch.bfloat16)
+
+
+@dataclasses.dataclass
+class DeviceWeights:
+    w_qkv: torch.Tensor       # [L][(n_q + 2 n_kv) D][H]
+    w_o: torch.Tensor         # [L][H][n_q D]
+    w_kv_cross: torch.Tensor  # [L][2 n_kv D][H]
+    w_yes: torch.Tensor       # [H]
+    w_no: torch.Tensor        # [H]
+
+    @classmethod
+    def from_bits(cls, w, device="cuda") -> "DeviceWeights":
+        return cls(bf16_from_bits(w.w_qkv, device), bf16_from_bits(w.w_o, device),
+                   bf16_from_bits(w.w_kv_cross, device), bf16_from_bits(w.w_yes, device),
+                   bf16_from_bits(w.w_no, device))
+
+
+class FBNLScorer:
+    def __init__(self, weights: DeviceWeights, n_q: int, n_kv: int, chunk: int = 4, head_dim: int = HEAD_DIM):
+        kalm_device_check()
+        self.w = weights
+        self.L, qkv_rows, self.H = weights.w_qkv.shape
+        self.n_q, self.n_kv, self.D, self.chunk = n_q, n_kv, head_dim, chunk
+        assert qkv_rows == (n_q + 2 * n_kv) * head_dim
+        self.scale = head_dim ** -0.5
+        self._shape = None
+        self.graph: Optional[torch.cuda.CUDAGraph] = None
+        # optional per-launch timing: (label, event) recorded after every entry-point call
+        self.marks: Optional[list] = None
+        self.launches = 0  # kernel launches issued by the last forward()
+
+    # ------------------------------------------------------------------ buffers
+    def prepare(self, n_docs: int, total_tokens: int, total_pooled: int, lq: int, device="cuda") -> None:
+        """Allocate the device buffers for one query shape (re-used across calls)."""
+        shape = (n_docs, total_tokens, total_pooled, lq)
+        if self._shape == shape:
+            return
+        self._shape = shape
+        self.graph = None
+        D, H, L = self.D, self.H, self.L
+        rows = n_docs * lq
+        kw = dict(device=device)
+        self.n_docs, self.total_tokens, self.total_pooled, self.lq = shape
+        self.enc = torch.empty(max(total_tokens, 1), H, dtype=torch.bfloat16, **kw)
+        self.doc_len = torch.empty(n_docs, dtype=torch.int32, **kw)
+        self.q_len = torch.full((n_docs,), lq, dtype=torch.int32, **kw)
+        self.x0 = torch.empty(lq, H, dtype=torch.bfloat16, **kw)
+        self.tok_off = torch.empty(n_docs + 1, dtype=torch.int64, **kw)
+        self.pool_off = torch.empty(n_docs + 1, dtype=torch.int64, **kw)
+        self.q_off = torch.empty(n_docs + 1, dtype=torch.int64, **kw)
+        self.pooled = torch.empty(max(total_pooled, 1), H, dtype=torch.bfloat16, **kw)
+        self.kv_cross = torch.empty(max(total_pooled, 1), L * 2 * self.n_kv * D, dtype=torch.bfloat16, **kw)
+        self.qkv = torch.empty(rows, (self.n_q + 2 * self.n_kv) * D, dtype=torch.bfloat16, **kw)
+        self.o = torch.empty(rows, self.n_q * D, dtype=torch.bfloat16, **kw)
+        self.x = torch.empty(rows, H, dtype=torch.bfloat16, **kw)
+        self.yes = torch.empty(n_docs, dtype=torch.float32, **kw)
+        self.no = torch.empty(n_docs, dtype=torch.float32, **kw)
+        self.margin = torch.empty(n_docs, dtype=torch.float32, **kw)
+        self.score = torch.empty(n_docs, dtype=torch.float32, **kw)
+        self.result = torch.empty(4, n_docs, dtype=torch.float32, **kw)
+
+    # ------------------------------------------------------------------ steps
+    def _mark(self, label: str) -> None:
+        self.launches += 1
+        if self.marks is not None:
+            ev = torch.cuda.Event(enable_timing=True, external=True)
+            ev.record()
+            self.marks.append((label, ev))
+
+    def pool(self) -> None:
+        kalm_ragged_offsets(self.doc_len, self.tok_off, self.pool_off, self.chunk)
+        self._mark("offsets")
+        kalm_ragged_offsets(self.q_len, self.q_off, None, 1)
+        self._mark("offsets")
+        kalm_chunk_pool(self.enc, self.tok_off, self.doc_len, self.pooled, self.pool_off, self.total_pooled,
+                        self.chunk)
+        self._mark("chunk_pool")
+
+    def cross_kv(self) -> None:
+        kalm_cross_kv_proj(self.pooled[: self.total_pooled], self.w.w_kv_cross, self.kv_cross[: self.total_pooled],
+                           self.n_kv, self.D)
+        self._mark("cross_kv_proj")
+
+    def cross_views(self, l: int):
+        w = self.n_kv * self.D
+        kc = self.kv_cross[:, (2 * l) * w:(2 * l + 1) * w]
+        vc = self.kv_cross[:, (2 * l + 1) * w:(2 * l + 2) * w]
+        return kc, vc
+
+    def qkv_views(self):
+        D, nq, nkv = self.D, self.n_q, self.n_kv
+        return (self.qkv[:, : nq * D], self.qkv[:, nq * D:(nq + nkv) * D], self.qkv[:, (nq + nkv) * D:])
+
+    def layer(self, l: int) -> None:
+        kalm_linear(self.x, self.w.w_qkv[l], self.qkv)
+        self._mark("qkv_proj")
+        q, ks, vs = self.qkv_views()
+        kc, vc = self.cross_views(l)
+        kalm_merged_attention(q, ks, vs, kc, vc, self.q_off, self.pool_off, self.lq, self.n_q, self.n_kv, self.o,
+                              self.scale)
+        self._mark("merged_attention")
+        kalm_linear(self.o, self.w.w_o[l], self.x, residual=self.x)
+        self._mark("o_proj")
+
+    def readout(self) -> None:
+        kalm_yes_no_score(self.x, self.q_off, self.w.w_yes, self.w.w_no, self.yes, self.no, self.score,
+                          self.margin)
+        self._mark("yes_no_score")
+
+    def forward(self) -> None:
+        """All steps on the current stream, from the inputs in self.enc / doc_len / x0."""
+        self.launches = 0
+        if self.marks is not None:
+            self._mark("start")
+            self.launches = 0
+        self.pool()
+        self.cross_kv()
+        kalm_broadcast_rows(self.x0, self.q_off, self.x)
+        self._mark("broadcast")
+        for l in range(self.L):
+            self.layer(l)
+        self.readout()
+
+    def capture(self, instrument: bool = False) -> None:
+        """Record forward() as a CUDA graph (buffers must stay allocated).
+
+        With ``instrument`` an external timing event is recorded after every
+        launch inside the graph, so each replay yields per-kernel durations
+        (``kernel_times()``)."""
+        s = torch.cuda.Stream()
+        s.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(s):
+            self.forward()  # warm-up: one-time device set-up happens outside capture
+        torch.cuda.current_stream().wait_stream(s)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        self.marks = [] if instrument else None
+        with torch.cuda.graph(g):
+            self.forward()
+        self.graph = g
+
+    def kernel_times(self) -> dict:
+        """{label: [ms per launch, ...]} of the last replay of an instrumented graph."""
+        out: dict = {}
+        if not self.marks:
+            return out
+        for (_, a), (label, b) in zip(self.marks[:-1], self.marks[1:]):
+            out.setdefault(label, []).append(a.elapsed_time(b))
+        return out
+
+    def run(self) -> None:
+        if self.graph is not None:
+            self.graph.replay()
+        else:
+            self.forward()
+
+    # ------------------------------------------------------------------ user API
+    def load_inputs(self, enc_host: torch.Tensor, doc_len_host: torch.Tensor, x0_host: torch.Tensor) -> None:
+        """Host -> device copies of one query's inputs (pinned host tensors copy asynchronously)."""
+        self.enc[: enc_host.shape[0]].copy_(enc_host, non_blocking=True)
+        self.doc_len.copy_(doc_len_host, non_blocking=True)
+        self.x0.copy_(x0_host, non_blocking=True)
+
+    def scores_to_host(self, out: Optional[torch.Tensor] = None) -> torch.Tensor:
+        """Device -> host copy of (yes, no, margin, score) as a [4][n_docs] fp32 tensor."""
+        torch.stack([self.yes, self.no, self.margin, self.score], out=self.result)
+        if out is None:
+            return self.result.cpu()
+        out.copy_(self.result, non_blocking=True)
+        return out
+
+    def rerank(self, x0: np.ndarray, enc: np.ndarray, doc_len: np.ndarray, top_n: Optional[int] = None):
+        """Score one query's documents and return [{index, relevance_score}] best first.
+
+        x0: bf16 bits [lq][H] (decoder input of the query); enc: bf16 bits
+        [sum(doc_len)][H] (packed encoder states); doc_len: int [n_docs]."""
+        doc_len = np.asarray(doc_len, dtype=np.int32)
+        n = int(doc_len.shape[0])
+        total_tokens = int(doc_len.sum())
+        total_pooled = int(((doc_len.astype(np.int64) + self.chunk - 1) // self.chunk).sum())
+        self.prepare(n, total_tokens, total_pooled, int(x0.shape[0]))
+        self.load_inputs(torch.from_numpy(np.ascontiguousarray(enc).view(np.int16)).view(torch.bfloat16),
+                         torch.from_numpy(doc_len), torch.from_numpy(np.ascontiguousarray(x0).view(np.int16))
+                         .view(torch.bfloat16))
+        self.run()
+        res = self.scores_to_host().numpy()
+        return rank(res[2], res[3], top_n)
+
+
+def rank(margin: np.ndarray, score: np.ndarray, top_n: Optional[int] = None):
+    """Best-first order: larger margin first, ties broken by the lower index."""
+    order = sorted(range(len(margin)), key=lambda i: (-float(margin[i]), i))
+    if top_n is not None:
+        order = order[:top_n]
+    return [{"index": i, "relevance_score": float(score[i])} for i in order]

@@ -1,0 +1,229 @@
+/*
+ * kalm.h - C ABI of the KaLM-Reranker-V1 "fast but not late interaction" (FBNL)
+ * scoring hot path on NVIDIA B200 (sm_100a).
+ *
+ * The path has four steps, each an entry point below:
+ *   1. kalm_chunk_pool        masked-mean chunk pooling of cached passage encoder
+ *                             states into the document cache;
+ *   2. kalm_cross_kv_proj     cross-attention K/V projection of the pooled vectors
+ *                             (kalm_linear is the same GEMM for the decoder's
+ *                             Q/K/V and output projections);
+ *   3. kalm_merged_attention  one softmax over [causal self K/V ; cross K/V];
+ *   4. kalm_yes_no_score      final-position yes/no readout, score = sigmoid(yes - no).
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * - All tensor pointers are DEVICE pointers owned by the caller; the library
+ *   allocates no device memory on these calls.  Host-side arguments are sizes,
+ *   strides, flags and the stream.
+ * - bf16 tensors are raw IEEE bfloat16 bit patterns (kalm_bf16).  Strides ("ld",
+ *   leading dimension) are in ELEMENTS between consecutive rows; every bf16
+ *   pointer must be 16-byte aligned and every bf16 row stride a multiple of 8.
+ * - Every call is asynchronous on `stream` (a cudaStream_t; NULL = the legacy
+ *   default stream).  Argument errors are detected on the host and returned
+ *   synchronously; nothing is launched in that case.
+ * - Errors found on the device (a bounded wait that expired, an out-of-range
+ *   length) are recorded in a per-device error word that
+ *   kalm_check_device_errors() reads after synchronising the stream.  Kernels
+ *   never trap.
+ * - There is no CPU fallback: without an sm_100 device every call returns
+ *   KALM_ERR_NO_DEVICE (the pages' "--require-gpu" rule: a missing GPU is an
+ *   explicit error, never a silent fallback).
+ *
+ * Ragged layout.  Documents are packed one after another.  For n documents:
+ *   tok_off[n+1]   exclusive prefix sum of the encoder lengths len[d];
+ *   pool_off[n+1]  exclusive prefix sum of Nc[d] = ceil(len[d] / chunk);
+ *   q_off[n+1]     exclusive prefix sum of the decoder lengths Lq[d].
+ * These are int64 device arrays; kalm_ragged_offsets() computes the first two.
+ */
+#ifndef KALM_H_
+#define KALM_H_
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef uint16_t kalm_bf16;   /* bfloat16 bit pattern */
+typedef void* kalm_stream_t;  /* cudaStream_t */
+
+typedef enum kalm_status {
+  KALM_OK = 0,
+  KALM_ERR_INVALID_ARG = 1,   /* null pointer, bad size/stride/alignment, limit exceeded */
+  KALM_ERR_UNSUPPORTED = 2,   /* valid but not implemented (e.g. head_dim != 256) */
+  KALM_ERR_NO_DEVICE = 3,     /* no sm_100 device current; never falls back to the CPU */
+  KALM_ERR_CUDA = 4,          /* a CUDA runtime call failed (see kalm_last_error) */
+  KALM_ERR_TIMEOUT = 5,       /* a device-side bounded wait expired (device error word) */
+  KALM_ERR_DEVICE_ARG = 6     /* a kernel found an invalid value in device data */
+} kalm_status;
+
+/* Limits of the pages' runtime contract ("KaLM-Reranker-V1-Small-Q4_K_M-GGUF",
+ * "Runtime boundaries"; "KaLM-Reranker-V1-Large-Q8_0-GGUF", "Frozen inference
+ * contract"): at most 1,024 encoder tokens per passage, a query budget of 512
+ * tokens, encoder chunk size 4. */
+#define KALM_MAX_DOC_TOKENS 1024
+#define KALM_MAX_QUERY_TOKENS 512
+#define KALM_DEFAULT_CHUNK 4
+#define KALM_HEAD_DIM 256
+
+/* Version of this ABI (major * 100 + minor). */
+int kalm_version(void);
+
+/* Human-readable name of a status code (static string). */
+const char* kalm_status_string(int status);
+
+/* Detail of the last error returned on the calling host thread (static,
+ * thread-local buffer; empty string if none). */
+const char* kalm_last_error(void);
+
+/* KALM_OK if the current CUDA device is an sm_100 part, else KALM_ERR_NO_DEVICE. */
+kalm_status kalm_device_check(void);
+
+/* Synchronise `stream`, read and clear the current device's error word.
+ * *word_out (nullable) receives the raw word: bit 0 = a bounded wait expired,
+ * bit 1 = invalid device data (e.g. a length above its limit); bits 8..15 name
+ * the kernel (1 pool, 2 linear, 3 attention, 4 readout, 5 offsets, 6 self-test).
+ * Returns KALM_ERR_TIMEOUT, KALM_ERR_DEVICE_ARG or KALM_OK. */
+kalm_status kalm_check_device_errors(kalm_stream_t stream, uint32_t* word_out);
+
+/* Ragged offsets: tok_off[d] = sum_{e<d} len[e], pool_off[d] = sum_{e<d}
+ * ceil(len[e] / chunk), for d = 0..n (both arrays hold n+1 int64 values).
+ * len: int32 device array of n values in [0, KALM_MAX_DOC_TOKENS]; a value out
+ * of range is clamped to the range and flagged in the device error word.
+ * n >= 0, chunk >= 1.  Either output may be NULL. */
+kalm_status kalm_ragged_offsets(const int32_t* len, int32_t n, int32_t chunk,
+                                int64_t* tok_off, int64_t* pool_off,
+                                kalm_stream_t stream);
+
+/* Step 1 - chunk pooling into the document cache.
+ * "KaLM-Reranker-V1-Nano - MLX (Apple Silicon)", "What this is": each passage is
+ * encoded once and chunk-pooled (chunk size 4 tokens, masked mean per chunk)
+ * into a small set of cached document vectors; "KaLM-Reranker-V1-Large-Q8_0-
+ * GGUF", "Frozen inference contract": right padding, masked mean pooling over
+ * consecutive groups of 4 tokens.
+ *
+ *   pooled[pool_off[d] + c][:] = mean of enc[tok_off[d] + t][:] over
+ *       t = chunk*c .. min(chunk*c + chunk, len[d]) - 1
+ * i.e. a partial last group is averaged over its valid tokens only; groups
+ * start at token 0; no vector is emitted for a group with no valid token.
+ * Accumulation in fp32, one rounding to bf16 (nearest even) per output.
+ *
+ * enc     [rows][enc_ld] bf16; document d starts at row tok_off[d] (packed or
+ *         padded layouts both work; rows past len[d] are never read)
+ * tok_off int64[n_docs] (entries beyond n_docs are not read)
+ * len     int32[n_docs], each in [0, KALM_MAX_DOC_TOKENS]
+ * pooled  [total_pooled][pooled_ld] bf16, written for rows pool_off[d] ..
+ *         pool_off[d] + ceil(len[d]/chunk) - 1
+ * pool_off int64[n_docs + 1], must equal the prefix sums of ceil(len/chunk);
+ *         total_pooled = pool_off[n_docs] (host-known, sizes the launch)
+ * hidden % 8 == 0; 1 <= chunk <= 64. */
+kalm_status kalm_chunk_pool(const kalm_bf16* enc, int64_t enc_ld, const int64_t* tok_off,
+                            const int32_t* len, int32_t n_docs, int32_t hidden,
+                            int32_t chunk, kalm_bf16* pooled, int64_t pooled_ld,
+                            const int64_t* pool_off, int64_t total_pooled,
+                            kalm_stream_t stream);
+
+/* Dense projection y = x . w^T (+ residual), bf16 in, fp32 accumulate, bf16 out.
+ * The tcgen05 (5th-generation tensor core) GEMM behind steps 2 and the decoder
+ * projections.
+ *
+ * x        [m][ldx] bf16 (m rows of k values)
+ * w        [n][ldw] bf16, the nn.Linear layout [out][in]
+ * residual [m][ldr] bf16 or NULL; added before the single rounding to bf16.
+ *          It may alias y (same pointer and stride): each element is read
+ *          before it is written by the same thread.
+ * y        [m][ldy] bf16
+ * Requirements: m >= 0, n % 32 == 0, k % 8 == 0, k >= 8. */
+kalm_status kalm_linear(const kalm_bf16* x, int64_t ldx, const kalm_bf16* w, int64_t ldw,
+                        const kalm_bf16* residual, int64_t ldr, kalm_bf16* y, int64_t ldy,
+                        int64_t m, int32_t n, int32_t k, kalm_stream_t stream);
+
+/* Step 2 - cross-attention K/V projection of the cached pooled vectors for
+ * n_layers decoder layers at once.
+ * "KaLM-Reranker-V1-Nano - MLX", "What this is": the cross-attention KV is
+ * computed over the cached passage encodings.  Reading: no bias, norm or
+ * rotary embedding on the cross K/V (the pages name none).
+ *
+ * pooled   [total_pooled][pooled_ld] bf16 (the document cache)
+ * w_kv     [n_layers][2][n_kv][head_dim][hidden] bf16 (per layer: cross K rows,
+ *          then cross V rows, nn.Linear layout)
+ * kv_cross [total_pooled][n_layers][2][n_kv][head_dim] bf16: for pooled row r,
+ *          layer l, cross K of KV head g starts at element
+ *          r*ld + (l*2 + 0)*n_kv*head_dim + g*head_dim and cross V at
+ *          r*ld + (l*2 + 1)*n_kv*head_dim + g*head_dim, ld = n_layers*2*n_kv*head_dim. */
+kalm_status kalm_cross_kv_proj(const kalm_bf16* pooled, int64_t pooled_ld, int64_t total_pooled,
+                               int32_t hidden, const kalm_bf16* w_kv, int32_t n_layers,
+                               int32_t n_kv, int32_t head_dim, kalm_bf16* kv_cross,
+                               kalm_stream_t stream);
+
+/* Step 3 - merged self + cross attention for a ragged batch of documents.
+ * "KaLM-Reranker-V1-Nano - MLX", "What this is": a single scaled-dot-product
+ * attention that concatenates the decoder's self-attention K/V with the
+ * cross-attention K/V of the document's cached vectors.
+ *
+ * For document d, query head h (KV head g = h / (n_q / n_kv)) and decoder row i
+ * (0 <= i < Lq[d]):
+ *   out[i, h] = sum_j softmax_j(scale * q[i,h] . key_j) value_j over
+ *   j in {self rows 0..i} U {cross rows 0..Nc[d]-1}
+ * one softmax over both segments (causal self part, diagonal included; cross
+ * part unmasked).  The concatenation is never materialised.
+ *
+ * q       [q_off[n_docs]][ldq] bf16; row q_off[d]+i, head h at element h*head_dim
+ * k_self, v_self  [q_off[n_docs]][ld_self] bf16; KV head g at element g*head_dim
+ * k_cross, v_cross [pool_off[n_docs]][ld_cross] bf16; KV head g at g*head_dim
+ * q_off   int64[n_docs+1] (decoder rows of document d: q_off[d] .. q_off[d+1]-1)
+ * pool_off int64[n_docs+1] (cross rows of document d: pool_off[d] .. pool_off[d+1]-1)
+ * max_q   host upper bound of Lq[d] (<= KALM_MAX_QUERY_TOKENS); sizes the grid
+ * total_q = q_off[n_docs], total_pool = pool_off[n_docs] (host-known; bound the
+ *         tensor views)
+ * scale   logit scale (1/sqrt(head_dim) for the standard attention)
+ * out     [total_q][ldo] bf16, head h at element h*head_dim
+ * lse     fp32 [total_q][n_q] or NULL: natural log of each row's softmax
+ *         denominator, in scaled-logit units.
+ * Requirements: head_dim == 256; n_q % n_kv == 0; (n_q / n_kv) divides 128;
+ * strides multiples of 8. */
+kalm_status kalm_merged_attention(const kalm_bf16* q, int64_t ldq,
+                                  const kalm_bf16* k_self, const kalm_bf16* v_self, int64_t ld_self,
+                                  const kalm_bf16* k_cross, const kalm_bf16* v_cross, int64_t ld_cross,
+                                  const int64_t* q_off, const int64_t* pool_off, int32_t n_docs,
+                                  int32_t max_q, int64_t total_q, int64_t total_pool,
+                                  int32_t n_q, int32_t n_kv, int32_t head_dim, float scale,
+                                  kalm_bf16* out, int64_t ldo, float* lse,
+                                  kalm_stream_t stream);
+
+/* Step 4 - yes/no readout at each document's final decoder position.
+ * "What this is": score = softmax([logit_yes, logit_no])[yes] at the final
+ * position; "Score a pair" / "Frozen inference contract": margin = yes - no,
+ * score = sigmoid(margin) (the same number).
+ *
+ * hidden  [q_off[n_docs]][ldh] bf16; document d's final row is q_off[d+1]-1
+ * w_yes, w_no  [hidden_dim] bf16 (the two LM-head rows)
+ * yes, no, score  fp32[n_docs]; margin fp32[n_docs] or NULL.  Documents with
+ * no decoder rows get yes = no = margin = 0, score = 0.5.
+ * Scores come back in input order. */
+kalm_status kalm_yes_no_score(const kalm_bf16* hidden, int64_t ldh, const int64_t* q_off,
+                              int32_t n_docs, int32_t hidden_dim,
+                              const kalm_bf16* w_yes, const kalm_bf16* w_no,
+                              float* yes, float* no, float* margin, float* score,
+                              kalm_stream_t stream);
+
+/* Copy rows of a shared [rows][ld_src] bf16 block into every document's slot:
+ * dst[q_off[d] + i] = src[i] for i < q_off[d+1]-q_off[d] (<= rows).  Used to
+ * start every document's decoder stream from the query's common input
+ * (the decoder reads the same instruction + query for each passage). */
+kalm_status kalm_broadcast_rows(const kalm_bf16* src, int64_t ld_src, int32_t rows,
+                                int32_t width, const int64_t* q_off, int32_t n_docs,
+                                kalm_bf16* dst, int64_t ld_dst, kalm_stream_t stream);
+
+/* Failure-detection self-test: one CTA waits on a shared-memory barrier that
+ * nothing completes, with a bound of `wait_ns` nanoseconds; on expiry it
+ * records a timeout in the device error word and returns.  Lets tests check
+ * the bounded-wait path without faulting or hanging the GPU. */
+kalm_status kalm_selftest_wait_timeout(uint64_t wait_ns, kalm_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif  /* KALM_H_ */

@@ -1,0 +1,409 @@
+"""Parity of the CUDA path (through the C ABI) with the fp64 oracle.
+
+Tolerances (stated for the scoring path): pooled vectors within 1e-2 abs;
+attention outputs within 2e-2 max abs and 5e-3 mean abs; scores within 1e-3
+abs; ranking identical wherever the oracle's score gap exceeds 1e-2.  The
+projections, which the tolerances do not name, are held to one bf16 rounding
+step: fp32 accumulation differs from fp64 by far less than half a bf16 ulp, so
+an output may only land on the neighbouring bf16 value.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synthetic
+from tests.gpu_util import f64_to_dev, from_dev, i32, i64, rand_bf16, to_dev
+
+pytestmark = pytest.mark.gpu
+
+POOL_TOL = 1e-2
+ATTN_MAX_TOL, ATTN_MEAN_TOL = 2e-2, 5e-3
+SCORE_TOL = 1e-3
+RANK_GAP = 1e-2
+
+
+@pytest.fixture(scope="module")
+def kalm():
+    import encoder_decoder_document_b200 as k
+    from encoder_decoder_document_b200 import _build
+    _build.build()
+    k.kalm_device_check()
+    yield k
+    k.kalm_check_device_errors()
+
+
+# ---------------------------------------------------------------------------
+# offsets
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("n", [1, 7, 100, 1024, 3001])
+def test_ragged_offsets(kalm, n):
+    rng = np.random.default_rng(n)
+    lens = rng.integers(0, 1025, n).astype(np.int32)
+    lens[: min(n, 4)] = [0, 1, 1024, 3][: min(n, 4)]
+    tok = torch.empty(n + 1, dtype=torch.int64, device="cuda")
+    pool = torch.empty(n + 1, dtype=torch.int64, device="cuda")
+    kalm.kalm_ragged_offsets(i32(lens), tok, pool, 4)
+    want_t = np.concatenate([[0], np.cumsum(lens.astype(np.int64))])
+    want_p = np.concatenate([[0], np.cumsum(oracle.pooled_counts(lens))])
+    np.testing.assert_array_equal(tok.cpu().numpy(), want_t)
+    np.testing.assert_array_equal(pool.cpu().numpy(), want_p)
+    kalm.kalm_check_device_errors()
+
+
+# ---------------------------------------------------------------------------
+# step 1: chunk pooling
+# ---------------------------------------------------------------------------
+def _run_pool(kalm, enc_bits, tok_off, lens, H, chunk=4, ld=None):
+    lens = np.asarray(lens, np.int32)
+    pool_off = np.concatenate([[0], np.cumsum(oracle.pooled_counts(lens, chunk))]).astype(np.int64)
+    total = int(pool_off[-1])
+    enc = to_dev(enc_bits)
+    if ld is not None:  # strided rows: copy into a wider buffer and pass a view
+        wide = torch.zeros(enc.shape[0], ld, dtype=torch.bfloat16, device="cuda")
+        wide[:, :H] = enc
+        enc = wide[:, :H]
+    pooled = torch.full((max(total, 1), H), float("nan"), dtype=torch.bfloat16, device="cuda")
+    kalm.kalm_chunk_pool(enc, i64(tok_off), i32(lens), pooled, i64(pool_off), total, chunk)
+    kalm.kalm_check_device_errors()
+    return from_dev(pooled[:total]), pool_off
+
+
+@pytest.mark.parametrize("name", ["tiny", "nano", "large"])
+def test_chunk_pool_configs(kalm, name):
+    q = synthetic.make_query(name, with_weights=False)
+    got, off = _run_pool(kalm, q.enc, q.tok_off[:-1], q.doc_len, q.hidden)
+    want, off_o = oracle.chunk_pool(oracle.bf16_bits_to_f64(q.enc), q.tok_off, q.doc_len, 4)
+    np.testing.assert_array_equal(off, off_o)
+    d = np.abs(got - want)
+    assert d.max() <= POOL_TOL
+    assert (d == 0).mean() > 0.99  # only rare rounding-boundary ties differ
+
+
+def test_chunk_pool_edge_lengths_padded_and_strided(kalm):
+    rng = np.random.default_rng(3)
+    H = 72
+    lens = np.array([0, 1, 2, 3, 4, 5, 7, 8, 9, 1023, 1024, 0, 13], np.int32)
+    Lmax = 1024
+    # padded layout: document d starts at row d * Lmax; padding rows are NaN-free garbage
+    enc = rand_bf16(rng, (len(lens) * Lmax, H))
+    tok = np.arange(len(lens), dtype=np.int64) * Lmax
+    got, _ = _run_pool(kalm, oracle.f64_to_bf16_bits(enc), tok, lens, H, ld=H + 40)
+    want, _ = oracle.chunk_pool(enc, tok, lens, 4)
+    assert np.abs(got - want).max() <= POOL_TOL
+    # chunk 1 is the identity; a chunk of 3 exercises the generic path
+    for chunk in (1, 3):
+        got, _ = _run_pool(kalm, oracle.f64_to_bf16_bits(enc), tok, lens, H, chunk=chunk)
+        want, _ = oracle.chunk_pool(enc, tok, lens, chunk)
+        assert np.abs(got - want).max() <= POOL_TOL
+        if chunk == 1:
+            np.testing.assert_array_equal(got, want)
+
+
+# ---------------------------------------------------------------------------
+# step 2: projections
+# ---------------------------------------------------------------------------
+def _one_step(got, want):
+    """Every output equals the oracle's bf16 value or its neighbour (one rounding step)."""
+    tol = np.abs(want) * 2.0 ** -7 + 1e-30
+    bad = np.abs(got - want) > tol
+    assert not bad.any(), f"{bad.sum()} outputs beyond one bf16 step; worst {np.abs(got - want).max():.3e}"
+    assert (got == want).mean() > 0.97
+
+
+@pytest.mark.parametrize("m,n,k,res", [
+    (1, 32, 8, False), (127, 64, 40, False), (300, 640, 640, False), (257, 1536, 640, True),
+    (1000, 512, 1152, True), (129, 2560, 72, False), (4096, 256, 2560, True)])
+def test_linear(kalm, m, n, k, res):
+    rng = np.random.default_rng(m * 7 + n + k)
+    x = rand_bf16(rng, (m, k))
+    w = rand_bf16(rng, (n, k), 0.02)
+    r = rand_bf16(rng, (m, n)) if res else None
+    y = torch.full((m, n), float("nan"), dtype=torch.bfloat16, device="cuda")
+    kalm.kalm_linear(f64_to_dev(x), f64_to_dev(w), y, residual=f64_to_dev(r) if res else None)
+    kalm.kalm_check_device_errors()
+    _one_step(from_dev(y), oracle.linear(x, w, residual=r))
+
+
+def test_linear_in_place_residual_and_strided(kalm):
+    rng = np.random.default_rng(21)
+    m, n, k = 200, 640, 1024
+    x = rand_bf16(rng, (m, k))
+    w = rand_bf16(rng, (n, k), 0.02)
+    r = rand_bf16(rng, (m, n))
+    buf = torch.zeros(m, n + 64, dtype=torch.bfloat16, device="cuda")
+    buf[:, :n] = f64_to_dev(r)
+    view = buf[:, :n]
+    kalm.kalm_linear(f64_to_dev(x), f64_to_dev(w), view, residual=view)
+    kalm.kalm_check_device_errors()
+    _one_step(from_dev(view), oracle.linear(x, w, residual=r))
+    assert float(buf[:, n:].abs().max()) == 0.0  # nothing written past the row width
+
+
+def test_cross_kv_proj_layout(kalm):
+    rng = np.random.default_rng(22)
+    L, n_kv, D, H, rows = 3, 2, 256, 640, 333
+    p = rand_bf16(rng, (rows, H))
+    w = rand_bf16(rng, (L, 2 * n_kv * D, H), 0.02)
+    kv = torch.empty(rows, L * 2 * n_kv * D, dtype=torch.bfloat16, device="cuda")
+    kalm.kalm_cross_kv_proj(f64_to_dev(p), f64_to_dev(w), kv, n_kv)
+    kalm.kalm_check_device_errors()
+    got = from_dev(kv).reshape(rows, L, 2, n_kv, D)
+    for l in range(L):
+        want = oracle.linear(p, w[l]).reshape(rows, 2, n_kv, D)
+        _one_step(got[:, l], want)
+
+
+# ---------------------------------------------------------------------------
+# step 3: merged attention
+# ---------------------------------------------------------------------------
+def _attn_arrays(rng, lq, nc, n_q, n_kv, q_std=0.5, k_std=0.5, kc_mult=1.0):
+    D = 256
+    lq = np.asarray(lq, np.int64)
+    nc = np.asarray(nc, np.int64)
+    q_off = np.concatenate([[0], np.cumsum(lq)])
+    p_off = np.concatenate([[0], np.cumsum(nc)])
+    R, C = int(q_off[-1]), int(p_off[-1])
+    return dict(q=rand_bf16(rng, (R, n_q, D), q_std), ks=rand_bf16(rng, (R, n_kv, D), k_std),
+                vs=rand_bf16(rng, (R, n_kv, D)), kc=rand_bf16(rng, (C, n_kv, D), k_std * kc_mult),
+                vc=rand_bf16(rng, (C, n_kv, D)), q_off=q_off, p_off=p_off, n_q=n_q, n_kv=n_kv)
+
+
+def _attn_run(kalm, a, p_off=None, scale=1.0 / 16):
+    """Run the kernel on fused row layouts as the scorer uses them: [q | k | v] and [k_cross | v_cross]."""
+    D, n_q, n_kv = 256, a["n_q"], a["n_kv"]
+    q_off = a["q_off"]
+    p_off = a["p_off"] if p_off is None else p_off
+    R, C = int(q_off[-1]), max(int(a["p_off"][-1]), 1)
+    kc = a["kc"] if a["kc"].shape[0] else np.zeros((1, n_kv, D))
+    vc = a["vc"] if a["vc"].shape[0] else np.zeros((1, n_kv, D))
+    qkv = torch.cat([f64_to_dev(a["q"].reshape(R, -1)), f64_to_dev(a["ks"].reshape(R, -1)),
+                     f64_to_dev(a["vs"].reshape(R, -1))], 1)
+    kvc = torch.cat([f64_to_dev(kc.reshape(C, -1)), f64_to_dev(vc.reshape(C, -1))], 1)
+    w = n_kv * D
+    out = torch.full((R, n_q * D), float("nan"), dtype=torch.bfloat16, device="cuda")
+    lse = torch.full((R, n_q), float("nan"), dtype=torch.float32, device="cuda")
+    kalm.kalm_merged_attention(qkv[:, : n_q * D], qkv[:, n_q * D: n_q * D + w], qkv[:, n_q * D + w:],
+                               kvc[:, :w], kvc[:, w:], i64(q_off), i64(p_off), int(np.diff(q_off).max()), n_q,
+                               n_kv, out, scale, lse)
+    kalm.kalm_check_device_errors()
+    return from_dev(out).reshape(R, n_q, D), lse.cpu().numpy().astype(np.float64)
+
+
+def _attn_oracle(a, scale=1.0 / 16):
+    C = int(a["p_off"][-1])
+    return oracle.merged_attention(a["q"], a["ks"], a["vs"], a["kc"][:C], a["vc"][:C], a["q_off"], a["p_off"],
+                                   scale)
+
+
+def _check_attn(got, want):
+    d = np.abs(got - want)
+    assert np.isfinite(got).all()
+    assert d.max() <= ATTN_MAX_TOL, d.max()
+    assert d.mean() <= ATTN_MEAN_TOL, d.mean()
+
+
+@pytest.mark.parametrize("lq,nc,n_q,n_kv", [
+    ([32, 32, 32, 32], [3, 16, 9, 1], 4, 1),              # Tiny shape
+    ([128] * 6, [256, 16, 1, 0, 255, 64], 4, 1),          # Nano shape, empty cross segment, ragged tails
+    ([1, 2, 31, 33, 65, 130], [0, 5, 64, 65, 128, 129], 4, 1),
+    ([256, 100], [75, 256], 8, 4),                        # Large GQA (2 q heads per KV head)
+    ([512, 3], [256, 2], 4, 1),                           # query budget
+    ([17, 64, 200], [7, 0, 100], 2, 2),                   # MHA
+    ([40, 130], [20, 70], 8, 1),                          # 8 q heads per KV head
+    ([5, 9], [0, 0], 4, 1),                               # no cross rows in the whole batch
+])
+def test_merged_attention(kalm, lq, nc, n_q, n_kv):
+    a = _attn_arrays(np.random.default_rng(sum(lq) + sum(nc) + n_q), lq, nc, n_q, n_kv)
+    got, lse = _attn_run(kalm, a)
+    want, want_lse = _attn_oracle(a)
+    _check_attn(got, want)
+    assert np.abs(lse - want_lse).max() < 1e-3
+
+
+def test_merged_attention_running_max_jumps(kalm):
+    # Large cross logits make the running max jump by far more than 2^8 after the
+    # self segment, which exercises the in-place rescale of the O accumulator.
+    a = _attn_arrays(np.random.default_rng(31), [128, 70], [200, 90], 4, 1, q_std=1.0, k_std=1.0, kc_mult=6.0)
+    got, lse = _attn_run(kalm, a)
+    want, want_lse = _attn_oracle(a)
+    _check_attn(got, want)
+    assert np.abs(lse - want_lse).max() < 2e-3
+
+
+def test_merged_attention_lse_two_segment_merge(kalm):
+    # The kernel's LSE of the self-only run, merged with the cross-only LSE (a
+    # plain log-sum-exp over the cross logits), equals the kernel's merged LSE.
+    a = _attn_arrays(np.random.default_rng(32), [64, 96], [40, 130], 4, 1)
+    _, lse = _attn_run(kalm, a)
+    _, lse_self = _attn_run(kalm, a, p_off=np.zeros(3, np.int64))
+    for d in range(2):
+        r0, r1 = a["q_off"][d], a["q_off"][d + 1]
+        c0, c1 = a["p_off"][d], a["p_off"][d + 1]
+        logits = np.einsum("rhd,cd->rhc", a["q"][r0:r1], a["kc"][c0:c1, 0]) / 16
+        lse_cross = np.log(np.exp(logits - logits.max(-1, keepdims=True)).sum(-1)) + logits.max(-1)
+        np.testing.assert_allclose(lse[r0:r1], np.logaddexp(lse_self[r0:r1], lse_cross), atol=2e-3, rtol=0)
+
+
+def test_merged_attention_batch_composition(kalm):
+    # a document's output is bit-identical alone and inside a batch
+    a = _attn_arrays(np.random.default_rng(33), [70, 128, 5], [33, 256, 1], 4, 1)
+    got, _ = _attn_run(kalm, a)
+    r0, r1, c0, c1 = 70, 198, 33, 289
+    b = dict(a, q=a["q"][r0:r1], ks=a["ks"][r0:r1], vs=a["vs"][r0:r1], kc=a["kc"][c0:c1], vc=a["vc"][c0:c1],
+             q_off=np.array([0, r1 - r0]), p_off=np.array([0, c1 - c0]))
+    alone, _ = _attn_run(kalm, b)
+    np.testing.assert_array_equal(alone, got[r0:r1])
+
+
+# ---------------------------------------------------------------------------
+# step 4: readout
+# ---------------------------------------------------------------------------
+def test_yes_no_score(kalm):
+    rng = np.random.default_rng(41)
+    H, lq = 640, [5, 1, 0, 9]
+    q_off = np.concatenate([[0], np.cumsum(lq)])
+    x = rand_bf16(rng, (q_off[-1], H))
+    wy = rand_bf16(rng, H, 0.05)
+    wn = rand_bf16(rng, H, 0.05)
+    n = len(lq)
+    outs = [torch.empty(n, dtype=torch.float32, device="cuda") for _ in range(4)]
+    kalm.kalm_yes_no_score(f64_to_dev(x), i64(q_off), f64_to_dev(wy), f64_to_dev(wn), outs[0], outs[1], outs[3],
+                           margin=outs[2])
+    kalm.kalm_check_device_errors()
+    got = [o.cpu().numpy().astype(np.float64) for o in outs]
+    rows = [q_off[d + 1] - 1 for d in range(n) if lq[d] > 0]
+    y, nn, m, s = oracle.yes_no_score(x[rows], wy, wn)
+    idx = [d for d in range(n) if lq[d] > 0]
+    np.testing.assert_allclose(got[0][idx], y, atol=1e-4, rtol=1e-5)
+    np.testing.assert_allclose(got[1][idx], nn, atol=1e-4, rtol=1e-5)
+    np.testing.assert_allclose(got[2][idx], m, atol=2e-4, rtol=1e-5)
+    assert np.abs(got[3][idx] - s).max() <= SCORE_TOL
+    assert got[3][2] == 0.5 and got[2][2] == 0.0  # empty document
+
+
+def test_yes_no_score_extreme_margins(kalm):
+    H = 8
+    x = np.zeros((4, H))
+    x[:, 0] = [100.0, -100.0, 0.0, 1.0]
+    wy = np.zeros(H)
+    wy[0] = 1.0
+    wn = np.zeros(H)
+    outs = [torch.empty(4, dtype=torch.float32, device="cuda") for _ in range(4)]
+    kalm.kalm_yes_no_score(f64_to_dev(x), i64([0, 1, 2, 3, 4]), f64_to_dev(wy), f64_to_dev(wn), outs[0], outs[1],
+                           outs[3], margin=outs[2])
+    s = outs[3].cpu().numpy()
+    assert s[0] == 1.0 and 0.0 <= s[1] < 1e-30 and s[2] == 0.5 and abs(s[3] - 1 / (1 + math.exp(-1))) < 1e-7
+
+
+# ---------------------------------------------------------------------------
+# end to end
+# ---------------------------------------------------------------------------
+def _scorer(q, graph=False):
+    from encoder_decoder_document_b200.scorer import DeviceWeights, FBNLScorer
+    sc = FBNLScorer(DeviceWeights.from_bits(q.weights), q.n_q, q.n_kv)
+    if graph:
+        doc_len = q.doc_len
+        sc.prepare(q.n_docs, int(doc_len.sum()), int(oracle.pooled_counts(doc_len).sum()), q.lq)
+        sc.load_inputs(torch.from_numpy(q.enc.view(np.int16)).view(torch.bfloat16), torch.from_numpy(doc_len),
+                       torch.from_numpy(q.x0.view(np.int16)).view(torch.bfloat16))
+        sc.capture()
+        sc.run()
+    else:
+        sc.rerank(q.x0, q.enc, q.doc_len)
+    return sc
+
+
+def _check_scores(got_score, want_score, want_margin):
+    assert np.abs(got_score - want_score).max() <= SCORE_TOL
+    # ranking: any pair the oracle separates by more than the gap keeps its order
+    n = len(want_score)
+    for i in range(n):
+        for j in range(n):
+            if want_score[i] - want_score[j] > RANK_GAP:
+                assert got_score[i] > got_score[j]
+
+
+def test_end_to_end_tiny(kalm):
+    q = synthetic.make_query("tiny")
+    sc = _scorer(q)
+    kalm.kalm_check_device_errors()
+    res = sc.scores_to_host().numpy()
+    y, n, m, s = oracle.forward_query(q)
+    _check_scores(res[3], s, m)
+    np.testing.assert_allclose(res[2], res[0] - res[1], atol=1e-5)
+    ranked = sc.rerank(q.x0, q.enc, q.doc_len, top_n=2)
+    assert len(ranked) == 2 and ranked[0]["relevance_score"] >= ranked[1]["relevance_score"]
+
+
+def test_end_to_end_tiny_batch_composition(kalm):
+    # a document's score is the same alone and inside the batch (bitwise)
+    q = synthetic.make_query("tiny")
+    full = _scorer(q).scores_to_host().numpy()[3]
+    for d in range(q.n_docs):
+        a, b = q.tok_off[d], q.tok_off[d + 1]
+        sc = _scorer(synthetic.Query(q.name, q.hidden, q.n_q, q.n_kv, q.head_dim, q.layers, q.doc_len[d:d + 1],
+                                     np.array([0, b - a]), q.enc[a:b], q.lq, q.x0, q.weights))
+        assert sc.scores_to_host().numpy()[3][0] == full[d]
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("name,docs", [("nano", [0, 17, 42, 99]), ("small", [3, 50]), ("large", [1, 77])])
+def test_end_to_end_full_size_sampled(kalm, name, docs):
+    """Full configuration in the launch configuration the benchmark times (CUDA graph);
+    the oracle scores a sample of documents one by one."""
+    q = synthetic.make_query(name)
+    sc = _scorer(q, graph=True)
+    kalm.kalm_check_device_errors()
+    res = sc.scores_to_host().numpy()
+    y, n, m, s = oracle.forward_query(q, docs=docs)
+    assert np.abs(res[3][docs] - s).max() <= SCORE_TOL
+    assert np.all(np.isfinite(res))
+    # stage parity at full size: the document cache and one layer's attention
+    pooled = from_dev(sc.pooled[: sc.total_pooled])
+    want, _ = oracle.chunk_pool(oracle.bf16_bits_to_f64(q.enc), q.tok_off, q.doc_len)
+    assert np.abs(pooled - want).max() <= POOL_TOL
+
+
+# ---------------------------------------------------------------------------
+# failure detection (host-injected; nothing faults, traps or hangs)
+# ---------------------------------------------------------------------------
+def test_bounded_wait_expires_and_context_survives(kalm):
+    from encoder_decoder_document_b200 import KalmError
+    kalm.kalm_selftest_wait_timeout(2_000_000)  # 2 ms on a barrier nobody completes
+    with pytest.raises(KalmError) as e:
+        kalm.kalm_check_device_errors()
+    assert e.value.name == "KALM_ERR_TIMEOUT"
+    assert kalm.kalm_check_device_errors() == 0  # cleared
+    test_yes_no_score(kalm)  # the context still runs kernels
+
+
+def test_invalid_arguments_are_rejected_on_the_host(kalm):
+    from encoder_decoder_document_b200 import KalmError
+    x = torch.zeros(64, 64, dtype=torch.bfloat16, device="cuda")
+    y = torch.zeros(64, 48, dtype=torch.bfloat16, device="cuda")
+    w = torch.zeros(48, 64, dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(KalmError) as e:
+        kalm.kalm_linear(x, w, y)  # n = 48 is not a multiple of 32
+    assert e.value.name == "KALM_ERR_UNSUPPORTED"
+    with pytest.raises(KalmError) as e:
+        kalm.kalm_linear(x[:, 1:57], torch.zeros(64, 56, dtype=torch.bfloat16, device="cuda"),
+                         torch.zeros(64, 64, dtype=torch.bfloat16, device="cuda"))  # misaligned
+    assert e.value.name == "KALM_ERR_INVALID_ARG"
+    q = torch.zeros(8, 512, dtype=torch.bfloat16, device="cuda")
+    off = i64([0, 8])
+    with pytest.raises(KalmError) as e:
+        kalm.kalm_merged_attention(q, q, q, q, q, off, off, 8, 4, 1, q, head_dim=128)
+    assert e.value.name == "KALM_ERR_UNSUPPORTED"
+    with pytest.raises(KalmError) as e:
+        kalm.kalm_merged_attention(q, q, q, q, q, off, off, 600, 2, 1, q)  # above the query budget
+    assert e.value.name == "KALM_ERR_INVALID_ARG"
+    lens = i32([5, 2000])
+    tok = torch.empty(3, dtype=torch.int64, device="cuda")
+    kalm.kalm_ragged_offsets(lens, tok, None, 4)  # 2000 > 1024: clamped and flagged
+    with pytest.raises(KalmError) as e:
+        kalm.kalm_check_device_errors()
+    assert e.value.name == "KALM_ERR_DEVICE_ARG"
+    assert tok.cpu().tolist() == [0, 5, 1029]
