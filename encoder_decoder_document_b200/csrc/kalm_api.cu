@@ -107,7 +107,7 @@ uint32_t* device_error_word() {
 }
 
 kalm_status make_tmap_bf16(CUtensorMap* map, const void* base, int rank, const uint64_t* dims,
-                           const uint64_t* strides_bytes, const uint32_t* box) {
+                           const uint64_t* strides_bytes, const uint32_t* box, int swizzle_bytes) {
   if (!g_encode) return fail(KALM_ERR_CUDA, "tensor-map encoder not initialised");
   cuuint64_t gdim[5];
   cuuint64_t gstride[4];
@@ -119,8 +119,12 @@ kalm_status make_tmap_bf16(CUtensorMap* map, const void* base, int rank, const u
     estride[i] = 1;
   }
   for (int i = 0; i + 1 < rank; ++i) gstride[i] = strides_bytes[i];
+  const CUtensorMapSwizzle sw = swizzle_bytes == 128  ? CU_TENSOR_MAP_SWIZZLE_128B
+                                : swizzle_bytes == 64 ? CU_TENSOR_MAP_SWIZZLE_64B
+                                : swizzle_bytes == 32 ? CU_TENSOR_MAP_SWIZZLE_32B
+                                                      : CU_TENSOR_MAP_SWIZZLE_NONE;
   CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, static_cast<cuuint32_t>(rank), const_cast<void*>(base),
-                        gdim, gstride, bdim, estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        gdim, gstride, bdim, estride, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(KALM_ERR_INVALID_ARG, "cuTensorMapEncodeTiled failed (CUresult %d)", (int)r);
   return KALM_OK;

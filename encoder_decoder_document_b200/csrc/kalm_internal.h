@@ -22,11 +22,11 @@ uint32_t* device_error_word();
 // Map a CUDA runtime error to KALM_ERR_CUDA with its message; KALM_OK if none.
 kalm_status check_cuda(cudaError_t e, const char* what);
 
-// Tiled bf16 tensor maps with 128-byte swizzle and zero fill outside the
-// tensor.  `dims`/`box` list the innermost dimension first; `strides_bytes`
-// holds the byte strides of dimensions 1.. (rank-1 values).
+// Tiled bf16 tensor maps with zero fill outside the tensor.  `dims`/`box` list
+// the innermost dimension first; `strides_bytes` holds the byte strides of
+// dimensions 1.. (rank-1 values); `swizzle_bytes` is 128 (default), 64, 32 or 0.
 kalm_status make_tmap_bf16(CUtensorMap* map, const void* base, int rank, const uint64_t* dims,
-                           const uint64_t* strides_bytes, const uint32_t* box);
+                           const uint64_t* strides_bytes, const uint32_t* box, int swizzle_bytes = 128);
 
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 

@@ -12,8 +12,11 @@
 //               K=16 per instruction) from one thread; tcgen05.commit frees a
 //               ring slot once the tensor core has read it;
 //   warps 2..5  epilogue: tcgen05.ld of the fp32 accumulator (one TMEM lane =
-//               one output row per thread), optional bf16 residual add, one
-//               rounding to bf16, 16-byte stores.
+//               one output row per thread) in 32-column chunks, optional bf16
+//               residual add (the residual chunk is fetched by TMA ahead of
+//               time), one rounding to bf16, then the 32 x 32 chunk is staged in
+//               shared memory (64-byte swizzle, bank-conflict free) and written
+//               by a TMA tile store, so global writes are full lines.
 // The accumulator is double-buffered in TMEM (2 x BN columns) so the epilogue
 // of tile i overlaps the main loop of tile i+1.  Out-of-range rows/columns of
 // x and w are zero-filled by TMA; the epilogue masks their stores.
@@ -28,14 +31,17 @@ constexpr int kBM = 128;
 constexpr int kBK = 64;  // one 128-byte swizzle row of bf16
 constexpr int kThreads = 192;
 
+constexpr int kChunkBytes = 32 * 32 * 2;  // one 32-row x 32-column bf16 epilogue chunk
+
 template <int BN>
 struct LinearCfg {
   static constexpr int STAGES = BN == 256 ? 4 : 6;
   static constexpr int A_BYTES = kBM * kBK * 2;
   static constexpr int B_BYTES = BN * kBK * 2;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int EPI_BYTES = 4 * 2 * kChunkBytes;  // per epilogue warp: 2 staging chunks
   static constexpr int BAR_BYTES = 256;
-  static constexpr int SMEM = 1024 + STAGES * STAGE_BYTES + BAR_BYTES;
+  static constexpr int SMEM = 1024 + STAGES * STAGE_BYTES + 2 * EPI_BYTES + BAR_BYTES;
   static constexpr uint32_t TMEM_COLS = 2 * BN;
   static constexpr uint32_t IDESC = idesc_bf16_f32(kBM, BN, false, false);
 };
@@ -43,18 +49,21 @@ struct LinearCfg {
 template <int BN>
 __global__ void __launch_bounds__(kThreads, 1)
     linear_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w,
-                  const __nv_bfloat16* __restrict__ residual, int64_t ldr, __nv_bfloat16* y, int64_t ldy, int M,
-                  int N, int K, uint64_t wait_ns, uint32_t* err) {
+                  const __grid_constant__ CUtensorMap tm_y, const __grid_constant__ CUtensorMap tm_r,
+                  bool has_residual, int M, int N, int K, uint64_t wait_ns, uint32_t* err) {
   using C = LinearCfg<BN>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
   uint8_t* sB = smem + C::STAGES * C::A_BYTES;
-  uint64_t* full = reinterpret_cast<uint64_t*>(sB + C::STAGES * C::B_BYTES);
+  uint8_t* sOut = sB + C::STAGES * C::B_BYTES;  // [4 warps][2][32 x 32 bf16]
+  uint8_t* sRes = sOut + C::EPI_BYTES;          // [4 warps][2][32 x 32 bf16]
+  uint64_t* full = reinterpret_cast<uint64_t*>(sRes + C::EPI_BYTES);
   uint64_t* empty = full + C::STAGES;
   uint64_t* acc_full = empty + C::STAGES;
   uint64_t* acc_empty = acc_full + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 2);
+  uint64_t* res_full = acc_empty + 2;  // [4 warps][2]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(res_full + 8);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -67,6 +76,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&acc_full[b], 1);
       mbar_init(&acc_empty[b], 128);
     }
+    for (int b = 0; b < 8; ++b) mbar_init(&res_full[b], 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -154,10 +164,26 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else {
     // epilogue warps 2..5: warp w may access TMEM lanes 32*(w%4) .. 32*(w%4)+31
     const int quarter = warp & 3;
-    const int row_in_tile = quarter * 32 + lane;
+    const int ew = warp - 2;
+    uint8_t* obuf = sOut + ew * 2 * kChunkBytes;
+    uint8_t* rbuf = sRes + ew * 2 * kChunkBytes;
+    uint64_t* rbar = res_full + ew * 2;
+    uint32_t rphase = 0u;  // bit b: parity of residual buffer b
     int acc = 0;
     uint32_t acc_phase = 0;
+    int out_slot = 0;
+    // 64-byte swizzle of a 32 x 64 B chunk: 16-byte unit i of row r sits at unit i ^ ((r >> 1) & 3)
+    const uint32_t swz = static_cast<uint32_t>((lane >> 1) & 3);
     for (int t = blockIdx.x; t < tiles; t += gridDim.x) {
+      const int m0 = (t / n_n) * kBM, n0 = (t % n_n) * BN;
+      const int row0 = m0 + quarter * 32;
+      const int nch = min(BN, N - n0) / 32;
+      if (has_residual && lane == 0) {
+        for (int c = 0; c < 2 && c < nch; ++c) {
+          mbar_arrive_expect_tx(&rbar[c], kChunkBytes);
+          tma_load_2d(rbuf + c * kChunkBytes, &tm_r, &rbar[c], n0 + c * 32, row0);
+        }
+      }
       bool ok = mbar_wait(&acc_full[acc], acc_phase, wait_ns);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok || *abort_flag) {
@@ -166,50 +192,70 @@ __global__ void __launch_bounds__(kThreads, 1)
         break;
       }
       tc_fence_after();
-      const int m0 = (t / n_n) * kBM, n0 = (t % n_n) * BN;
-      const int m = m0 + row_in_tile;
       const uint32_t t_row = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + static_cast<uint32_t>(acc * BN);
 #pragma unroll 1
-      for (int c0 = 0; c0 < BN; c0 += 32) {
+      for (int c = 0; c < nch; ++c) {
         uint32_t r[32];
-        tmem_ld32(t_row + c0, r);
+        tmem_ld32(t_row + c * 32, r);
         tmem_ld_wait();
-        const int n = n0 + c0;
-        if (m < M && n < N) {
-          float v[32];
+        float v[32];
 #pragma unroll
-          for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
-          if (residual) {
-            const uint4* rp = reinterpret_cast<const uint4*>(residual + static_cast<int64_t>(m) * ldr + n);
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              const uint4 rv = rp[q];
-              const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&rv);
-#pragma unroll
-              for (int k = 0; k < 4; ++k) {
-                const float2 f = __bfloat1622float2(h[k]);
-                v[q * 8 + 2 * k] += f.x;
-                v[q * 8 + 2 * k + 1] += f.y;
-              }
-            }
+        for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
+        if (has_residual) {
+          const int b = c & 1;
+          bool okr = mbar_wait(&rbar[b], (rphase >> b) & 1u, wait_ns);
+          rphase ^= 1u << b;
+          if (!__all_sync(0xffffffffu, okr)) {
+            if (lane == 0) record_error(err, kErrTimeout | kSiteLinear);
+            *abort_flag = 1;
+            break;
           }
-          uint4* yp = reinterpret_cast<uint4*>(y + static_cast<int64_t>(m) * ldy + n);
+          const uint8_t* rrow = rbuf + b * kChunkBytes + lane * 64;
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
-            uint4 o;
-            o.x = pack_bf16x2(v[q * 8 + 0], v[q * 8 + 1]);
-            o.y = pack_bf16x2(v[q * 8 + 2], v[q * 8 + 3]);
-            o.z = pack_bf16x2(v[q * 8 + 4], v[q * 8 + 5]);
-            o.w = pack_bf16x2(v[q * 8 + 6], v[q * 8 + 7]);
-            yp[q] = o;
+            const uint4 rv = *reinterpret_cast<const uint4*>(rrow + ((q ^ swz) << 4));
+            const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&rv);
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              const float2 f = __bfloat1622float2(h[k]);
+              v[q * 8 + 2 * k] += f.x;
+              v[q * 8 + 2 * k + 1] += f.y;
+            }
+          }
+          __syncwarp();
+          if (lane == 0 && c + 2 < nch) {  // refill this residual buffer two chunks ahead
+            mbar_arrive_expect_tx(&rbar[b], kChunkBytes);
+            tma_load_2d(rbuf + b * kChunkBytes, &tm_r, &rbar[b], n0 + (c + 2) * 32, row0);
           }
         }
+        // the staging slot is free once the store issued from it two chunks ago has read it
+        if (lane == 0) bulk_wait_group_read<1>();
+        __syncwarp();
+        uint8_t* orow = obuf + out_slot * kChunkBytes + lane * 64;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          uint4 o;
+          o.x = pack_bf16x2(v[q * 8 + 0], v[q * 8 + 1]);
+          o.y = pack_bf16x2(v[q * 8 + 2], v[q * 8 + 3]);
+          o.z = pack_bf16x2(v[q * 8 + 4], v[q * 8 + 5]);
+          o.w = pack_bf16x2(v[q * 8 + 6], v[q * 8 + 7]);
+          *reinterpret_cast<uint4*>(orow + ((q ^ swz) << 4)) = o;
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          tma_store_2d(&tm_y, obuf + out_slot * kChunkBytes, n0 + c * 32, row0);
+          bulk_commit_group();
+        }
+        out_slot ^= 1;
       }
+      if (*abort_flag) break;
       tc_fence_before();
       mbar_arrive(&acc_empty[acc]);
       acc ^= 1;
       if (acc == 0) acc_phase ^= 1u;
     }
+    if (lane == 0) bulk_wait_group<0>();
   }
   tc_fence_before();
   __syncthreads();
@@ -279,15 +325,29 @@ kalm_status launch_linear(const kalm_bf16* x, int64_t ldx, const kalm_bf16* w, i
     kalm_status st = make_tmap_bf16(&tw, w, 2, dims, strides, box);
     if (st != KALM_OK) return st;
   }
+  CUtensorMap ty, tr;
+  {
+    const uint64_t dims[2] = {static_cast<uint64_t>(n), static_cast<uint64_t>(m)};
+    const uint64_t strides[1] = {static_cast<uint64_t>(ldy) * 2};
+    const uint32_t box[2] = {32, 32};
+    kalm_status st = make_tmap_bf16(&ty, y, 2, dims, strides, box, 64);
+    if (st != KALM_OK) return st;
+    if (residual) {
+      const uint64_t rstrides[1] = {static_cast<uint64_t>(ldr) * 2};
+      st = make_tmap_bf16(&tr, residual, 2, dims, rstrides, box, 64);
+      if (st != KALM_OK) return st;
+    } else {
+      tr = ty;  // never read
+    }
+  }
   const int64_t tiles = ((m + kBM - 1) / kBM) * ((n + BN - 1) / BN);
   const int grid = static_cast<int>(tiles < num_sms() ? tiles : num_sms());
-  const auto* r = reinterpret_cast<const __nv_bfloat16*>(residual);
-  auto* yy = reinterpret_cast<__nv_bfloat16*>(y);
+  const bool has_r = residual != nullptr;
   if (wide)
-    linear_kernel<256><<<grid, kThreads, LinearCfg<256>::SMEM, stream>>>(tx, tw, r, ldr, yy, ldy, (int)m, n, k,
+    linear_kernel<256><<<grid, kThreads, LinearCfg<256>::SMEM, stream>>>(tx, tw, ty, tr, has_r, (int)m, n, k,
                                                                           kWaitNs, device_error_word());
   else
-    linear_kernel<128><<<grid, kThreads, LinearCfg<128>::SMEM, stream>>>(tx, tw, r, ldr, yy, ldy, (int)m, n, k,
+    linear_kernel<128><<<grid, kThreads, LinearCfg<128>::SMEM, stream>>>(tx, tw, ty, tr, has_r, (int)m, n, k,
                                                                           kWaitNs, device_error_word());
   return check_cuda(cudaGetLastError(), "launch linear_kernel");
 }

@@ -68,7 +68,8 @@ struct AttnParams {
 __global__ void __launch_bounds__(kThreads, 1)
     merged_attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_ks,
                             const __grid_constant__ CUtensorMap tm_vs, const __grid_constant__ CUtensorMap tm_kc,
-                            const __grid_constant__ CUtensorMap tm_vc, const AttnParams p) {
+                            const __grid_constant__ CUtensorMap tm_vc, const __grid_constant__ CUtensorMap tm_o,
+                            const AttnParams p) {
   // ---- work item: heaviest query tiles (largest t) first
   const int per_t = p.n_docs * p.n_kv;
   const int t = p.tiles_per_doc - 1 - static_cast<int>(blockIdx.x) / per_t;
@@ -312,14 +313,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float inv_l = 1.f / l_run;
         const bool valid = pos < pos1;
         const int head = g * p.G + hh;
-        __nv_bfloat16* orow = p.out + (q0 + pos) * p.ldo + static_cast<int64_t>(head) * kD;
+        if (pos0 + p.P <= Lq) {
+          // Full tile: stage O as bf16 in the (now idle) Q tile, in the same
+          // 128-byte-swizzled slabs, and write it with four 3-D TMA stores whose
+          // boxes match the Q boxes (positions x heads x 64 columns).
 #pragma unroll 1
-        for (int c = 0; c < kD; c += 32) {
-          uint32_t o[32];
-          tmem_ld32(lane_base + c, o);
-          tmem_ld_wait();
-          if (valid) {
-            uint4* dst = reinterpret_cast<uint4*>(orow + c);
+          for (int c = 0; c < kD; c += 32) {
+            uint32_t o[32];
+            tmem_ld32(lane_base + c, o);
+            tmem_ld_wait();
+            uint8_t* row = sQ + (c >> 6) * kQSlab + r * 128;
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
               uint4 v;
@@ -327,7 +330,29 @@ __global__ void __launch_bounds__(kThreads, 1)
               v.y = pack_bf16x2(__uint_as_float(o[8 * q + 2]) * inv_l, __uint_as_float(o[8 * q + 3]) * inv_l);
               v.z = pack_bf16x2(__uint_as_float(o[8 * q + 4]) * inv_l, __uint_as_float(o[8 * q + 5]) * inv_l);
               v.w = pack_bf16x2(__uint_as_float(o[8 * q + 6]) * inv_l, __uint_as_float(o[8 * q + 7]) * inv_l);
-              dst[q] = v;
+              const int unit = ((c & 63) >> 3) + q;  // 16-byte unit inside the 128-byte row
+              *reinterpret_cast<uint4*>(row + ((unit ^ (r & 7)) << 4)) = v;
+            }
+          }
+          fence_proxy_async_smem();  // the TMA stores are issued after the CTA barrier below
+        } else {
+          __nv_bfloat16* orow = p.out + (q0 + pos) * p.ldo + static_cast<int64_t>(head) * kD;
+#pragma unroll 1
+          for (int c = 0; c < kD; c += 32) {
+            uint32_t o[32];
+            tmem_ld32(lane_base + c, o);
+            tmem_ld_wait();
+            if (valid) {
+              uint4* dst = reinterpret_cast<uint4*>(orow + c);
+#pragma unroll
+              for (int q = 0; q < 4; ++q) {
+                uint4 v;
+                v.x = pack_bf16x2(__uint_as_float(o[8 * q + 0]) * inv_l, __uint_as_float(o[8 * q + 1]) * inv_l);
+                v.y = pack_bf16x2(__uint_as_float(o[8 * q + 2]) * inv_l, __uint_as_float(o[8 * q + 3]) * inv_l);
+                v.z = pack_bf16x2(__uint_as_float(o[8 * q + 4]) * inv_l, __uint_as_float(o[8 * q + 5]) * inv_l);
+                v.w = pack_bf16x2(__uint_as_float(o[8 * q + 6]) * inv_l, __uint_as_float(o[8 * q + 7]) * inv_l);
+                dst[q] = v;
+              }
             }
           }
         }
@@ -343,6 +368,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 5) {
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
+  } else if (threadIdx.x == 0 && pos0 + p.P <= Lq && !*abort_flag) {
+    for (int j = 0; j < 4; ++j)
+      tma_store_3d(&tm_o, sQ + j * kQSlab, j * 64, g * p.G, static_cast<int32_t>(q0 + pos0));
+    bulk_commit_group();
+    bulk_wait_group<0>();
   }
 }
 
@@ -386,12 +416,14 @@ extern "C" kalm_status kalm_merged_attention(const kalm_bf16* q, int64_t ldq, co
   if (total_q > INT32_MAX - 1024 || total_pool > INT32_MAX - 1024)
     return fail(KALM_ERR_INVALID_ARG, "kalm_merged_attention: too many rows");
 
-  CUtensorMap tq, tks, tvs, tkc, tvc;
+  CUtensorMap tq, tks, tvs, tkc, tvc, to;
   {
     const uint64_t dims[3] = {kD, static_cast<uint64_t>(n_q), static_cast<uint64_t>(total_q)};
     const uint64_t strides[2] = {kD * 2, static_cast<uint64_t>(ldq) * 2};
     const uint32_t box[3] = {64, static_cast<uint32_t>(G), static_cast<uint32_t>(kBM / G)};
     if ((st = make_tmap_bf16(&tq, q, 3, dims, strides, box)) != KALM_OK) return st;
+    const uint64_t ostrides[2] = {kD * 2, static_cast<uint64_t>(ldo) * 2};
+    if ((st = make_tmap_bf16(&to, out, 3, dims, ostrides, box)) != KALM_OK) return st;
   }
   auto kv_map = [&](CUtensorMap* m, const kalm_bf16* base, int64_t ld, int64_t rows) -> kalm_status {
     const uint64_t dims[2] = {static_cast<uint64_t>(n_kv) * kD, static_cast<uint64_t>(rows > 0 ? rows : 1)};
@@ -427,6 +459,6 @@ extern "C" kalm_status kalm_merged_attention(const kalm_bf16* q, int64_t ldq, co
   const int64_t grid = static_cast<int64_t>(prm.tiles_per_doc) * n_docs * n_kv;
   if (grid > INT32_MAX) return fail(KALM_ERR_INVALID_ARG, "kalm_merged_attention: grid too large");
   merged_attention_kernel<<<static_cast<unsigned>(grid), kThreads, kSmem, static_cast<cudaStream_t>(stream)>>>(
-      tq, tks, tvs, tkc, tvc, prm);
+      tq, tks, tvs, tkc, tvc, to, prm);
   return check_cuda(cudaGetLastError(), "launch merged_attention_kernel");
 }

@@ -127,16 +127,25 @@ class FBNLScorer:
         D, nq, nkv = self.D, self.n_q, self.n_kv
         return (self.qkv[:, : nq * D], self.qkv[:, nq * D:(nq + nkv) * D], self.qkv[:, (nq + nkv) * D:])
 
-    def layer(self, l: int) -> None:
+    def layer_qkv(self, l: int) -> None:
         kalm_linear(self.x, self.w.w_qkv[l], self.qkv)
         self._mark("qkv_proj")
+
+    def layer_attention(self, l: int) -> None:
         q, ks, vs = self.qkv_views()
         kc, vc = self.cross_views(l)
         kalm_merged_attention(q, ks, vs, kc, vc, self.q_off, self.pool_off, self.lq, self.n_q, self.n_kv, self.o,
                               self.scale)
         self._mark("merged_attention")
+
+    def layer_out(self, l: int) -> None:
         kalm_linear(self.o, self.w.w_o[l], self.x, residual=self.x)
         self._mark("o_proj")
+
+    def layer(self, l: int) -> None:
+        self.layer_qkv(l)
+        self.layer_attention(l)
+        self.layer_out(l)
 
     def readout(self) -> None:
         kalm_yes_no_score(self.x, self.q_off, self.w.w_yes, self.w.w_no, self.yes, self.no, self.score,

@@ -35,6 +35,7 @@ from .kalm_oracle import (  # noqa: F401
     linear,
     merged_attention_doc,
     merged_attention,
+    decoder_layer,
     yes_no_score,
     sigmoid,
     forward_doc,

@@ -237,33 +237,41 @@ def yes_no_score(x_last: np.ndarray, w_yes: np.ndarray, w_no: np.ndarray):
 # ----------------------------------------------------------------------------
 # End to end (oracle mode (ii): the oracle chains its own rounded outputs)
 # ----------------------------------------------------------------------------
+def decoder_layer(X: np.ndarray, pooled: np.ndarray, w_qkv_l, w_o_l, w_kv_l, n_q: int, n_kv: int,
+                  head_dim: int, scale: float, trace: Optional[dict] = None) -> np.ndarray:
+    """One layer of the synthetic attention-only decoder for one document.
+
+    Reading of the synthetic stack (the pages name no MLP/norm on this path):
+    ``X <- X + MergedAttn(X Wq, X Wk, X Wv, P Wk_c, P Wv_c) Wo`` with P the
+    document's pooled vectors.  Returns the new X (bf16-rounded)."""
+    D = head_dim
+    Lq = X.shape[0]
+    kv = linear(pooled, w_kv_l).reshape(-1, 2, n_kv, D)
+    qkv = linear(X, w_qkv_l)
+    q = qkv[:, : n_q * D].reshape(Lq, n_q, D)
+    ks = qkv[:, n_q * D:(n_q + n_kv) * D].reshape(Lq, n_kv, D)
+    vs = qkv[:, (n_q + n_kv) * D:].reshape(Lq, n_kv, D)
+    o, lse = merged_attention_doc(q, ks, vs, kv[:, 0], kv[:, 1], scale)
+    Xn = linear(o.reshape(Lq, n_q * D), w_o_l, residual=X)
+    if trace is not None:
+        trace.setdefault("layers", []).append(dict(x_in=X, qkv=qkv, kv_cross=kv, o=o, lse=lse, x_out=Xn))
+    return Xn
+
+
 def forward_doc(enc_doc: np.ndarray, x0: np.ndarray, w_qkv, w_o, w_kv_cross,
                 w_yes, w_no, n_q: int, n_kv: int, head_dim: int, scale: float,
                 chunk: int = 4, layers: Optional[Sequence[int]] = None,
                 trace: Optional[dict] = None):
-    """Score one document with the synthetic attention-only decoder stack.
-
-    Reading of the synthetic stack: per layer l,
-    ``X <- X + MergedAttn(X Wq, X Wk, X Wv, P Wk_c, P Wv_c) Wo`` with P the
-    document's pooled vectors and X0 the query's decoder input; no MLP, no norm.
+    """Score one document with the synthetic attention-only decoder stack
+    (``decoder_layer`` per layer, X0 = the query's decoder input).
     Returns ``(yes, no, margin, score)`` as floats.  ``trace`` (a dict), if
     given, receives the intermediate tensors of every layer."""
-    D = head_dim
     Lq = x0.shape[0]
     pooled, _ = chunk_pool(enc_doc, [0], [enc_doc.shape[0]], chunk)
     X = np.asarray(x0, np.float64)
     lay = range(len(w_qkv)) if layers is None else layers
     for l in lay:
-        kv = linear(pooled, w_kv_cross[l]).reshape(-1, 2, n_kv, D)
-        qkv = linear(X, w_qkv[l])
-        q = qkv[:, : n_q * D].reshape(Lq, n_q, D)
-        ks = qkv[:, n_q * D:(n_q + n_kv) * D].reshape(Lq, n_kv, D)
-        vs = qkv[:, (n_q + n_kv) * D:].reshape(Lq, n_kv, D)
-        o, lse = merged_attention_doc(q, ks, vs, kv[:, 0], kv[:, 1], scale)
-        Xn = linear(o.reshape(Lq, n_q * D), w_o[l], residual=X)
-        if trace is not None:
-            trace.setdefault("layers", []).append(dict(x_in=X, qkv=qkv, kv_cross=kv, o=o, lse=lse, x_out=Xn))
-        X = Xn
+        X = decoder_layer(X, pooled, w_qkv[l], w_o[l], w_kv_cross[l], n_q, n_kv, head_dim, scale, trace)
     if trace is not None:
         trace["pooled"] = pooled
         trace["x_final"] = X

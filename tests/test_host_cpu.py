@@ -1,0 +1,119 @@
+"""Host-side checks that need no GPU: the C-ABI library builds, loads and exports
+every symbol include/kalm.h declares; without a device every entry point
+refuses with KALM_ERR_NO_DEVICE (no CPU fallback); document sharding and the
+two-rank gather (gloo) reproduce the single-process scores in input order."""
+import os
+import re
+import socket
+
+import numpy as np
+import pytest
+import torch
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared_symbols():
+    names = []
+    for fn in sorted(os.listdir(os.path.join(ROOT, "include"))):
+        if fn.endswith(".h"):
+            text = open(os.path.join(ROOT, "include", fn)).read()
+            text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+            names += re.findall(r"^\s*(?:const\s+)?\w+\s*\*?\s*(kalm_\w+)\s*\(", text, flags=re.M)
+    return sorted(set(names))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    import __graft_entry__
+    __graft_entry__.build()
+    import encoder_decoder_document_b200 as k
+    return k.load()
+
+
+def test_library_exports_every_declared_symbol(lib):
+    names = _declared_symbols()
+    assert len(names) >= 12
+    import encoder_decoder_document_b200._abi as abi
+    for n in names:
+        assert hasattr(lib, n), f"{n} is declared in include/ but not exported"
+        assert n in abi.SIGNATURES, f"{n} has no binding signature"
+
+
+def test_status_strings_and_version(lib):
+    assert lib.kalm_version() == 100
+    for code, name in [(0, b"KALM_OK"), (3, b"KALM_ERR_NO_DEVICE"), (5, b"KALM_ERR_TIMEOUT")]:
+        assert lib.kalm_status_string(code) == name
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-device path")
+def test_no_device_is_an_explicit_error(lib):
+    import encoder_decoder_document_b200 as k
+    assert lib.kalm_device_check() == 3
+    assert lib.kalm_linear(None, 0, None, 0, None, 0, None, 0, 0, 32, 8, None) == 3
+    assert lib.kalm_chunk_pool(None, 0, None, None, 0, 8, 4, None, 0, None, 0, None) == 3
+    with pytest.raises(k.KalmError) as e:
+        k.kalm_device_check()
+    assert e.value.name == "KALM_ERR_NO_DEVICE"
+
+
+def test_shard_documents_balanced_and_complete():
+    from encoder_decoder_document_b200.sharding import shard_documents
+    rng = np.random.default_rng(0)
+    lens = rng.integers(1, 1025, 100)
+    for world in (1, 2, 3, 8):
+        shards = shard_documents(lens, world)
+        allidx = np.sort(np.concatenate(shards))
+        np.testing.assert_array_equal(allidx, np.arange(100))
+        loads = [float((512 + lens[s]).sum()) for s in shards]
+        assert max(loads) - min(loads) <= 512 + 1024  # LPT bound: one document's cost
+    assert [len(s) for s in shard_documents([5], 4)] == [1, 0, 0, 0]
+
+
+def _free_port():
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    p = s.getsockname()[1]
+    s.close()
+    return p
+
+
+def _rank_main(rank, world, port, out):
+    import torch.distributed as dist
+    import datetime
+    import oracle
+    import synthetic
+    from encoder_decoder_document_b200.sharding import merge_scores, shard_documents
+    dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{port}", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=60))
+    q = synthetic.make_query("tiny", hidden=64, n_docs=5)
+    shards = shard_documents(q.doc_len, world)
+    mine = shards[rank]
+    part = np.stack(oracle.forward_query(q, docs=mine), 1) if len(mine) else np.zeros((0, 4))
+    gathered = [None] * world
+    dist.all_gather_object(gathered, part)
+    if rank == 0:
+        out.put(merge_scores(shards, gathered, q.n_docs))
+    dist.barrier()
+    dist.destroy_process_group()
+
+
+def test_two_rank_document_sharding_gloo():
+    import multiprocessing as mp
+    import oracle
+    import synthetic
+    ctx = mp.get_context("spawn")
+    out = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_rank_main, args=(r, 2, port, out)) for r in range(2)]
+    for p in procs:
+        p.start()
+    merged = out.get(timeout=240)
+    for p in procs:
+        p.join(timeout=120)
+        assert p.exitcode == 0
+    q = synthetic.make_query("tiny", hidden=64, n_docs=5)
+    want = np.stack(oracle.forward_query(q), 1)
+    np.testing.assert_array_equal(merged, want)
+    from encoder_decoder_document_b200.scorer import rank
+    assert rank(merged[:, 2], merged[:, 3]) == rank(want[:, 2], want[:, 3])
