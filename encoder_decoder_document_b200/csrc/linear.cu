@@ -6,12 +6,15 @@
 // output projections.
 //
 // Design (sm_100a): a persistent, warp-specialised kernel, one CTA per SM.
-//   warp 0      TMA producer: 128 x 64 tiles of x and BN x 64 tiles of w (128-byte
-//               swizzle) into a STAGES-deep shared-memory ring;
-//   warp 1      allocates tensor memory and issues tcgen05.mma (M=128, N=BN,
+//   warps 0-3   TMA producers: 128 x 64 tiles of x and BN x 64 tiles of w (128-byte
+//               swizzle) into a STAGES-deep shared-memory ring.  A warp's tile
+//               copies are served one after another, so the copies are spread
+//               over four warps (x or w, even or odd k-block) to keep enough of
+//               them in flight;
+//   warp 4      allocates tensor memory and issues tcgen05.mma (M=128, N=BN,
 //               K=16 per instruction) from one thread; tcgen05.commit frees a
 //               ring slot once the tensor core has read it;
-//   warps 2..5  epilogue: tcgen05.ld of the fp32 accumulator (one TMEM lane =
+//   warps 5..8  epilogue: tcgen05.ld of the fp32 accumulator (one TMEM lane =
 //               one output row per thread) in 32-column chunks, optional bf16
 //               residual add (the residual chunk is fetched by TMA ahead of
 //               time), one rounding to bf16, then the 32 x 32 chunk is staged in
@@ -29,7 +32,10 @@ namespace {
 
 constexpr int kBM = 128;
 constexpr int kBK = 64;  // one 128-byte swizzle row of bf16
-constexpr int kThreads = 192;
+constexpr int kProdWarps = 4;
+constexpr int kMmaWarp = 4;
+constexpr int kEpiWarp0 = 5;
+constexpr int kThreads = 32 * (kEpiWarp0 + 4);
 
 constexpr int kChunkBytes = 32 * 32 * 2;  // one 32-row x 32-column bf16 epilogue chunk
 
@@ -69,7 +75,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::STAGES; ++s) {
-      mbar_init(&full[s], 1);
+      mbar_init(&full[s], 2);  // the x copy and the w copy each arrive with their bytes
       mbar_init(&empty[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
@@ -80,7 +86,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 1) {
+  if (warp == kMmaWarp) {
     tmem_alloc(tmem_slot, C::TMEM_COLS);
     tmem_relinquish();
   }
@@ -94,23 +100,32 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int tiles = n_m * n_n;
   const int kblocks = (K + kBK - 1) / kBK;
 
-  if (warp == 0) {
+  if (warp < kProdWarps) {
     if (lane == 0) {
-      tma_prefetch_desc(&tm_x);
-      tma_prefetch_desc(&tm_w);
+      const bool is_w = warp >= 2;      // which operand this warp copies
+      const uint32_t mine = warp & 1;   // which k-blocks (by parity of the running count)
+      const CUtensorMap* tm = is_w ? &tm_w : &tm_x;
+      tma_prefetch_desc(tm);
       int stage = 0;
       uint32_t phase = 0;
+      uint32_t it = 0;
       for (int t = blockIdx.x; t < tiles && !*abort_flag; t += gridDim.x) {
         const int m0 = (t / n_n) * kBM, n0 = (t % n_n) * BN;
-        for (int kb = 0; kb < kblocks; ++kb) {
-          if (!mbar_wait(&empty[stage], phase ^ 1u, wait_ns)) {
-            record_error(err, kErrTimeout | kSiteLinear);
-            *abort_flag = 1;
-            break;
+        for (int kb = 0; kb < kblocks; ++kb, ++it) {
+          if ((it & 1u) == mine) {
+            if (!mbar_wait(&empty[stage], phase ^ 1u, wait_ns)) {
+              record_error(err, kErrTimeout | kSiteLinear);
+              *abort_flag = 1;
+              break;
+            }
+            if (is_w) {
+              mbar_arrive_expect_tx(&full[stage], C::B_BYTES);
+              tma_load_2d(sB + stage * C::B_BYTES, tm, &full[stage], kb * kBK, n0);
+            } else {
+              mbar_arrive_expect_tx(&full[stage], C::A_BYTES);
+              tma_load_2d(sA + stage * C::A_BYTES, tm, &full[stage], kb * kBK, m0);
+            }
           }
-          mbar_arrive_expect_tx(&full[stage], C::STAGE_BYTES);
-          tma_load_2d(sA + stage * C::A_BYTES, &tm_x, &full[stage], kb * kBK, m0);
-          tma_load_2d(sB + stage * C::B_BYTES, &tm_w, &full[stage], kb * kBK, n0);
           if (++stage == C::STAGES) {
             stage = 0;
             phase ^= 1u;
@@ -118,7 +133,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
     }
-  } else if (warp == 1) {
+  } else if (warp == kMmaWarp) {
     if (lane == 0) {
       int stage = 0;
       uint32_t phase = 0;
@@ -162,9 +177,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
   } else {
-    // epilogue warps 2..5: warp w may access TMEM lanes 32*(w%4) .. 32*(w%4)+31
+    // epilogue warps 5..8: warp w may access TMEM lanes 32*(w%4) .. 32*(w%4)+31
     const int quarter = warp & 3;
-    const int ew = warp - 2;
+    const int ew = warp - kEpiWarp0;
     uint8_t* obuf = sOut + ew * 2 * kChunkBytes;
     uint8_t* rbuf = sRes + ew * 2 * kChunkBytes;
     uint64_t* rbar = res_full + ew * 2;
@@ -259,7 +274,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 1) {
+  if (warp == kMmaWarp) {
     tc_fence_after();
     tmem_dealloc(tmem, C::TMEM_COLS);
   }

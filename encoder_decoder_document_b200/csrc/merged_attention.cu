@@ -15,15 +15,24 @@
 //     loop order; nothing is materialised in memory.
 //   * S = Q K^T and O += P V run on the tensor cores (tcgen05.mma, fp32
 //     accumulators in tensor memory: O = 256 columns, S double-buffered 2 x 64).
-//   * Softmax: one thread per row reads its S row with tcgen05.ld, keeps an
-//     online (running max / running sum) softmax in fp32 with exp2, and writes P
-//     as bf16 into a 128-byte-swizzled shared tile that is the A operand of PV.
+//   * Softmax: two threads per row (warps w and w+4 share TMEM lane quarter
+//     w % 4).  Both read the row's 64 scores with tcgen05.ld and take the same
+//     row max, so they agree on the running max without talking to each other;
+//     each then exponentiates (ex2 on the fused scale) and writes its own 32
+//     columns of P as bf16 into a 128-byte-swizzled shared tile (the A operand
+//     of PV), and keeps its own partial row sum.  The two partial sums meet
+//     once, in the epilogue, which again splits the 256 O columns in halves.
 //     The running max is only raised when it grows by more than 2^8 in the
 //     exponent; otherwise P keeps the stale max (values stay below 256), so the
 //     O accumulator is rescaled in tensor memory only on such rare jumps.  The
 //     final O / l is exact either way.
-//   * Warp roles: warps 0-3 softmax + epilogue, warp 4 TMA producer, warp 5
-//     tensor-memory allocation and MMA issue.  K, V and P are double-buffered.
+//   * Warp roles: warps 0-7 softmax + epilogue, warp 8 TMA producer of Q and K,
+//     warp 10 TMA producer of V, warp 9 tensor-memory allocation and MMA issue.
+//     K, V and P are double-buffered.  Each tile is one TMA box: a 64-key K or V
+//     tile is a 3-D box (64 columns x 64 keys x 4 column slabs) and the Q tile a
+//     4-D box (64 columns x heads x positions x 4 slabs), because a warp's tile
+//     copies are served one after another and few large boxes keep the copy
+//     engine busy where many small ones would not.
 #include <cmath>
 
 #include "kalm.h"
@@ -36,13 +45,17 @@ namespace {
 constexpr int kD = 256;
 constexpr int kBM = 128;
 constexpr int kBKV = 64;
-constexpr int kThreads = 192;
+constexpr int kThreads = 352;
+constexpr int kSoftmaxThreads = 256;
+constexpr int kTmaWarp = 8;
+constexpr int kMmaWarp = 9;
+constexpr int kTmaWarpV = 10;
 constexpr int kQBytes = kBM * kD * 2;          // 4 slabs of 128 rows x 128 B
 constexpr int kQSlab = kBM * 128;              // 16 KB
 constexpr int kKVBytes = kBKV * kD * 2;        // 4 slabs of 64 rows x 128 B
 constexpr int kKVSlab = kBKV * 128;            // 8 KB
 constexpr int kPBytes = kBM * kBKV * 2;        // 1 slab of 128 rows x 128 B
-constexpr int kSmem = 1024 + kQBytes + 2 * kKVBytes + 2 * kKVBytes + 2 * kPBytes + 256;
+constexpr int kSmem = 1024 + kQBytes + 2 * kKVBytes + 2 * kKVBytes + 2 * kPBytes + 128 + 2 * 128 * 4;
 constexpr uint32_t kTmemCols = 512;            // O: [0,256), S0: [256,320), S1: [320,384)
 constexpr uint32_t kIdescS = idesc_bf16_f32(kBM, kBKV, false, false);
 constexpr uint32_t kIdescPV = idesc_bf16_f32(kBM, kD, false, true);
@@ -100,8 +113,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* bar_s = bars + 5;   // [2]
   uint64_t* bar_p = bars + 7;   // [2]
   uint64_t* bar_pv = bars + 9;  // [2]
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 11);
+  uint64_t* bar_l = bars + 11;  // partial row sums published
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 12);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  float* l_part = reinterpret_cast<float*>(bars + 16);  // [2][128]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
@@ -110,13 +125,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&bar_k[i], 1);
       mbar_init(&bar_v[i], 1);
       mbar_init(&bar_s[i], 1);
-      mbar_init(&bar_p[i], 128);
+      mbar_init(&bar_p[i], kSoftmaxThreads);
       mbar_init(&bar_pv[i], 1);
     }
+    mbar_init(bar_l, kSoftmaxThreads);
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 5) {
+  if (warp == kMmaWarp) {
     tmem_alloc(tmem_slot, kTmemCols);
     tmem_relinquish();
   }
@@ -125,38 +141,33 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 4) {
-    // ------------------------------------------------------------ TMA producer
+  if (warp == kTmaWarp || warp == kTmaWarpV) {
+    // ------------------------------------------------------------ TMA producers (Q+K, V)
     if (lane == 0) {
-      mbar_arrive_expect_tx(bar_q, kQBytes);
-      for (int j = 0; j < 4; ++j)
-        tma_load_3d(sQ + j * kQSlab, &tm_q, bar_q, j * 64, g * p.G, static_cast<int32_t>(q0 + pos0));
+      const bool is_v = warp == kTmaWarpV;
+      if (!is_v) {
+        mbar_arrive_expect_tx(bar_q, kQBytes);
+        tma_load_4d(sQ, &tm_q, bar_q, 0, g * p.G, static_cast<int32_t>(q0 + pos0), 0);
+      }
+      uint64_t* bar_free = is_v ? bar_pv : bar_s;   // slot reusable once S (for K) / PV (for V) is done
+      uint64_t* bar_full = is_v ? bar_v : bar_k;
+      uint8_t* ring = is_v ? sV : sK;
       for (int j = 0; j < nt && !*abort_flag; ++j) {
         const int s = j & 1;
         const bool self = j < n_self;
         const int32_t row = self ? static_cast<int32_t>(q0 + j * kBKV)
                                  : static_cast<int32_t>(c0 + (j - n_self) * kBKV);
-        const CUtensorMap* mk = self ? &tm_ks : &tm_kc;
-        const CUtensorMap* mv = self ? &tm_vs : &tm_vc;
-        if (j >= 2 && !mbar_wait(&bar_s[s], ((j - 2) >> 1) & 1, p.wait_ns)) {
+        const CUtensorMap* m = is_v ? (self ? &tm_vs : &tm_vc) : (self ? &tm_ks : &tm_kc);
+        if (j >= 2 && !mbar_wait(&bar_free[s], ((j - 2) >> 1) & 1, p.wait_ns)) {
           record_error(p.err, kErrTimeout | kSiteAttention);
           *abort_flag = 1;
           break;
         }
-        mbar_arrive_expect_tx(&bar_k[s], kKVBytes);
-        for (int q = 0; q < 4; ++q)
-          tma_load_2d(sK + s * kKVBytes + q * kKVSlab, mk, &bar_k[s], g * kD + q * 64, row);
-        if (j >= 2 && !mbar_wait(&bar_pv[s], ((j - 2) >> 1) & 1, p.wait_ns)) {
-          record_error(p.err, kErrTimeout | kSiteAttention);
-          *abort_flag = 1;
-          break;
-        }
-        mbar_arrive_expect_tx(&bar_v[s], kKVBytes);
-        for (int q = 0; q < 4; ++q)
-          tma_load_2d(sV + s * kKVBytes + q * kKVSlab, mv, &bar_v[s], g * kD + q * 64, row);
+        mbar_arrive_expect_tx(&bar_full[s], kKVBytes);
+        tma_load_3d(ring + s * kKVBytes, m, &bar_full[s], 0, row, g * 4);
       }
     }
-  } else if (warp == 5) {
+  } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       const uint32_t q_base = smem_u32(sQ), k_base = smem_u32(sK), v_base = smem_u32(sV), p_base = smem_u32(sP);
@@ -203,12 +214,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
   } else {
-    // ------------------------------------------------------------ softmax warps 0..3
-    const int r = warp * 32 + lane;          // packed row = TMEM lane
-    const int pos = pos0 + r / p.G;          // decoder position of this row
-    const int hh = r % p.G;                  // query head within the KV group
-    const uint32_t lane_base = tmem + (static_cast<uint32_t>(warp * 32) << 16);
-    float m_run = -INFINITY, l_run = 0.f;
+    // ------------------------------------------------------------ softmax warps 0..7
+    const int quarter = warp & 3;             // TMEM lane quarter
+    const int half = warp >> 2;               // which 32 of the 64 keys / 128 of the 256 O columns
+    const int r = quarter * 32 + lane;        // packed row = TMEM lane
+    const int pos = pos0 + r / p.G;           // decoder position of this row
+    const int hh = r % p.G;                   // query head within the KV group
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
+    const float c2 = p.scale_log2;
+    float m_run = -INFINITY, l_run = 0.f;     // running max (log2 units) and this half's sum
     bool ok = true;
     for (int j = 0; j < nt; ++j) {
       const int s = j & 1;
@@ -222,40 +236,47 @@ __global__ void __launch_bounds__(kThreads, 1)
       tmem_ld32(lane_base + 256u + s * kBKV, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
       tmem_ld32(lane_base + 256u + s * kBKV + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
       tmem_ld_wait();
-      // visible keys of this tile: self keys k <= pos (and < pos1 rows exist), cross keys k < Nc
-      int n_vis;
-      if (j < n_self) {
-        n_vis = pos + 1 - j * kBKV;
-      } else {
-        n_vis = Nc - (j - n_self) * kBKV;
-      }
+      // visible keys of this tile: self keys k <= pos, cross keys k < Nc
+      int n_vis = (j < n_self) ? pos + 1 - j * kBKV : Nc - (j - n_self) * kBKV;
       n_vis = max(0, min(kBKV, n_vis));
-      float x[64];
-      float mx = -INFINITY;
+      const bool masked = !__all_sync(0xffffffffu, n_vis == kBKV);
+      if (masked) {
 #pragma unroll
-      for (int k = 0; k < 64; ++k) {
-        x[k] = k < n_vis ? __uint_as_float(sr[k]) * p.scale_log2 : -INFINITY;
-        mx = fmaxf(mx, x[k]);
+        for (int k = 0; k < 64; ++k)
+          if (k >= n_vis) sr[k] = __float_as_uint(-INFINITY);
       }
+      // row max of the raw scores (scale > 0 keeps the order), as a tree
+      float t32[32];
+#pragma unroll
+      for (int k = 0; k < 32; ++k) t32[k] = fmaxf(__uint_as_float(sr[k]), __uint_as_float(sr[k + 32]));
+#pragma unroll
+      for (int w2 = 16; w2 > 0; w2 >>= 1)
+#pragma unroll
+        for (int k = 0; k < w2; ++k) t32[k] = fmaxf(t32[k], t32[k + w2]);
+      const float mx = t32[0] * c2;
       float alpha = 1.f;
       bool rescale = false;
       if (j == 0) {
         m_run = mx;  // every row sees self key 0, so mx is finite
       } else if (mx > m_run + kRescaleThreshold) {
-        alpha = exp2f(m_run - mx);
+        alpha = ex2_approx(m_run - mx);
         m_run = mx;
         rescale = true;
       }
-      float sum = 0.f;
-      uint32_t pk[32];
+      // this half's 32 probabilities: 2^(s * scale_log2 - m_run)
+      const float neg_m = -m_run;
+      float acc[4] = {0.f, 0.f, 0.f, 0.f};
+      uint32_t pk[16];
 #pragma unroll
-      for (int k = 0; k < 64; k += 2) {
-        const float e0 = exp2f(x[k] - m_run);
-        const float e1 = exp2f(x[k + 1] - m_run);
-        sum += e0 + e1;
+      for (int k = 0; k < 32; k += 2) {
+        const float s0 = __uint_as_float(half ? sr[32 + k] : sr[k]);
+        const float s1 = __uint_as_float(half ? sr[33 + k] : sr[k + 1]);
+        const float e0 = ex2_approx(fmaf(s0, c2, neg_m));
+        const float e1 = ex2_approx(fmaf(s1, c2, neg_m));
+        acc[(k >> 1) & 3] += e0 + e1;
         pk[k >> 1] = pack_bf16x2(e0, e1);
       }
-      l_run = l_run * alpha + sum;
+      l_run = l_run * alpha + ((acc[0] + acc[1]) + (acc[2] + acc[3]));
       // P stage s is free once PV_{j-2} has completed
       if (j >= 2) {
         w = mbar_wait(&bar_pv[s], ((j - 2) >> 1) & 1, p.wait_ns);
@@ -264,16 +285,16 @@ __global__ void __launch_bounds__(kThreads, 1)
           break;
         }
       }
-      // 128-byte swizzled K-major row: 16-byte chunk c of row r sits at chunk c ^ (r & 7)
+      // 128-byte swizzled K-major row: 16-byte unit u of row r sits at unit u ^ (r & 7)
       uint8_t* prow = sP + s * kPBytes + r * 128;
 #pragma unroll
-      for (int c = 0; c < 8; ++c) {
+      for (int c = 0; c < 4; ++c) {
         uint4 v;
         v.x = pk[4 * c + 0];
         v.y = pk[4 * c + 1];
         v.z = pk[4 * c + 2];
         v.w = pk[4 * c + 3];
-        *reinterpret_cast<uint4*>(prow + ((c ^ (r & 7)) << 4)) = v;
+        *reinterpret_cast<uint4*>(prow + (((half * 4 + c) ^ (r & 7)) << 4)) = v;
       }
       fence_proxy_async_smem();
       if (__any_sync(0xffffffffu, rescale)) {
@@ -285,7 +306,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tc_fence_after();
 #pragma unroll 1
-        for (int c = 0; c < kD; c += 32) {
+        for (int c = half * 128; c < half * 128 + 128; c += 32) {
           uint32_t o[32];
           tmem_ld32(lane_base + c, o);
           tmem_ld_wait();
@@ -298,79 +319,71 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_before();
       mbar_arrive(&bar_p[s]);
     }
+    // publish this half's row sum (every softmax thread arrives, also on failure)
+    l_part[half * 128 + r] = l_run;
+    mbar_arrive(bar_l);
     if (!ok) {
       if (lane == 0) record_error(p.err, kErrTimeout | kSiteAttention);
       *abort_flag = 1;
     } else {
-      // ---- epilogue: O / l -> bf16
+      // ---- epilogue: O / l -> bf16, this half's 128 columns
       const int jl = nt - 1;
-      bool w = mbar_wait(&bar_pv[jl & 1], (jl >> 1) & 1, p.wait_ns);
+      bool w = mbar_wait(&bar_pv[jl & 1], (jl >> 1) & 1, p.wait_ns) && mbar_wait(bar_l, 0, p.wait_ns);
       if (!__all_sync(0xffffffffu, w)) {
         if (lane == 0) record_error(p.err, kErrTimeout | kSiteAttention);
         *abort_flag = 1;
       } else {
         tc_fence_after();
-        const float inv_l = 1.f / l_run;
+        const float l_tot = l_part[r] + l_part[128 + r];
+        const float inv_l = 1.f / l_tot;
         const bool valid = pos < pos1;
         const int head = g * p.G + hh;
-        if (pos0 + p.P <= Lq) {
-          // Full tile: stage O as bf16 in the (now idle) Q tile, in the same
-          // 128-byte-swizzled slabs, and write it with four 3-D TMA stores whose
-          // boxes match the Q boxes (positions x heads x 64 columns).
+        const bool full_tile = pos0 + p.P <= Lq;
+        __nv_bfloat16* orow = p.out + (q0 + pos) * p.ldo + static_cast<int64_t>(head) * kD;
 #pragma unroll 1
-          for (int c = 0; c < kD; c += 32) {
-            uint32_t o[32];
-            tmem_ld32(lane_base + c, o);
-            tmem_ld_wait();
+        for (int c = half * 128; c < half * 128 + 128; c += 32) {
+          uint32_t o[32];
+          tmem_ld32(lane_base + c, o);
+          tmem_ld_wait();
+          uint4 v[4];
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            v[q].x = pack_bf16x2(__uint_as_float(o[8 * q + 0]) * inv_l, __uint_as_float(o[8 * q + 1]) * inv_l);
+            v[q].y = pack_bf16x2(__uint_as_float(o[8 * q + 2]) * inv_l, __uint_as_float(o[8 * q + 3]) * inv_l);
+            v[q].z = pack_bf16x2(__uint_as_float(o[8 * q + 4]) * inv_l, __uint_as_float(o[8 * q + 5]) * inv_l);
+            v[q].w = pack_bf16x2(__uint_as_float(o[8 * q + 6]) * inv_l, __uint_as_float(o[8 * q + 7]) * inv_l);
+          }
+          if (full_tile) {
+            // Full tile: stage O in the (now idle) Q tile, in the same 128-byte
+            // swizzled slabs; four 3-D TMA stores whose boxes match the Q boxes
+            // (positions x heads x 64 columns) write it after the CTA barrier.
             uint8_t* row = sQ + (c >> 6) * kQSlab + r * 128;
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
-              uint4 v;
-              v.x = pack_bf16x2(__uint_as_float(o[8 * q + 0]) * inv_l, __uint_as_float(o[8 * q + 1]) * inv_l);
-              v.y = pack_bf16x2(__uint_as_float(o[8 * q + 2]) * inv_l, __uint_as_float(o[8 * q + 3]) * inv_l);
-              v.z = pack_bf16x2(__uint_as_float(o[8 * q + 4]) * inv_l, __uint_as_float(o[8 * q + 5]) * inv_l);
-              v.w = pack_bf16x2(__uint_as_float(o[8 * q + 6]) * inv_l, __uint_as_float(o[8 * q + 7]) * inv_l);
               const int unit = ((c & 63) >> 3) + q;  // 16-byte unit inside the 128-byte row
-              *reinterpret_cast<uint4*>(row + ((unit ^ (r & 7)) << 4)) = v;
+              *reinterpret_cast<uint4*>(row + ((unit ^ (r & 7)) << 4)) = v[q];
             }
-          }
-          fence_proxy_async_smem();  // the TMA stores are issued after the CTA barrier below
-        } else {
-          __nv_bfloat16* orow = p.out + (q0 + pos) * p.ldo + static_cast<int64_t>(head) * kD;
-#pragma unroll 1
-          for (int c = 0; c < kD; c += 32) {
-            uint32_t o[32];
-            tmem_ld32(lane_base + c, o);
-            tmem_ld_wait();
-            if (valid) {
-              uint4* dst = reinterpret_cast<uint4*>(orow + c);
+          } else if (valid) {
+            uint4* dst = reinterpret_cast<uint4*>(orow + c);
 #pragma unroll
-              for (int q = 0; q < 4; ++q) {
-                uint4 v;
-                v.x = pack_bf16x2(__uint_as_float(o[8 * q + 0]) * inv_l, __uint_as_float(o[8 * q + 1]) * inv_l);
-                v.y = pack_bf16x2(__uint_as_float(o[8 * q + 2]) * inv_l, __uint_as_float(o[8 * q + 3]) * inv_l);
-                v.z = pack_bf16x2(__uint_as_float(o[8 * q + 4]) * inv_l, __uint_as_float(o[8 * q + 5]) * inv_l);
-                v.w = pack_bf16x2(__uint_as_float(o[8 * q + 6]) * inv_l, __uint_as_float(o[8 * q + 7]) * inv_l);
-                dst[q] = v;
-              }
-            }
+            for (int q = 0; q < 4; ++q) dst[q] = v[q];
           }
         }
-        if (valid && p.lse) {
+        if (full_tile) fence_proxy_async_smem();
+        if (valid && half == 0 && p.lse) {
           // natural-log softmax denominator in scaled-logit units
-          p.lse[(q0 + pos) * p.n_q + head] = (m_run + log2f(l_run)) * 0.69314718055994531f;
+          p.lse[(q0 + pos) * p.n_q + head] = (m_run + log2f(l_tot)) * 0.69314718055994531f;
         }
       }
     }
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == kMmaWarp) {
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
   } else if (threadIdx.x == 0 && pos0 + p.P <= Lq && !*abort_flag) {
-    for (int j = 0; j < 4; ++j)
-      tma_store_3d(&tm_o, sQ + j * kQSlab, j * 64, g * p.G, static_cast<int32_t>(q0 + pos0));
+    tma_store_4d(&tm_o, sQ, 0, g * p.G, static_cast<int32_t>(q0 + pos0), 0);
     bulk_commit_group();
     bulk_wait_group<0>();
   }
@@ -416,20 +429,24 @@ extern "C" kalm_status kalm_merged_attention(const kalm_bf16* q, int64_t ldq, co
   if (total_q > INT32_MAX - 1024 || total_pool > INT32_MAX - 1024)
     return fail(KALM_ERR_INVALID_ARG, "kalm_merged_attention: too many rows");
 
+  // Q and O: 4-D views (64 columns, head, row, 64-column slab) so one box moves a whole
+  // 128-row x 256-column tile in the slab-major order the tensor-core descriptors read.
   CUtensorMap tq, tks, tvs, tkc, tvc, to;
   {
-    const uint64_t dims[3] = {kD, static_cast<uint64_t>(n_q), static_cast<uint64_t>(total_q)};
-    const uint64_t strides[2] = {kD * 2, static_cast<uint64_t>(ldq) * 2};
-    const uint32_t box[3] = {64, static_cast<uint32_t>(G), static_cast<uint32_t>(kBM / G)};
-    if ((st = make_tmap_bf16(&tq, q, 3, dims, strides, box)) != KALM_OK) return st;
-    const uint64_t ostrides[2] = {kD * 2, static_cast<uint64_t>(ldo) * 2};
-    if ((st = make_tmap_bf16(&to, out, 3, dims, ostrides, box)) != KALM_OK) return st;
+    const uint64_t dims[4] = {64, static_cast<uint64_t>(n_q), static_cast<uint64_t>(total_q), 4};
+    const uint64_t strides[3] = {kD * 2, static_cast<uint64_t>(ldq) * 2, 128};
+    const uint32_t box[4] = {64, static_cast<uint32_t>(G), static_cast<uint32_t>(kBM / G), 4};
+    if ((st = make_tmap_bf16(&tq, q, 4, dims, strides, box)) != KALM_OK) return st;
+    const uint64_t ostrides[3] = {kD * 2, static_cast<uint64_t>(ldo) * 2, 128};
+    if ((st = make_tmap_bf16(&to, out, 4, dims, ostrides, box)) != KALM_OK) return st;
   }
+  // K and V: 3-D views (64 columns, row, 64-column slab over all KV heads); a box is
+  // one 64-key x 256-column tile of one KV head.
   auto kv_map = [&](CUtensorMap* m, const kalm_bf16* base, int64_t ld, int64_t rows) -> kalm_status {
-    const uint64_t dims[2] = {static_cast<uint64_t>(n_kv) * kD, static_cast<uint64_t>(rows > 0 ? rows : 1)};
-    const uint64_t strides[1] = {static_cast<uint64_t>(ld) * 2};
-    const uint32_t box[2] = {64, kBKV};
-    return make_tmap_bf16(m, base, 2, dims, strides, box);
+    const uint64_t dims[3] = {64, static_cast<uint64_t>(rows > 0 ? rows : 1), static_cast<uint64_t>(n_kv) * 4};
+    const uint64_t strides[2] = {static_cast<uint64_t>(ld) * 2, 128};
+    const uint32_t box[3] = {64, kBKV, 4};
+    return make_tmap_bf16(m, base, 3, dims, strides, box);
   };
   if ((st = kv_map(&tks, k_self, ld_self, total_q)) != KALM_OK) return st;
   if ((st = kv_map(&tvs, v_self, ld_self, total_q)) != KALM_OK) return st;
