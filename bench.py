@@ -50,6 +50,27 @@ def parse():
     return ap.parse_args()
 
 
+def traffic(label: str):
+    """DRAM bytes per launch of a kernel from profiles/dram_traffic.txt, or None if its
+    sources changed since the capture (the counters no longer describe this kernel)."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", "dram_traffic.txt")
+    if not os.path.exists(path):
+        return None
+    for line in open(path):
+        if line.startswith("#") or not line.strip():
+            continue
+        k, b, digest, srcs = line.split()
+        if k != label:
+            continue
+        h = hashlib.sha256()
+        for src in srcs.split(","):
+            with open(os.path.join(ROOT, src), "rb") as f:
+                h.update(f.read())
+        return int(b) if h.hexdigest()[:16] == digest else None
+    return None
+
+
 def peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -286,7 +307,7 @@ def main():
     dom = max(tensor_kernels, key=lambda k: kern[k]["share"])
     dom_ach = flops_per_launch[dom] / (kern[dom]["avg_us"] * 1e-6) / 1e12
     roofline = {"kernel": dom, "bound": "tensor", "achieved": dom_ach, "peak": pk["bf16"], "unit": "TFLOP/s",
-                "frac": dom_ach / pk["bf16"], "traffic": None,
+                "frac": dom_ach / pk["bf16"], "traffic": traffic(dom),
                 "peak_source": f"{pk['source']} dense bf16 burst (cuBLAS)"}
     pool_gbs = w["pool_bytes"] / (kern["chunk_pool"]["avg_us"] * 1e-6) / 1e9
     attn_proj_us = sum(kern[k]["avg_us"] * kern[k]["launches_per_step"] for k in
@@ -298,7 +319,7 @@ def main():
     if rank == 0:
         cb = None
         if not args.no_cpu_baseline and world == 1:
-            cb = cpu_baseline(q, args.cpu_sample_docs or 20)
+            cb = cpu_baseline(q, args.cpu_sample_docs or q.n_docs)
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
