@@ -52,6 +52,79 @@ struct LinearCfg {
   static constexpr uint32_t IDESC = idesc_bf16_f32(kBM, BN, false, false);
 };
 
+// Residual prefetch of the first two 32-column chunks of a tile (one lane per warp).
+__device__ __forceinline__ void epi_prefetch_residual(const CUtensorMap* tm_r, uint8_t* rbuf, uint64_t* rbar,
+                                                      int nch, int n0, int row0) {
+  for (int c = 0; c < 2 && c < nch; ++c) {
+    mbar_arrive_expect_tx(&rbar[c], kChunkBytes);
+    tma_load_2d(rbuf + c * kChunkBytes, tm_r, &rbar[c], n0 + c * 32, row0);
+  }
+}
+
+// Epilogue of one tile for one warp: 32 rows (TMEM lanes of this warp) x nch
+// 32-column chunks.  fp32 accumulator (+ residual) -> bf16 -> swizzled staging
+// chunk -> TMA tile store.  Returns false if a bounded wait expired.
+__device__ __forceinline__ bool epi_tile(uint32_t t_row, int nch, int n0, int row0, bool has_residual,
+                                         const CUtensorMap* tm_y, const CUtensorMap* tm_r, uint8_t* obuf,
+                                         uint8_t* rbuf, uint64_t* rbar, uint32_t& rphase, int& out_slot, int lane,
+                                         uint64_t wait_ns) {
+  // 64-byte swizzle of a 32 x 64 B chunk: 16-byte unit i of row r sits at unit i ^ ((r >> 1) & 3)
+  const uint32_t swz = static_cast<uint32_t>((lane >> 1) & 3);
+#pragma unroll 1
+  for (int c = 0; c < nch; ++c) {
+    uint32_t r[32];
+    tmem_ld32(t_row + c * 32, r);
+    tmem_ld_wait();
+    float v[32];
+#pragma unroll
+    for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
+    if (has_residual) {
+      const int b = c & 1;
+      const bool okr = mbar_wait(&rbar[b], (rphase >> b) & 1u, wait_ns);
+      rphase ^= 1u << b;
+      if (!__all_sync(0xffffffffu, okr)) return false;
+      const uint8_t* rrow = rbuf + b * kChunkBytes + lane * 64;
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const uint4 rv = *reinterpret_cast<const uint4*>(rrow + ((q ^ swz) << 4));
+        const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&rv);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const float2 f = __bfloat1622float2(h[k]);
+          v[q * 8 + 2 * k] += f.x;
+          v[q * 8 + 2 * k + 1] += f.y;
+        }
+      }
+      __syncwarp();
+      if (lane == 0 && c + 2 < nch) {  // refill this residual buffer two chunks ahead
+        mbar_arrive_expect_tx(&rbar[b], kChunkBytes);
+        tma_load_2d(rbuf + b * kChunkBytes, tm_r, &rbar[b], n0 + (c + 2) * 32, row0);
+      }
+    }
+    // the staging slot is free once the store issued from it two chunks ago has read it
+    if (lane == 0) bulk_wait_group_read<1>();
+    __syncwarp();
+    uint8_t* orow = obuf + out_slot * kChunkBytes + lane * 64;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      uint4 o;
+      o.x = pack_bf16x2(v[q * 8 + 0], v[q * 8 + 1]);
+      o.y = pack_bf16x2(v[q * 8 + 2], v[q * 8 + 3]);
+      o.z = pack_bf16x2(v[q * 8 + 4], v[q * 8 + 5]);
+      o.w = pack_bf16x2(v[q * 8 + 6], v[q * 8 + 7]);
+      *reinterpret_cast<uint4*>(orow + ((q ^ swz) << 4)) = o;
+    }
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) {
+      tma_store_2d(tm_y, obuf + out_slot * kChunkBytes, n0 + c * 32, row0);
+      bulk_commit_group();
+    }
+    out_slot ^= 1;
+  }
+  return true;
+}
+
 template <int BN>
 __global__ void __launch_bounds__(kThreads, 1)
     linear_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w,
@@ -187,84 +260,25 @@ __global__ void __launch_bounds__(kThreads, 1)
     int acc = 0;
     uint32_t acc_phase = 0;
     int out_slot = 0;
-    // 64-byte swizzle of a 32 x 64 B chunk: 16-byte unit i of row r sits at unit i ^ ((r >> 1) & 3)
-    const uint32_t swz = static_cast<uint32_t>((lane >> 1) & 3);
     for (int t = blockIdx.x; t < tiles; t += gridDim.x) {
       const int m0 = (t / n_n) * kBM, n0 = (t % n_n) * BN;
       const int row0 = m0 + quarter * 32;
       const int nch = min(BN, N - n0) / 32;
-      if (has_residual && lane == 0) {
-        for (int c = 0; c < 2 && c < nch; ++c) {
-          mbar_arrive_expect_tx(&rbar[c], kChunkBytes);
-          tma_load_2d(rbuf + c * kChunkBytes, &tm_r, &rbar[c], n0 + c * 32, row0);
-        }
-      }
+      if (has_residual && lane == 0) epi_prefetch_residual(&tm_r, rbuf, rbar, nch, n0, row0);
       bool ok = mbar_wait(&acc_full[acc], acc_phase, wait_ns);
       ok = __all_sync(0xffffffffu, ok);
+      if (ok && !*abort_flag) {
+        tc_fence_after();
+        const uint32_t t_row =
+            tmem + (static_cast<uint32_t>(quarter * 32) << 16) + static_cast<uint32_t>(acc * BN);
+        ok = epi_tile(t_row, nch, n0, row0, has_residual, &tm_y, &tm_r, obuf, rbuf, rbar, rphase, out_slot, lane,
+                      wait_ns);
+      }
       if (!ok || *abort_flag) {
         if (lane == 0) record_error(err, kErrTimeout | kSiteLinear);
         *abort_flag = 1;
         break;
       }
-      tc_fence_after();
-      const uint32_t t_row = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + static_cast<uint32_t>(acc * BN);
-#pragma unroll 1
-      for (int c = 0; c < nch; ++c) {
-        uint32_t r[32];
-        tmem_ld32(t_row + c * 32, r);
-        tmem_ld_wait();
-        float v[32];
-#pragma unroll
-        for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
-        if (has_residual) {
-          const int b = c & 1;
-          bool okr = mbar_wait(&rbar[b], (rphase >> b) & 1u, wait_ns);
-          rphase ^= 1u << b;
-          if (!__all_sync(0xffffffffu, okr)) {
-            if (lane == 0) record_error(err, kErrTimeout | kSiteLinear);
-            *abort_flag = 1;
-            break;
-          }
-          const uint8_t* rrow = rbuf + b * kChunkBytes + lane * 64;
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const uint4 rv = *reinterpret_cast<const uint4*>(rrow + ((q ^ swz) << 4));
-            const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&rv);
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-              const float2 f = __bfloat1622float2(h[k]);
-              v[q * 8 + 2 * k] += f.x;
-              v[q * 8 + 2 * k + 1] += f.y;
-            }
-          }
-          __syncwarp();
-          if (lane == 0 && c + 2 < nch) {  // refill this residual buffer two chunks ahead
-            mbar_arrive_expect_tx(&rbar[b], kChunkBytes);
-            tma_load_2d(rbuf + b * kChunkBytes, &tm_r, &rbar[b], n0 + (c + 2) * 32, row0);
-          }
-        }
-        // the staging slot is free once the store issued from it two chunks ago has read it
-        if (lane == 0) bulk_wait_group_read<1>();
-        __syncwarp();
-        uint8_t* orow = obuf + out_slot * kChunkBytes + lane * 64;
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          uint4 o;
-          o.x = pack_bf16x2(v[q * 8 + 0], v[q * 8 + 1]);
-          o.y = pack_bf16x2(v[q * 8 + 2], v[q * 8 + 3]);
-          o.z = pack_bf16x2(v[q * 8 + 4], v[q * 8 + 5]);
-          o.w = pack_bf16x2(v[q * 8 + 6], v[q * 8 + 7]);
-          *reinterpret_cast<uint4*>(orow + ((q ^ swz) << 4)) = o;
-        }
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) {
-          tma_store_2d(&tm_y, obuf + out_slot * kChunkBytes, n0 + c * 32, row0);
-          bulk_commit_group();
-        }
-        out_slot ^= 1;
-      }
-      if (*abort_flag) break;
       tc_fence_before();
       mbar_arrive(&acc_empty[acc]);
       acc ^= 1;
@@ -280,7 +294,227 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
+// ---------------------------------------------------------------------------
+// CTA-pair variant: a 2-CTA cluster computes a 256 x BN tile with tcgen05.mma
+// cta_group::2.  Each CTA fetches its own 128 rows of x and its own BN/2 rows of
+// w, so every SM moves fewer operand bytes per FLOP than a 128 x BN tile on one
+// SM; the even CTA issues the MMAs, its commits arrive on both CTAs' barriers.
+// ---------------------------------------------------------------------------
+template <int BN>
+struct Linear2Cfg {
+  static constexpr int BNH = BN / 2;
+  static constexpr int A_BYTES = kBM * kBK * 2;
+  static constexpr int B_BYTES = BNH * kBK * 2;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int EPI_BYTES = 4 * 2 * kChunkBytes;
+  static constexpr int BAR_BYTES = 256;
+  static constexpr int STAGES_FIT = (232448 - 1024 - BAR_BYTES - 2 * EPI_BYTES) / STAGE_BYTES;
+  static constexpr int STAGES = STAGES_FIT > 8 ? 8 : STAGES_FIT;
+  static constexpr int SMEM = 1024 + STAGES * STAGE_BYTES + 2 * EPI_BYTES + BAR_BYTES;
+  static constexpr uint32_t TMEM_COLS = 512;  // two accumulators at columns 0 and 256
+  static constexpr uint32_t ACC_STRIDE = 256;
+  static constexpr uint32_t IDESC = idesc_bf16_f32(2 * kBM, BN, false, false);
+  static_assert(BNH % 8 == 0, "B half-tile must be whole 8-row groups");
+};
+
+template <int BN>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+    linear_pair_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w,
+                       const __grid_constant__ CUtensorMap tm_y, const __grid_constant__ CUtensorMap tm_r,
+                       bool has_residual, int M, int N, int K, uint64_t wait_ns, uint32_t* err) {
+  using C = Linear2Cfg<BN>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + C::STAGES * C::A_BYTES;
+  uint8_t* sOut = sB + C::STAGES * C::B_BYTES;
+  uint8_t* sRes = sOut + C::EPI_BYTES;
+  uint64_t* full = reinterpret_cast<uint64_t*>(sRes + C::EPI_BYTES);  // used in the even CTA
+  uint64_t* empty = full + C::STAGES;
+  uint64_t* acc_full = empty + C::STAGES;
+  uint64_t* acc_empty = acc_full + 2;  // used in the even CTA
+  uint64_t* res_full = acc_empty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(res_full + 8);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = rank == 0;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::STAGES; ++s) {
+      mbar_init(&full[s], 2);  // the even CTA's x copy and w copy arrive with both CTAs' bytes
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&acc_full[b], 1);
+      mbar_init(&acc_empty[b], 8);  // one arrival per epilogue warp of both CTAs
+    }
+    for (int b = 0; b < 8; ++b) mbar_init(&res_full[b], 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == kMmaWarp) {
+    tmem_alloc_pair(tmem_slot, C::TMEM_COLS);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  cluster_sync_all();  // barriers of both CTAs initialised, tensor memory allocated
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  const int n_m = (M + 2 * kBM - 1) / (2 * kBM);
+  const int n_n = (N + BN - 1) / BN;
+  const int tiles = n_m * n_n;
+  const int kblocks = (K + kBK - 1) / kBK;
+  const int pair = blockIdx.x >> 1, n_pairs = gridDim.x >> 1;
+
+  if (warp < kProdWarps) {
+    if (lane == 0) {
+      const bool is_w = warp >= 2;
+      const uint32_t mine = warp & 1;
+      const CUtensorMap* tm = is_w ? &tm_w : &tm_x;
+      tma_prefetch_desc(tm);
+      const uint32_t full0 = map_to_rank(smem_u32(full), 0);  // the even CTA's full barriers
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t it = 0;
+      for (int t = pair; t < tiles && !*abort_flag; t += n_pairs) {
+        const int m0 = (t / n_n) * 2 * kBM + static_cast<int>(rank) * kBM;
+        const int n0 = (t % n_n) * BN + static_cast<int>(rank) * C::BNH;
+        for (int kb = 0; kb < kblocks; ++kb, ++it) {
+          if ((it & 1u) == mine) {
+            if (!mbar_wait(&empty[stage], phase ^ 1u, wait_ns)) {
+              record_error(err, kErrTimeout | kSiteLinear);
+              *abort_flag = 1;
+              break;
+            }
+            const uint32_t bar = full0 + stage * 8;
+            if (is_w) {
+              if (leader) mbar_arrive_expect_tx(&full[stage], 2 * C::B_BYTES);
+              tma_load_2d_pair(sB + stage * C::B_BYTES, tm, bar, kb * kBK, n0);
+            } else {
+              if (leader) mbar_arrive_expect_tx(&full[stage], 2 * C::A_BYTES);
+              tma_load_2d_pair(sA + stage * C::A_BYTES, tm, bar, kb * kBK, m0);
+            }
+          }
+          if (++stage == C::STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+    }
+  } else if (warp == kMmaWarp) {
+    if (leader && lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      const uint32_t a_base = smem_u32(sA), b_base = smem_u32(sB);
+      for (int t = pair; t < tiles && !*abort_flag; t += n_pairs) {
+        if (!mbar_wait(&acc_empty[acc], acc_phase ^ 1u, wait_ns)) {
+          record_error(err, kErrTimeout | kSiteLinear);
+          *abort_flag = 1;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem + static_cast<uint32_t>(acc) * C::ACC_STRIDE;
+        bool ok = true;
+        for (int kb = 0; kb < kblocks; ++kb) {
+          if (!mbar_wait(&full[stage], phase, wait_ns)) {
+            record_error(err, kErrTimeout | kSiteLinear);
+            *abort_flag = 1;
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a0 = a_base + stage * C::A_BYTES, b0 = b_base + stage * C::B_BYTES;
+#pragma unroll
+          for (int kk = 0; kk < kBK / 16; ++kk) {
+            const uint64_t ad = sdesc_sw128(a0 + kk * 32, 16, 1024);
+            const uint64_t bd = sdesc_sw128(b0 + kk * 32, 16, 1024);
+            umma_bf16_ss_pair(d_tmem, ad, bd, C::IDESC, (kb | kk) != 0 ? 1u : 0u);
+          }
+          umma_commit_pair_multicast(&empty[stage], 0x3);
+          if (++stage == C::STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        umma_commit_pair_multicast(&acc_full[acc], 0x3);
+        acc ^= 1;
+        if (acc == 0) acc_phase ^= 1u;
+      }
+    }
+  } else {
+    // epilogue warps: this CTA's 128 rows of the pair tile
+    const int quarter = warp & 3;
+    const int ew = warp - kEpiWarp0;
+    uint8_t* obuf = sOut + ew * 2 * kChunkBytes;
+    uint8_t* rbuf = sRes + ew * 2 * kChunkBytes;
+    uint64_t* rbar = res_full + ew * 2;
+    const uint32_t acc_empty0 = map_to_rank(smem_u32(acc_empty), 0);
+    uint32_t rphase = 0u;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    int out_slot = 0;
+    for (int t = pair; t < tiles; t += n_pairs) {
+      const int m0 = (t / n_n) * 2 * kBM + static_cast<int>(rank) * kBM, n0 = (t % n_n) * BN;
+      const int row0 = m0 + quarter * 32;
+      const int nch = min(BN, N - n0) / 32;
+      if (has_residual && lane == 0) epi_prefetch_residual(&tm_r, rbuf, rbar, nch, n0, row0);
+      bool ok = mbar_wait(&acc_full[acc], acc_phase, wait_ns);
+      ok = __all_sync(0xffffffffu, ok);
+      if (ok && !*abort_flag) {
+        tc_fence_after();
+        const uint32_t t_row =
+            tmem + (static_cast<uint32_t>(quarter * 32) << 16) + static_cast<uint32_t>(acc) * C::ACC_STRIDE;
+        ok = epi_tile(t_row, nch, n0, row0, has_residual, &tm_y, &tm_r, obuf, rbuf, rbar, rphase, out_slot, lane,
+                      wait_ns);
+      }
+      if (!ok || *abort_flag) {
+        if (lane == 0) record_error(err, kErrTimeout | kSiteLinear);
+        *abort_flag = 1;
+        break;
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(acc_empty0 + acc * 8);
+      acc ^= 1;
+      if (acc == 0) acc_phase ^= 1u;
+    }
+    if (lane == 0) bulk_wait_group<0>();
+  }
+  tc_fence_before();
+  cluster_sync_all();  // the peer's shared memory is read by the pair MMAs until here
+  if (warp == kMmaWarp) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem, C::TMEM_COLS);
+  }
+}
+
 int g_num_sms[64] = {0};
+int g_pair_slots[64][3] = {};  // co-resident CTA pairs for BN = 256, 192, 160
+
+template <int BN>
+kalm_status setup_pair(int dev, int slot) {
+  kalm_status st = check_cuda(cudaFuncSetAttribute(linear_pair_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                   Linear2Cfg<BN>::SMEM),
+                              "cudaFuncSetAttribute(linear_pair_kernel)");
+  if (st != KALM_OK) return st;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * 74, 1, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = Linear2Cfg<BN>::SMEM;
+  int clusters = 0;
+  if (cudaOccupancyMaxActiveClusters(&clusters, linear_pair_kernel<BN>, &cfg) != cudaSuccess || clusters <= 0) {
+    cudaGetLastError();
+    clusters = g_num_sms[dev] / 2;
+  }
+  g_pair_slots[dev][slot] = clusters;
+  return KALM_OK;
+}
 
 }  // namespace
 
@@ -295,10 +529,14 @@ kalm_status setup_linear_kernels() {
   if (st != KALM_OK) return st;
   int dev = 0;
   cudaGetDevice(&dev);
+  if (dev >= 64) return fail(KALM_ERR_NO_DEVICE, "device index %d out of range", dev);
   int sms = 0;
   st = check_cuda(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev), "SM count");
   if (st != KALM_OK) return st;
-  if (dev < 64) g_num_sms[dev] = sms;
+  g_num_sms[dev] = sms;
+  if ((st = setup_pair<256>(dev, 0)) != KALM_OK) return st;
+  if ((st = setup_pair<192>(dev, 1)) != KALM_OK) return st;
+  if ((st = setup_pair<160>(dev, 2)) != KALM_OK) return st;
   return KALM_OK;
 }
 
@@ -308,13 +546,69 @@ int num_sms() {
   return (dev < 64 && g_num_sms[dev] > 0) ? g_num_sms[dev] : 148;
 }
 
+namespace {
+
+int pair_slots(int slot) {
+  int dev = 0;
+  cudaGetDevice(&dev);
+  const int v = (dev < 64) ? g_pair_slots[dev][slot] : 0;
+  return v > 0 ? v : num_sms() / 2;
+}
+
+kalm_status make_operand_maps(CUtensorMap* tx, CUtensorMap* tw, CUtensorMap* ty, CUtensorMap* tr, const kalm_bf16* x,
+                              int64_t ldx, const kalm_bf16* w, int64_t ldw, const kalm_bf16* residual, int64_t ldr,
+                              kalm_bf16* y, int64_t ldy, int64_t m, int32_t n, int32_t k, uint32_t w_box_rows) {
+  kalm_status st;
+  {
+    const uint64_t dims[2] = {static_cast<uint64_t>(k), static_cast<uint64_t>(m)};
+    const uint64_t strides[1] = {static_cast<uint64_t>(ldx) * 2};
+    const uint32_t box[2] = {kBK, kBM};
+    if ((st = make_tmap_bf16(tx, x, 2, dims, strides, box)) != KALM_OK) return st;
+  }
+  {
+    const uint64_t dims[2] = {static_cast<uint64_t>(k), static_cast<uint64_t>(n)};
+    const uint64_t strides[1] = {static_cast<uint64_t>(ldw) * 2};
+    const uint32_t box[2] = {kBK, w_box_rows};
+    if ((st = make_tmap_bf16(tw, w, 2, dims, strides, box)) != KALM_OK) return st;
+  }
+  {
+    const uint64_t dims[2] = {static_cast<uint64_t>(n), static_cast<uint64_t>(m)};
+    const uint64_t strides[1] = {static_cast<uint64_t>(ldy) * 2};
+    const uint32_t box[2] = {32, 32};
+    if ((st = make_tmap_bf16(ty, y, 2, dims, strides, box, 64)) != KALM_OK) return st;
+    if (residual) {
+      const uint64_t rstrides[1] = {static_cast<uint64_t>(ldr) * 2};
+      if ((st = make_tmap_bf16(tr, residual, 2, dims, rstrides, box, 64)) != KALM_OK) return st;
+    } else {
+      *tr = *ty;  // never read
+    }
+  }
+  return KALM_OK;
+}
+
+template <int BN>
+kalm_status launch_pair(const kalm_bf16* x, int64_t ldx, const kalm_bf16* w, int64_t ldw, const kalm_bf16* residual,
+                        int64_t ldr, kalm_bf16* y, int64_t ldy, int64_t m, int32_t n, int32_t k, int slots,
+                        cudaStream_t stream) {
+  CUtensorMap tx, tw, ty, tr;
+  kalm_status st = make_operand_maps(&tx, &tw, &ty, &tr, x, ldx, w, ldw, residual, ldr, y, ldy, m, n, k, BN / 2);
+  if (st != KALM_OK) return st;
+  const int64_t tiles = ((m + 2 * kBM - 1) / (2 * kBM)) * ((n + BN - 1) / BN);
+  const int pairs = static_cast<int>(tiles < slots ? tiles : slots);
+  linear_pair_kernel<BN><<<2 * pairs, kThreads, Linear2Cfg<BN>::SMEM, stream>>>(
+      tx, tw, ty, tr, residual != nullptr, (int)m, n, k, kWaitNs, device_error_word());
+  return check_cuda(cudaGetLastError(), "launch linear_pair_kernel");
+}
+
+}  // namespace
+
 // Shared by kalm_linear and kalm_cross_kv_proj.
 kalm_status launch_linear(const kalm_bf16* x, int64_t ldx, const kalm_bf16* w, int64_t ldw, const kalm_bf16* residual,
                           int64_t ldr, kalm_bf16* y, int64_t ldy, int64_t m, int32_t n, int32_t k,
                           cudaStream_t stream, const char* who) {
   if (m < 0 || n <= 0 || k <= 0) return fail(KALM_ERR_INVALID_ARG, "%s: m=%lld n=%d k=%d", who, (long long)m, n, k);
   if (m == 0) return KALM_OK;
-  if (m > INT32_MAX - 256) return fail(KALM_ERR_INVALID_ARG, "%s: m=%lld too large", who, (long long)m);
+  if (m > INT32_MAX - 512) return fail(KALM_ERR_INVALID_ARG, "%s: m=%lld too large", who, (long long)m);
   if (!x || !w || !y) return fail(KALM_ERR_INVALID_ARG, "%s: NULL pointer", who);
   if (n % 32) return fail(KALM_ERR_UNSUPPORTED, "%s: n=%d must be a multiple of 32", who, n);
   if (k % 8) return fail(KALM_ERR_INVALID_ARG, "%s: k=%d must be a multiple of 8", who, k);
@@ -323,38 +617,33 @@ kalm_status launch_linear(const kalm_bf16* x, int64_t ldx, const kalm_bf16* w, i
     return fail(KALM_ERR_INVALID_ARG, "%s: strides must be multiples of 8 and >= the row width", who);
   if (!aligned16(x) || !aligned16(w) || !aligned16(y) || (residual && !aligned16(residual)))
     return fail(KALM_ERR_INVALID_ARG, "%s: bf16 pointers must be 16-byte aligned", who);
+  if (m >= 2 * kBM && n >= 128) {
+    // CTA-pair tiles of 256 x BN.  Time ~ rounds of co-resident pairs x (BN + fixed
+    // per-tile cost); the fixed cost, measured at the Nano projection shapes, is worth
+    // ~480 columns, so narrower tiles pay off only when they save a round.
+    const int bns[3] = {256, 192, 160};
+    const int64_t n_m = (m + 2 * kBM - 1) / (2 * kBM);
+    int best = 0;
+    int64_t best_cost = INT64_MAX;
+    for (int i = 0; i < 3; ++i) {
+      const int64_t tiles = n_m * ((n + bns[i] - 1) / bns[i]);
+      const int64_t slots = pair_slots(i);
+      const int64_t cost = ((tiles + slots - 1) / slots) * (bns[i] + 480);
+      if (cost < best_cost) {
+        best_cost = cost;
+        best = i;
+      }
+    }
+    const int slots = pair_slots(best);
+    if (best == 0) return launch_pair<256>(x, ldx, w, ldw, residual, ldr, y, ldy, m, n, k, slots, stream);
+    if (best == 1) return launch_pair<192>(x, ldx, w, ldw, residual, ldr, y, ldy, m, n, k, slots, stream);
+    return launch_pair<160>(x, ldx, w, ldw, residual, ldr, y, ldy, m, n, k, slots, stream);
+  }
   const bool wide = (n % 256) == 0;
   const int BN = wide ? 256 : 128;
-  CUtensorMap tx, tw;
-  {
-    const uint64_t dims[2] = {static_cast<uint64_t>(k), static_cast<uint64_t>(m)};
-    const uint64_t strides[1] = {static_cast<uint64_t>(ldx) * 2};
-    const uint32_t box[2] = {kBK, kBM};
-    kalm_status st = make_tmap_bf16(&tx, x, 2, dims, strides, box);
-    if (st != KALM_OK) return st;
-  }
-  {
-    const uint64_t dims[2] = {static_cast<uint64_t>(k), static_cast<uint64_t>(n)};
-    const uint64_t strides[1] = {static_cast<uint64_t>(ldw) * 2};
-    const uint32_t box[2] = {kBK, static_cast<uint32_t>(BN)};
-    kalm_status st = make_tmap_bf16(&tw, w, 2, dims, strides, box);
-    if (st != KALM_OK) return st;
-  }
-  CUtensorMap ty, tr;
-  {
-    const uint64_t dims[2] = {static_cast<uint64_t>(n), static_cast<uint64_t>(m)};
-    const uint64_t strides[1] = {static_cast<uint64_t>(ldy) * 2};
-    const uint32_t box[2] = {32, 32};
-    kalm_status st = make_tmap_bf16(&ty, y, 2, dims, strides, box, 64);
-    if (st != KALM_OK) return st;
-    if (residual) {
-      const uint64_t rstrides[1] = {static_cast<uint64_t>(ldr) * 2};
-      st = make_tmap_bf16(&tr, residual, 2, dims, rstrides, box, 64);
-      if (st != KALM_OK) return st;
-    } else {
-      tr = ty;  // never read
-    }
-  }
+  CUtensorMap tx, tw, ty, tr;
+  kalm_status st = make_operand_maps(&tx, &tw, &ty, &tr, x, ldx, w, ldw, residual, ldr, y, ldy, m, n, k, BN);
+  if (st != KALM_OK) return st;
   const int64_t tiles = ((m + kBM - 1) / kBM) * ((n + BN - 1) / BN);
   const int grid = static_cast<int>(tiles < num_sms() ? tiles : num_sms());
   const bool has_r = residual != nullptr;
