@@ -98,18 +98,23 @@ def kalm_cross_kv_proj(pooled: torch.Tensor, w_kv: torch.Tensor, kv_cross: torch
 def kalm_merged_attention(q: torch.Tensor, k_self: torch.Tensor, v_self: torch.Tensor, k_cross: torch.Tensor,
                           v_cross: torch.Tensor, q_off: torch.Tensor, pool_off: torch.Tensor, max_q: int,
                           n_q: int, n_kv: int, out: torch.Tensor, scale: Optional[float] = None,
-                          lse: Optional[torch.Tensor] = None, head_dim: int = HEAD_DIM, stream=None) -> None:
-    """2-D row views: q/out [rows][>= n_q*D], k/v self [rows][>= n_kv*D], k/v cross [pooled rows][>= n_kv*D]."""
+                          lse: Optional[torch.Tensor] = None, head_dim: int = HEAD_DIM,
+                          in_off: Optional[torch.Tensor] = None, last_tile_only: bool = False,
+                          total_q: Optional[int] = None, stream=None) -> None:
+    """2-D row views: q/k/v self [input rows][...], out [q_off[-1] rows][>= n_q*D],
+    k/v cross [pooled rows][>= n_kv*D].  ``in_off`` (optional) gives each document's
+    first input row; by default it is q_off."""
     if scale is None:
         scale = head_dim ** -0.5
     if _ld(k_self) != _ld(v_self) or _ld(k_cross) != _ld(v_cross):
         raise KalmError(1, "kalm_merged_attention", "K and V views must share a row stride")
     n_docs = q_off.numel() - 1
+    total_q = out.shape[0] if total_q is None else total_q
     call("kalm_merged_attention", _p(q, torch.bfloat16), _ld(q), _p(k_self, torch.bfloat16),
          _p(v_self, torch.bfloat16), _ld(k_self), _p(k_cross, torch.bfloat16), _p(v_cross, torch.bfloat16),
-         _ld(k_cross), _p(q_off, torch.int64), _p(pool_off, torch.int64), n_docs, int(max_q), q.shape[0],
-         k_cross.shape[0], n_q, n_kv, head_dim, float(scale), _p(out, torch.bfloat16), _ld(out),
-         _p(lse, torch.float32), _stream(stream))
+         _ld(k_cross), _p(q_off, torch.int64), _p(in_off, torch.int64), q.shape[0], _p(pool_off, torch.int64),
+         n_docs, int(max_q), int(total_q), k_cross.shape[0], n_q, n_kv, head_dim, float(scale),
+         1 if last_tile_only else 0, _p(out, torch.bfloat16), _ld(out), _p(lse, torch.float32), _stream(stream))
 
 
 def kalm_yes_no_score(hidden: torch.Tensor, q_off: torch.Tensor, w_yes: torch.Tensor, w_no: torch.Tensor,

@@ -30,8 +30,8 @@ SIGNATURES = {
     "kalm_chunk_pool": [c_vp, c_i64, c_vp, c_vp, c_i32, c_i32, c_i32, c_vp, c_i64, c_vp, c_i64, c_vp],
     "kalm_linear": [c_vp, c_i64, c_vp, c_i64, c_vp, c_i64, c_vp, c_i64, c_i64, c_i32, c_i32, c_vp],
     "kalm_cross_kv_proj": [c_vp, c_i64, c_i64, c_i32, c_vp, c_i32, c_i32, c_i32, c_vp, c_vp],
-    "kalm_merged_attention": [c_vp, c_i64, c_vp, c_vp, c_i64, c_vp, c_vp, c_i64, c_vp, c_vp, c_i32, c_i32,
-                              c_i64, c_i64, c_i32, c_i32, c_i32, c_f32, c_vp, c_i64, c_vp, c_vp],
+    "kalm_merged_attention": [c_vp, c_i64, c_vp, c_vp, c_i64, c_vp, c_vp, c_i64, c_vp, c_vp, c_i64, c_vp, c_i32,
+                              c_i32, c_i64, c_i64, c_i32, c_i32, c_i32, c_f32, c_i32, c_vp, c_i64, c_vp, c_vp],
     "kalm_yes_no_score": [c_vp, c_i64, c_vp, c_i32, c_i32, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp],
     "kalm_broadcast_rows": [c_vp, c_i64, c_i32, c_i32, c_vp, c_i32, c_vp, c_i64, c_vp],
     "kalm_selftest_wait_timeout": [c_u64, c_vp],

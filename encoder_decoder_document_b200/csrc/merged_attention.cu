@@ -63,6 +63,8 @@ constexpr float kRescaleThreshold = 8.0f;      // log2 units
 
 struct AttnParams {
   const int64_t* q_off;
+  const int64_t* in_off;  // first q / self-K/V row of each document; NULL: q_off
+  int last_only;          // compute only the query tile holding each document's last row
   const int64_t* pool_off;
   __nv_bfloat16* out;
   float* lse;
@@ -85,12 +87,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                             const AttnParams p) {
   // ---- work item: heaviest query tiles (largest t) first
   const int per_t = p.n_docs * p.n_kv;
-  const int t = p.tiles_per_doc - 1 - static_cast<int>(blockIdx.x) / per_t;
   const int rem = static_cast<int>(blockIdx.x) % per_t;
   const int g = rem % p.n_kv;
   const int d = rem / p.n_kv;
-  const int64_t q0 = p.q_off[d];
+  const int64_t q0 = p.q_off[d];                      // output rows
   const int Lq = static_cast<int>(p.q_off[d + 1] - q0);
+  const int64_t qi = p.in_off ? p.in_off[d] : q0;     // input (q, self K/V) rows
+  const int t = p.last_only ? (Lq > 0 ? (Lq - 1) / p.P : 0)
+                            : p.tiles_per_doc - 1 - static_cast<int>(blockIdx.x) / per_t;
   const int64_t c0 = p.pool_off[d];
   const int Nc = static_cast<int>(p.pool_off[d + 1] - c0);
   const int pos0 = t * p.P;
@@ -147,7 +151,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool is_v = warp == kTmaWarpV;
       if (!is_v) {
         mbar_arrive_expect_tx(bar_q, kQBytes);
-        tma_load_4d(sQ, &tm_q, bar_q, 0, g * p.G, static_cast<int32_t>(q0 + pos0), 0);
+        tma_load_4d(sQ, &tm_q, bar_q, 0, g * p.G, static_cast<int32_t>(qi + pos0), 0);
       }
       uint64_t* bar_free = is_v ? bar_pv : bar_s;   // slot reusable once S (for K) / PV (for V) is done
       uint64_t* bar_full = is_v ? bar_v : bar_k;
@@ -155,7 +159,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int j = 0; j < nt && !*abort_flag; ++j) {
         const int s = j & 1;
         const bool self = j < n_self;
-        const int32_t row = self ? static_cast<int32_t>(q0 + j * kBKV)
+        const int32_t row = self ? static_cast<int32_t>(qi + j * kBKV)
                                  : static_cast<int32_t>(c0 + (j - n_self) * kBKV);
         const CUtensorMap* m = is_v ? (self ? &tm_vs : &tm_vc) : (self ? &tm_ks : &tm_kc);
         if (j >= 2 && !mbar_wait(&bar_free[s], ((j - 2) >> 1) & 1, p.wait_ns)) {
@@ -403,9 +407,10 @@ using namespace kalm;
 extern "C" kalm_status kalm_merged_attention(const kalm_bf16* q, int64_t ldq, const kalm_bf16* k_self,
                                              const kalm_bf16* v_self, int64_t ld_self, const kalm_bf16* k_cross,
                                              const kalm_bf16* v_cross, int64_t ld_cross, const int64_t* q_off,
-                                             const int64_t* pool_off, int32_t n_docs, int32_t max_q,
-                                             int64_t total_q, int64_t total_pool, int32_t n_q, int32_t n_kv,
-                                             int32_t head_dim, float scale, kalm_bf16* out, int64_t ldo, float* lse,
+                                             const int64_t* in_off, int64_t total_in, const int64_t* pool_off,
+                                             int32_t n_docs, int32_t max_q, int64_t total_q, int64_t total_pool,
+                                             int32_t n_q, int32_t n_kv, int32_t head_dim, float scale,
+                                             int32_t last_tile_only, kalm_bf16* out, int64_t ldo, float* lse,
                                              kalm_stream_t stream) {
   kalm_status st = ensure_device(nullptr);
   if (st != KALM_OK) return st;
@@ -426,19 +431,22 @@ extern "C" kalm_status kalm_merged_attention(const kalm_bf16* q, int64_t ldq, co
   if (!aligned16(q) || !aligned16(k_self) || !aligned16(v_self) || !aligned16(out) ||
       (total_pool > 0 && (!aligned16(k_cross) || !aligned16(v_cross))))
     return fail(KALM_ERR_INVALID_ARG, "kalm_merged_attention: bf16 pointers must be 16-byte aligned");
-  if (total_q > INT32_MAX - 1024 || total_pool > INT32_MAX - 1024)
+  if (!in_off) total_in = total_q;
+  if (total_in <= 0) return fail(KALM_ERR_INVALID_ARG, "kalm_merged_attention: total_in=%lld", (long long)total_in);
+  if (total_q > INT32_MAX - 1024 || total_pool > INT32_MAX - 1024 || total_in > INT32_MAX - 1024)
     return fail(KALM_ERR_INVALID_ARG, "kalm_merged_attention: too many rows");
 
   // Q and O: 4-D views (64 columns, head, row, 64-column slab) so one box moves a whole
   // 128-row x 256-column tile in the slab-major order the tensor-core descriptors read.
   CUtensorMap tq, tks, tvs, tkc, tvc, to;
   {
-    const uint64_t dims[4] = {64, static_cast<uint64_t>(n_q), static_cast<uint64_t>(total_q), 4};
+    const uint64_t dims[4] = {64, static_cast<uint64_t>(n_q), static_cast<uint64_t>(total_in), 4};
     const uint64_t strides[3] = {kD * 2, static_cast<uint64_t>(ldq) * 2, 128};
     const uint32_t box[4] = {64, static_cast<uint32_t>(G), static_cast<uint32_t>(kBM / G), 4};
     if ((st = make_tmap_bf16(&tq, q, 4, dims, strides, box)) != KALM_OK) return st;
+    const uint64_t odims[4] = {64, static_cast<uint64_t>(n_q), static_cast<uint64_t>(total_q), 4};
     const uint64_t ostrides[3] = {kD * 2, static_cast<uint64_t>(ldo) * 2, 128};
-    if ((st = make_tmap_bf16(&to, out, 4, dims, ostrides, box)) != KALM_OK) return st;
+    if ((st = make_tmap_bf16(&to, out, 4, odims, ostrides, box)) != KALM_OK) return st;
   }
   // K and V: 3-D views (64 columns, row, 64-column slab over all KV heads); a box is
   // one 64-key x 256-column tile of one KV head.
@@ -448,18 +456,20 @@ extern "C" kalm_status kalm_merged_attention(const kalm_bf16* q, int64_t ldq, co
     const uint32_t box[3] = {64, kBKV, 4};
     return make_tmap_bf16(m, base, 3, dims, strides, box);
   };
-  if ((st = kv_map(&tks, k_self, ld_self, total_q)) != KALM_OK) return st;
-  if ((st = kv_map(&tvs, v_self, ld_self, total_q)) != KALM_OK) return st;
+  if ((st = kv_map(&tks, k_self, ld_self, total_in)) != KALM_OK) return st;
+  if ((st = kv_map(&tvs, v_self, ld_self, total_in)) != KALM_OK) return st;
   // with no cross rows at all, the cross maps are never read; point them at the self tensors
   if ((st = kv_map(&tkc, total_pool > 0 ? k_cross : k_self, total_pool > 0 ? ld_cross : ld_self,
-                   total_pool > 0 ? total_pool : total_q)) != KALM_OK)
+                   total_pool > 0 ? total_pool : total_in)) != KALM_OK)
     return st;
   if ((st = kv_map(&tvc, total_pool > 0 ? v_cross : v_self, total_pool > 0 ? ld_cross : ld_self,
-                   total_pool > 0 ? total_pool : total_q)) != KALM_OK)
+                   total_pool > 0 ? total_pool : total_in)) != KALM_OK)
     return st;
 
   AttnParams prm;
   prm.q_off = q_off;
+  prm.in_off = in_off;
+  prm.last_only = last_tile_only ? 1 : 0;
   prm.pool_off = pool_off;
   prm.out = reinterpret_cast<__nv_bfloat16*>(out);
   prm.lse = lse;
@@ -473,7 +483,7 @@ extern "C" kalm_status kalm_merged_attention(const kalm_bf16* q, int64_t ldq, co
   prm.scale_log2 = scale * 1.4426950408889634f;
   prm.wait_ns = kWaitNs;
   prm.err = device_error_word();
-  const int64_t grid = static_cast<int64_t>(prm.tiles_per_doc) * n_docs * n_kv;
+  const int64_t grid = static_cast<int64_t>(last_tile_only ? 1 : prm.tiles_per_doc) * n_docs * n_kv;
   if (grid > INT32_MAX) return fail(KALM_ERR_INVALID_ARG, "kalm_merged_attention: grid too large");
   merged_attention_kernel<<<static_cast<unsigned>(grid), kThreads, kSmem, static_cast<cudaStream_t>(stream)>>>(
       tq, tks, tvs, tkc, tvc, to, prm);

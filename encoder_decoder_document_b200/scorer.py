@@ -52,13 +52,22 @@ class DeviceWeights:
 
 
 class FBNLScorer:
-    def __init__(self, weights: DeviceWeights, n_q: int, n_kv: int, chunk: int = 4, head_dim: int = HEAD_DIM):
+    """Scores one query's documents.  With ``prune`` (the default) work that
+    cannot reach the score is skipped, exactly: the first layer's Q/K/V are
+    computed once for the query's common decoder input (every document starts
+    from it), and the last layer computes attention only for the query tile that
+    holds each document's final row and the output projection only for that row
+    (the readout reads nothing else)."""
+
+    def __init__(self, weights: DeviceWeights, n_q: int, n_kv: int, chunk: int = 4, head_dim: int = HEAD_DIM,
+                 prune: bool = True):
         kalm_device_check()
         self.w = weights
         self.L, qkv_rows, self.H = weights.w_qkv.shape
         self.n_q, self.n_kv, self.D, self.chunk = n_q, n_kv, head_dim, chunk
         assert qkv_rows == (n_q + 2 * n_kv) * head_dim
         self.scale = head_dim ** -0.5
+        self.prune = prune
         self._shape = None
         self.graph: Optional[torch.cuda.CUDAGraph] = None
         # optional per-launch timing: (label, event) recorded after every entry-point call
@@ -84,6 +93,7 @@ class FBNLScorer:
         self.tok_off = torch.empty(n_docs + 1, dtype=torch.int64, **kw)
         self.pool_off = torch.empty(n_docs + 1, dtype=torch.int64, **kw)
         self.q_off = torch.empty(n_docs + 1, dtype=torch.int64, **kw)
+        self.zero_off = torch.zeros(n_docs, dtype=torch.int64, **kw)
         self.pooled = torch.empty(max(total_pooled, 1), H, dtype=torch.bfloat16, **kw)
         self.kv_cross = torch.empty(max(total_pooled, 1), L * 2 * self.n_kv * D, dtype=torch.bfloat16, **kw)
         self.qkv = torch.empty(rows, (self.n_q + 2 * self.n_kv) * D, dtype=torch.bfloat16, **kw)
@@ -147,6 +157,32 @@ class FBNLScorer:
         self.layer_attention(l)
         self.layer_out(l)
 
+    def layer_pruned(self, l: int) -> None:
+        """Layer l with the exact pruning described in the class docstring."""
+        first, last = l == 0, l == self.L - 1
+        Lq = self.lq
+        kc, vc = self.cross_views(l)
+        if first:
+            # every document's decoder input is the query's common input: one Q|K|V for all
+            kalm_linear(self.x0, self.w.w_qkv[l], self.qkv[:Lq])
+            self._mark("qkv_proj")
+            q, ks, vs = (t[:Lq] for t in self.qkv_views())
+            in_off = self.zero_off
+        else:
+            self.layer_qkv(l)
+            q, ks, vs = self.qkv_views()
+            in_off = None
+        kalm_merged_attention(q, ks, vs, kc, vc, self.q_off, self.pool_off, Lq, self.n_q, self.n_kv, self.o,
+                              self.scale, in_off=in_off, last_tile_only=last)
+        self._mark("merged_attention")
+        if last:
+            # only each document's final row reaches the readout
+            x_last = self.x[Lq - 1::Lq]
+            kalm_linear(self.o[Lq - 1::Lq], self.w.w_o[l], x_last, residual=x_last)
+            self._mark("o_proj")
+        else:
+            self.layer_out(l)
+
     def readout(self) -> None:
         kalm_yes_no_score(self.x, self.q_off, self.w.w_yes, self.w.w_no, self.yes, self.no, self.score,
                           self.margin)
@@ -163,7 +199,10 @@ class FBNLScorer:
         kalm_broadcast_rows(self.x0, self.q_off, self.x)
         self._mark("broadcast")
         for l in range(self.L):
-            self.layer(l)
+            if self.prune:
+                self.layer_pruned(l)
+            else:
+                self.layer(l)
         self.readout()
 
     def capture(self, instrument: bool = False) -> None:

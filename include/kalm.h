@@ -131,8 +131,8 @@ kalm_status kalm_chunk_pool(const kalm_bf16* enc, int64_t enc_ld, const int64_t*
  * x        [m][ldx] bf16 (m rows of k values)
  * w        [n][ldw] bf16, the nn.Linear layout [out][in]
  * residual [m][ldr] bf16 or NULL; added before the single rounding to bf16.
- *          It may alias y (same pointer and stride): each element is read
- *          before it is written by the same thread.
+ *          It may alias y (same pointer and stride): every output tile reads
+ *          its residual tile before it writes that tile.
  * y        [m][ldy] bf16
  * Requirements: m >= 0, n % 32 == 0, k % 8 == 0, k >= 8. */
 kalm_status kalm_linear(const kalm_bf16* x, int64_t ldx, const kalm_bf16* w, int64_t ldw,
@@ -169,15 +169,26 @@ kalm_status kalm_cross_kv_proj(const kalm_bf16* pooled, int64_t pooled_ld, int64
  * one softmax over both segments (causal self part, diagonal included; cross
  * part unmasked).  The concatenation is never materialised.
  *
- * q       [q_off[n_docs]][ldq] bf16; row q_off[d]+i, head h at element h*head_dim
- * k_self, v_self  [q_off[n_docs]][ld_self] bf16; KV head g at element g*head_dim
+ * q       [rows][ldq] bf16; row in(d)+i, head h at element h*head_dim
+ * k_self, v_self  [rows][ld_self] bf16; KV head g at element g*head_dim
  * k_cross, v_cross [pool_off[n_docs]][ld_cross] bf16; KV head g at g*head_dim
- * q_off   int64[n_docs+1] (decoder rows of document d: q_off[d] .. q_off[d+1]-1)
+ * q_off   int64[n_docs+1]: document d has Lq[d] = q_off[d+1]-q_off[d] decoder
+ *         rows; its outputs go to rows q_off[d] .. q_off[d+1]-1 of `out`
+ * in_off  int64[n_docs] or NULL: first row in(d) of document d's q / k_self /
+ *         v_self rows (NULL: in(d) = q_off[d]).  Documents may share input rows
+ *         (e.g. in_off all zero when every document's decoder input is the same,
+ *         as in the first decoder layer, where all documents start from the
+ *         query's common input).  total_in = number of input rows (ignored when
+ *         in_off is NULL).
  * pool_off int64[n_docs+1] (cross rows of document d: pool_off[d] .. pool_off[d+1]-1)
  * max_q   host upper bound of Lq[d] (<= KALM_MAX_QUERY_TOKENS); sizes the grid
  * total_q = q_off[n_docs], total_pool = pool_off[n_docs] (host-known; bound the
  *         tensor views)
  * scale   logit scale (1/sqrt(head_dim) for the standard attention)
+ * last_tile_only  nonzero: compute only the 128-row query tile (128/(n_q/n_kv)
+ *         positions) that holds each document's last decoder row; the other
+ *         rows of `out` are left untouched.  Enough when only the final
+ *         position is read afterwards (the yes/no readout of the last layer).
  * out     [total_q][ldo] bf16, head h at element h*head_dim
  * lse     fp32 [total_q][n_q] or NULL: natural log of each row's softmax
  *         denominator, in scaled-logit units.
@@ -186,10 +197,11 @@ kalm_status kalm_cross_kv_proj(const kalm_bf16* pooled, int64_t pooled_ld, int64
 kalm_status kalm_merged_attention(const kalm_bf16* q, int64_t ldq,
                                   const kalm_bf16* k_self, const kalm_bf16* v_self, int64_t ld_self,
                                   const kalm_bf16* k_cross, const kalm_bf16* v_cross, int64_t ld_cross,
-                                  const int64_t* q_off, const int64_t* pool_off, int32_t n_docs,
-                                  int32_t max_q, int64_t total_q, int64_t total_pool,
+                                  const int64_t* q_off, const int64_t* in_off, int64_t total_in,
+                                  const int64_t* pool_off, int32_t n_docs, int32_t max_q,
+                                  int64_t total_q, int64_t total_pool,
                                   int32_t n_q, int32_t n_kv, int32_t head_dim, float scale,
-                                  kalm_bf16* out, int64_t ldo, float* lse,
+                                  int32_t last_tile_only, kalm_bf16* out, int64_t ldo, float* lse,
                                   kalm_stream_t stream);
 
 /* Step 4 - yes/no readout at each document's final decoder position.

@@ -267,6 +267,45 @@ def test_merged_attention_batch_composition(kalm):
     np.testing.assert_array_equal(alone, got[r0:r1])
 
 
+def test_merged_attention_shared_inputs_and_last_tile(kalm):
+    """Documents that share their q / self-K/V rows (the first decoder layer, where
+    every document starts from the query's common input) and the last-tile-only mode."""
+    D, n_q, n_kv, Lq = 256, 4, 1, 70
+    nc = np.array([5, 130, 0, 64])
+    n = len(nc)
+    rng = np.random.default_rng(34)
+    q = rand_bf16(rng, (Lq, n_q, D), 0.5)
+    ks = rand_bf16(rng, (Lq, n_kv, D), 0.5)
+    vs = rand_bf16(rng, (Lq, n_kv, D))
+    C = int(nc.sum())
+    kc = rand_bf16(rng, (C, n_kv, D), 0.5)
+    vc = rand_bf16(rng, (C, n_kv, D))
+    q_off = np.arange(n + 1) * Lq
+    p_off = np.concatenate([[0], np.cumsum(nc)])
+    qkv = torch.cat([f64_to_dev(q.reshape(Lq, -1)), f64_to_dev(ks.reshape(Lq, -1)), f64_to_dev(vs.reshape(Lq, -1))], 1)
+    kvc = torch.cat([f64_to_dev(kc.reshape(C, -1)), f64_to_dev(vc.reshape(C, -1))], 1)
+    w = n_kv * D
+    # the oracle sees every document with its own copy of the shared rows
+    rep = lambda a: np.concatenate([a] * n)
+    want, _ = oracle.merged_attention(rep(q), rep(ks), rep(vs), kc, vc, q_off, p_off, 1.0 / 16)
+    for last_only in (False, True):
+        out = torch.full((n * Lq, n_q * D), float("nan"), dtype=torch.bfloat16, device="cuda")
+        kalm.kalm_merged_attention(qkv[:, : n_q * D], qkv[:, n_q * D: n_q * D + w], qkv[:, n_q * D + w:],
+                                   kvc[:, :w], kvc[:, w:], i64(q_off), i64(p_off), Lq, n_q, n_kv, out, 1.0 / 16,
+                                   in_off=i64(np.zeros(n)), last_tile_only=last_only)
+        kalm.kalm_check_device_errors()
+        got = from_dev(out).reshape(n * Lq, n_q, D)
+        if not last_only:
+            _check_attn(got, want.reshape(n * Lq, n_q, D))
+        else:
+            P = 128 // (n_q // n_kv)
+            first = ((Lq - 1) // P) * P  # first position of the tile holding row Lq-1
+            for d in range(n):
+                rows = slice(d * Lq + first, (d + 1) * Lq)
+                _check_attn(got[rows], want[rows])
+                assert np.isnan(got[d * Lq: d * Lq + first]).all()  # untouched
+
+
 # ---------------------------------------------------------------------------
 # step 4: readout
 # ---------------------------------------------------------------------------
@@ -356,6 +395,22 @@ def test_end_to_end_tiny_batch_composition(kalm):
         sc = _scorer(synthetic.Query(q.name, q.hidden, q.n_q, q.n_kv, q.head_dim, q.layers, q.doc_len[d:d + 1],
                                      np.array([0, b - a]), q.enc[a:b], q.lq, q.x0, q.weights))
         assert sc.scores_to_host().numpy()[3][0] == full[d]
+
+
+@pytest.mark.parametrize("name,layers", [("tiny", 1), ("tiny", 3), ("nano", 2)])
+def test_pruned_stack_matches_full_stack(kalm, name, layers):
+    """Skipping work that cannot reach the score changes no score."""
+    from encoder_decoder_document_b200.scorer import DeviceWeights, FBNLScorer
+    q = synthetic.make_query(name, layers=layers)
+    res = []
+    for prune in (False, True):
+        sc = FBNLScorer(DeviceWeights.from_bits(q.weights), q.n_q, q.n_kv, prune=prune)
+        sc.rerank(q.x0, q.enc, q.doc_len)
+        kalm.kalm_check_device_errors()
+        res.append(sc.scores_to_host().numpy())
+    assert np.abs(res[0] - res[1]).max() <= 1e-6
+    y, n, m, s = oracle.forward_query(q)
+    assert np.abs(res[1][3] - s).max() <= SCORE_TOL
 
 
 @pytest.mark.slow
