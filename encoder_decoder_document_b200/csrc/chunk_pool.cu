@@ -33,6 +33,8 @@ __global__ void __launch_bounds__(256) chunk_pool_kernel(const uint4* __restrict
                                                          int chunk_rt, uint4* __restrict__ pooled,
                                                          int64_t pooled_ld_v, const int64_t* __restrict__ pool_off,
                                                          int64_t total_vec, uint32_t* err) {
+  pdl_launch_dependents();
+  pdl_wait_predecessor();
   const int chunk = CHUNK > 0 ? CHUNK : chunk_rt;
   for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total_vec;
        i += (int64_t)gridDim.x * blockDim.x) {
@@ -126,11 +128,10 @@ extern "C" kalm_status kalm_chunk_pool(const kalm_bf16* enc, int64_t enc_ld, con
   uint32_t* err = device_error_word();
   const uint4* e = reinterpret_cast<const uint4*>(enc);
   uint4* p = reinterpret_cast<uint4*>(pooled);
-  if (chunk == 4)
-    chunk_pool_kernel<4><<<(unsigned)blocks, 256, 0, s>>>(e, enc_ld / 8, tok_off, len, n_docs, vpr, chunk, p,
-                                                          pooled_ld / 8, pool_off, total_vec, err);
-  else
-    chunk_pool_kernel<0><<<(unsigned)blocks, 256, 0, s>>>(e, enc_ld / 8, tok_off, len, n_docs, vpr, chunk, p,
-                                                          pooled_ld / 8, pool_off, total_vec, err);
-  return check_cuda(cudaGetLastError(), "launch chunk_pool_kernel");
+  const cudaError_t ce =
+      chunk == 4 ? launch_pdl(chunk_pool_kernel<4>, dim3((unsigned)blocks), dim3(256), 0, s, e, enc_ld / 8, tok_off,
+                              len, n_docs, vpr, chunk, p, pooled_ld / 8, pool_off, total_vec, err)
+                 : launch_pdl(chunk_pool_kernel<0>, dim3((unsigned)blocks), dim3(256), 0, s, e, enc_ld / 8, tok_off,
+                              len, n_docs, vpr, chunk, p, pooled_ld / 8, pool_off, total_vec, err);
+  return check_cuda(ce, "launch chunk_pool_kernel");
 }

@@ -140,6 +140,8 @@ namespace {
 __global__ void __launch_bounds__(1024) ragged_offsets_kernel(const int32_t* __restrict__ len, int32_t n,
                                                               int32_t chunk, int64_t* __restrict__ tok_off,
                                                               int64_t* __restrict__ pool_off, uint32_t* err) {
+  pdl_launch_dependents();
+  pdl_wait_predecessor();
   __shared__ int64_t warp_tok[32];
   __shared__ int64_t warp_pool[32];
   __shared__ int64_t carry[2];
@@ -215,6 +217,8 @@ __global__ void __launch_bounds__(1024) ragged_offsets_kernel(const int32_t* __r
 __global__ void broadcast_rows_kernel(const uint4* __restrict__ src, int64_t ld_src_v, int32_t rows, int32_t width_v,
                                       const int64_t* __restrict__ q_off, int32_t n_docs, uint4* __restrict__ dst,
                                       int64_t ld_dst_v) {
+  pdl_launch_dependents();
+  pdl_wait_predecessor();
   const int d = blockIdx.y;
   const int64_t r0 = q_off[d];
   int64_t nr = q_off[d + 1] - r0;
@@ -290,9 +294,9 @@ kalm_status kalm_ragged_offsets(const int32_t* len, int32_t n, int32_t chunk, in
   if (n < 0 || chunk < 1) return fail(KALM_ERR_INVALID_ARG, "kalm_ragged_offsets: n=%d chunk=%d", n, chunk);
   if (n > 0 && !len) return fail(KALM_ERR_INVALID_ARG, "kalm_ragged_offsets: len is NULL");
   if (!tok_off && !pool_off) return KALM_OK;
-  ragged_offsets_kernel<<<1, 1024, 0, static_cast<cudaStream_t>(stream)>>>(len, n, chunk, tok_off, pool_off,
-                                                                           device_error_word());
-  return check_cuda(cudaGetLastError(), "launch ragged_offsets_kernel");
+  return check_cuda(launch_pdl(ragged_offsets_kernel, dim3(1), dim3(1024), 0, static_cast<cudaStream_t>(stream), len,
+                                n, chunk, tok_off, pool_off, device_error_word()),
+                    "launch ragged_offsets_kernel");
 }
 
 kalm_status kalm_broadcast_rows(const kalm_bf16* src, int64_t ld_src, int32_t rows, int32_t width,
@@ -312,10 +316,10 @@ kalm_status kalm_broadcast_rows(const kalm_bf16* src, int64_t ld_src, int32_t ro
   int bx = (int)((per_doc + 255) / 256);
   if (bx > 64) bx = 64;
   dim3 grid(bx, n_docs);
-  broadcast_rows_kernel<<<grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(
-      reinterpret_cast<const uint4*>(src), ld_src / 8, rows, wv, q_off, n_docs, reinterpret_cast<uint4*>(dst),
-      ld_dst / 8);
-  return check_cuda(cudaGetLastError(), "launch broadcast_rows_kernel");
+  return check_cuda(launch_pdl(broadcast_rows_kernel, grid, dim3(256), 0, static_cast<cudaStream_t>(stream),
+                                reinterpret_cast<const uint4*>(src), ld_src / 8, rows, wv, q_off, n_docs,
+                                reinterpret_cast<uint4*>(dst), ld_dst / 8),
+                    "launch broadcast_rows_kernel");
 }
 
 kalm_status kalm_selftest_wait_timeout(uint64_t wait_ns, kalm_stream_t stream) {

@@ -167,6 +167,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  pdl_launch_dependents();
+  pdl_wait_predecessor();  // inputs of this GEMM are written by the previous kernel
 
   const int n_m = (M + kBM - 1) / kBM;
   const int n_n = (N + BN - 1) / BN;
@@ -361,6 +363,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   cluster_sync_all();  // barriers of both CTAs initialised, tensor memory allocated
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  pdl_launch_dependents();
+  pdl_wait_predecessor();  // inputs of this GEMM are written by the previous kernel
 
   const int n_m = (M + 2 * kBM - 1) / (2 * kBM);
   const int n_n = (N + BN - 1) / BN;
@@ -595,9 +599,10 @@ kalm_status launch_pair(const kalm_bf16* x, int64_t ldx, const kalm_bf16* w, int
   if (st != KALM_OK) return st;
   const int64_t tiles = ((m + 2 * kBM - 1) / (2 * kBM)) * ((n + BN - 1) / BN);
   const int pairs = static_cast<int>(tiles < slots ? tiles : slots);
-  linear_pair_kernel<BN><<<2 * pairs, kThreads, Linear2Cfg<BN>::SMEM, stream>>>(
-      tx, tw, ty, tr, residual != nullptr, (int)m, n, k, kWaitNs, device_error_word());
-  return check_cuda(cudaGetLastError(), "launch linear_pair_kernel");
+  return check_cuda(launch_pdl(linear_pair_kernel<BN>, dim3(2 * pairs), dim3(kThreads), Linear2Cfg<BN>::SMEM,
+                                stream, tx, tw, ty, tr, residual != nullptr, (int)m, n, k, kWaitNs,
+                                device_error_word()),
+                    "launch linear_pair_kernel");
 }
 
 }  // namespace
@@ -647,13 +652,12 @@ kalm_status launch_linear(const kalm_bf16* x, int64_t ldx, const kalm_bf16* w, i
   const int64_t tiles = ((m + kBM - 1) / kBM) * ((n + BN - 1) / BN);
   const int grid = static_cast<int>(tiles < num_sms() ? tiles : num_sms());
   const bool has_r = residual != nullptr;
-  if (wide)
-    linear_kernel<256><<<grid, kThreads, LinearCfg<256>::SMEM, stream>>>(tx, tw, ty, tr, has_r, (int)m, n, k,
-                                                                          kWaitNs, device_error_word());
-  else
-    linear_kernel<128><<<grid, kThreads, LinearCfg<128>::SMEM, stream>>>(tx, tw, ty, tr, has_r, (int)m, n, k,
-                                                                          kWaitNs, device_error_word());
-  return check_cuda(cudaGetLastError(), "launch linear_kernel");
+  const cudaError_t ce =
+      wide ? launch_pdl(linear_kernel<256>, dim3(grid), dim3(kThreads), LinearCfg<256>::SMEM, stream, tx, tw, ty, tr,
+                        has_r, (int)m, n, k, kWaitNs, device_error_word())
+           : launch_pdl(linear_kernel<128>, dim3(grid), dim3(kThreads), LinearCfg<128>::SMEM, stream, tx, tw, ty, tr,
+                        has_r, (int)m, n, k, kWaitNs, device_error_word());
+  return check_cuda(ce, "launch linear_kernel");
 }
 
 }  // namespace kalm

@@ -85,6 +85,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                             const __grid_constant__ CUtensorMap tm_vs, const __grid_constant__ CUtensorMap tm_kc,
                             const __grid_constant__ CUtensorMap tm_vc, const __grid_constant__ CUtensorMap tm_o,
                             const AttnParams p) {
+  pdl_launch_dependents();
+  pdl_wait_predecessor();  // q/K/V come from the previous kernel; offsets are read right below
   // ---- work item: heaviest query tiles (largest t) first
   const int per_t = p.n_docs * p.n_kv;
   const int rem = static_cast<int>(blockIdx.x) % per_t;
@@ -485,7 +487,7 @@ extern "C" kalm_status kalm_merged_attention(const kalm_bf16* q, int64_t ldq, co
   prm.err = device_error_word();
   const int64_t grid = static_cast<int64_t>(last_tile_only ? 1 : prm.tiles_per_doc) * n_docs * n_kv;
   if (grid > INT32_MAX) return fail(KALM_ERR_INVALID_ARG, "kalm_merged_attention: grid too large");
-  merged_attention_kernel<<<static_cast<unsigned>(grid), kThreads, kSmem, static_cast<cudaStream_t>(stream)>>>(
-      tq, tks, tvs, tkc, tvc, to, prm);
-  return check_cuda(cudaGetLastError(), "launch merged_attention_kernel");
+  return check_cuda(launch_pdl(merged_attention_kernel, dim3(static_cast<unsigned>(grid)), dim3(kThreads), kSmem,
+                                static_cast<cudaStream_t>(stream), tq, tks, tvs, tkc, tvc, to, prm),
+                    "launch merged_attention_kernel");
 }

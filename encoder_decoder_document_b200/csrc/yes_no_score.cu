@@ -18,6 +18,8 @@ __global__ void __launch_bounds__(128) yes_no_kernel(const uint4* __restrict__ h
                                                      const uint4* __restrict__ w_yes, const uint4* __restrict__ w_no,
                                                      float* __restrict__ yes, float* __restrict__ no,
                                                      float* __restrict__ margin, float* __restrict__ score) {
+  pdl_launch_dependents();
+  pdl_wait_predecessor();
   const int lane = threadIdx.x & 31;
   const int d = blockIdx.x * 4 + (threadIdx.x >> 5);
   if (d >= n_docs) return;
@@ -82,8 +84,9 @@ extern "C" kalm_status kalm_yes_no_score(const kalm_bf16* hidden, int64_t ldh, c
   if (!aligned16(hidden) || !aligned16(w_yes) || !aligned16(w_no))
     return fail(KALM_ERR_INVALID_ARG, "kalm_yes_no_score: bf16 pointers must be 16-byte aligned");
   const unsigned blocks = (unsigned)((n_docs + 3) / 4);
-  yes_no_kernel<<<blocks, 128, 0, static_cast<cudaStream_t>(stream)>>>(
-      reinterpret_cast<const uint4*>(hidden), ldh / 8, q_off, n_docs, hidden_dim / 8,
-      reinterpret_cast<const uint4*>(w_yes), reinterpret_cast<const uint4*>(w_no), yes, no, margin, score);
-  return check_cuda(cudaGetLastError(), "launch yes_no_kernel");
+  return check_cuda(launch_pdl(yes_no_kernel, dim3(blocks), dim3(128), 0, static_cast<cudaStream_t>(stream),
+                                reinterpret_cast<const uint4*>(hidden), ldh / 8, q_off, n_docs, hidden_dim / 8,
+                                reinterpret_cast<const uint4*>(w_yes), reinterpret_cast<const uint4*>(w_no), yes,
+                                no, margin, score),
+                    "launch yes_no_kernel");
 }

@@ -208,23 +208,32 @@ class FBNLScorer:
     def capture(self, instrument: bool = False) -> None:
         """Record forward() as a CUDA graph (buffers must stay allocated).
 
-        With ``instrument`` an external timing event is recorded after every
-        launch inside the graph, so each replay yields per-kernel durations
-        (``kernel_times()``)."""
+        With ``instrument`` a second graph is recorded with an external timing
+        event after every launch (``graph_inst``), so each of its replays yields
+        per-kernel durations (``kernel_times()``).  The events sit between the
+        launches and keep them from overlapping, so the plain graph is the one to
+        time a step with."""
         s = torch.cuda.Stream()
         s.wait_stream(torch.cuda.current_stream())
         with torch.cuda.stream(s):
             self.forward()  # warm-up: one-time device set-up happens outside capture
         torch.cuda.current_stream().wait_stream(s)
         torch.cuda.synchronize()
+        self.marks = None
         g = torch.cuda.CUDAGraph()
-        self.marks = [] if instrument else None
         with torch.cuda.graph(g):
             self.forward()
         self.graph = g
+        self.graph_inst = None
+        if instrument:
+            self.marks = []
+            gi = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(gi):
+                self.forward()
+            self.graph_inst = gi
 
     def kernel_times(self) -> dict:
-        """{label: [ms per launch, ...]} of the last replay of an instrumented graph."""
+        """{label: [ms per launch, ...]} of the last replay of the instrumented graph."""
         out: dict = {}
         if not self.marks:
             return out
