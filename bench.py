@@ -286,10 +286,25 @@ def main():
         total_ms = float(t.item())
     value = world * q.n_docs * args.steps / (total_ms / 1e3)
 
-    # ---------------- end to end through the public API: H2D inputs, graph, D2H scores
-    e2e_ms = []
+    # ---------------- end to end through the public API: every step copies its inputs
+    # host -> device (pinned) and reads its scores back.  Pipelined: FBNLScorer.score_stream
+    # copies query k+1 while query k runs (the serving path); serial: copy, run, read back.
+    n_e2e = args.steps
+    outs = [torch.empty(4, q.n_docs, dtype=torch.float32).pin_memory() for _ in range(2)]
+    inputs = [(enc_h, len_h, x0_h)] * n_e2e
+    sc.score_stream(inputs[: max(args.warmup, 3)], [outs[k % 2] for k in range(max(args.warmup, 3))])
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    sc.score_stream(inputs, [outs[k % 2] for k in range(n_e2e)])
+    b.record(stream)
+    b.synchronize()
+    e2e_total = a.elapsed_time(b)
+    serial_ms = []
     for _ in range(max(args.warmup, 3) + args.steps):
-        flush.fill_(1.0)
         a = torch.cuda.Event(enable_timing=True)
         b = torch.cuda.Event(enable_timing=True)
         a.record(stream)
@@ -298,13 +313,13 @@ def main():
         sc.scores_to_host(out_h)
         b.record(stream)
         b.synchronize()
-        e2e_ms.append(a.elapsed_time(b))
-    e2e_ms = e2e_ms[max(args.warmup, 3):]
-    e2e_total = sum(e2e_ms)
+        serial_ms.append(a.elapsed_time(b))
+    serial_total = sum(serial_ms[max(args.warmup, 3):])
     if world > 1:
-        t = torch.tensor([e2e_total], device="cuda", dtype=torch.float64)
+        t = torch.tensor([e2e_total, serial_total], device="cuda", dtype=torch.float64)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_total = float(t.item())
+        e2e_total, serial_total = float(t[0].item()), float(t[1].item())
+    kalm_check_device_errors()
     h2d = enc_h.numel() * 2 + len_h.numel() * 4 + x0_h.numel() * 2
     d2h = out_h.numel() * 4
 
@@ -354,9 +369,14 @@ def main():
                                      "frac": attn_proj_flops / (attn_proj_us * 1e-6) / 1e12 / pk["bf16"]},
             "step_tflops": step_flops / (ms_step * 1e-3) / 1e12,
             "kernels": kern,
-            "e2e": {"value": world * q.n_docs * args.steps / (e2e_total / 1e3), "unit": UNIT,
+            "e2e": {"value": world * q.n_docs * n_e2e / (e2e_total / 1e3), "unit": UNIT,
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                    "ms_per_step": e2e_total / args.steps},
+                    "ms_per_step": e2e_total / n_e2e,
+                    "how": "FBNLScorer.score_stream over K queries: pinned host inputs copied to the device and "
+                           "scores read back every step; query k+1's copy overlaps query k's compute",
+                    "serial": {"value": world * q.n_docs * args.steps / (serial_total / 1e3),
+                               "ms_per_step": serial_total / args.steps,
+                               "how": "copy in, replay, copy out, one step at a time"}},
             "gpu_launches": sc.launches * args.steps,
             "clocks": clk,
             "cpu_baseline": cb,

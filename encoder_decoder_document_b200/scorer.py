@@ -86,10 +86,12 @@ class FBNLScorer:
         rows = n_docs * lq
         kw = dict(device=device)
         self.n_docs, self.total_tokens, self.total_pooled, self.lq = shape
-        self.enc = torch.empty(max(total_tokens, 1), H, dtype=torch.bfloat16, **kw)
-        self.doc_len = torch.empty(n_docs, dtype=torch.int32, **kw)
+        # two input slots, so the next query's inputs can be copied while this one runs
+        self.slots = [dict(enc=torch.empty(max(total_tokens, 1), H, dtype=torch.bfloat16, **kw),
+                           doc_len=torch.empty(n_docs, dtype=torch.int32, **kw),
+                           x0=torch.empty(lq, H, dtype=torch.bfloat16, **kw)) for _ in range(2)]
+        self.use_slot(0)
         self.q_len = torch.full((n_docs,), lq, dtype=torch.int32, **kw)
-        self.x0 = torch.empty(lq, H, dtype=torch.bfloat16, **kw)
         self.tok_off = torch.empty(n_docs + 1, dtype=torch.int64, **kw)
         self.pool_off = torch.empty(n_docs + 1, dtype=torch.int64, **kw)
         self.q_off = torch.empty(n_docs + 1, dtype=torch.int64, **kw)
@@ -99,11 +101,15 @@ class FBNLScorer:
         self.qkv = torch.empty(rows, (self.n_q + 2 * self.n_kv) * D, dtype=torch.bfloat16, **kw)
         self.o = torch.empty(rows, self.n_q * D, dtype=torch.bfloat16, **kw)
         self.x = torch.empty(rows, H, dtype=torch.bfloat16, **kw)
-        self.yes = torch.empty(n_docs, dtype=torch.float32, **kw)
-        self.no = torch.empty(n_docs, dtype=torch.float32, **kw)
-        self.margin = torch.empty(n_docs, dtype=torch.float32, **kw)
-        self.score = torch.empty(n_docs, dtype=torch.float32, **kw)
+        # (yes, no, margin, score) rows of one buffer: one device->host copy per query
         self.result = torch.empty(4, n_docs, dtype=torch.float32, **kw)
+        self.yes, self.no, self.margin, self.score = self.result[0], self.result[1], self.result[2], self.result[3]
+        self.graphs = None
+
+    def use_slot(self, i: int) -> None:
+        """Point the input buffers at slot i (for the next forward() or capture)."""
+        self.slot = i
+        self.enc, self.doc_len, self.x0 = (self.slots[i][k] for k in ("enc", "doc_len", "x0"))
 
     # ------------------------------------------------------------------ steps
     def _mark(self, label: str) -> None:
@@ -220,10 +226,16 @@ class FBNLScorer:
         torch.cuda.current_stream().wait_stream(s)
         torch.cuda.synchronize()
         self.marks = None
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g):
-            self.forward()
-        self.graph = g
+        slot = self.slot
+        self.graphs = []
+        for i in range(2):  # one graph per input slot
+            self.use_slot(i)
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                self.forward()
+            self.graphs.append(g)
+        self.use_slot(slot)
+        self.graph = self.graphs[slot]
         self.graph_inst = None
         if instrument:
             self.marks = []
@@ -256,11 +268,52 @@ class FBNLScorer:
 
     def scores_to_host(self, out: Optional[torch.Tensor] = None) -> torch.Tensor:
         """Device -> host copy of (yes, no, margin, score) as a [4][n_docs] fp32 tensor."""
-        torch.stack([self.yes, self.no, self.margin, self.score], out=self.result)
         if out is None:
             return self.result.cpu()
         out.copy_(self.result, non_blocking=True)
         return out
+
+    def score_stream(self, inputs, outs) -> None:
+        """Score a stream of queries of this shape, overlapping transfers with compute.
+
+        inputs[k] = (enc, doc_len, x0) pinned host tensors of query k; outs[k] a
+        pinned [4][n_docs] fp32 host tensor that receives (yes, no, margin, score).
+        Query k+1's inputs are copied on a side stream into the other input slot
+        while query k runs (one captured graph per slot); every copy and every
+        result read happen inside the call, which returns without synchronising.
+        Requires capture() first."""
+        if self.graphs is None:
+            raise RuntimeError("score_stream needs capture() first")
+        comp = torch.cuda.current_stream()
+        if getattr(self, "_copy_stream", None) is None:
+            self._copy_stream = torch.cuda.Stream()
+            self._ready = [torch.cuda.Event(), torch.cuda.Event()]
+            self._free = [torch.cuda.Event(), torch.cuda.Event()]
+        cs = self._copy_stream
+        cs.wait_stream(comp)
+
+        def h2d(k):
+            i = k % 2
+            slot = self.slots[i]
+            with torch.cuda.stream(cs):
+                if k >= 2:
+                    cs.wait_event(self._free[i])  # the query that last used this slot is done with it
+                enc, doc_len, x0 = inputs[k]
+                slot["enc"][: enc.shape[0]].copy_(enc, non_blocking=True)
+                slot["doc_len"].copy_(doc_len, non_blocking=True)
+                slot["x0"].copy_(x0, non_blocking=True)
+                self._ready[i].record(cs)
+
+        if inputs:
+            h2d(0)
+        for k in range(len(inputs)):
+            if k + 1 < len(inputs):
+                h2d(k + 1)
+            i = k % 2
+            comp.wait_event(self._ready[i])
+            self.graphs[i].replay()
+            self._free[i].record(comp)
+            outs[k].copy_(self.result, non_blocking=True)
 
     def rerank(self, x0: np.ndarray, enc: np.ndarray, doc_len: np.ndarray, top_n: Optional[int] = None):
         """Score one query's documents and return [{index, relevance_score}] best first.

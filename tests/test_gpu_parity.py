@@ -549,3 +549,25 @@ def test_invalid_arguments_are_rejected_on_the_host(kalm):
         kalm.kalm_check_device_errors()
     assert e.value.name == "KALM_ERR_DEVICE_ARG"
     assert tok.cpu().tolist() == [0, 5, 1029]
+
+
+def test_score_stream_matches_single_queries(kalm):
+    """The pipelined public API (copies of the next query overlap the current one)
+    returns, for every query of a stream, the scores of that query alone."""
+    from encoder_decoder_document_b200.scorer import DeviceWeights, FBNLScorer
+    base = synthetic.make_query("tiny")
+    qs = [synthetic.make_query("tiny", seed=s, doc_len=base.doc_len) for s in range(5)]
+    sc = FBNLScorer(DeviceWeights.from_bits(base.weights), base.n_q, base.n_kv)
+    singles = []
+    for q in qs:
+        sc.rerank(q.x0, q.enc, q.doc_len)
+        singles.append(sc.scores_to_host().numpy().copy())
+    sc.capture()
+    pin = lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).pin_memory()
+    inputs = [(pin(q.enc), torch.from_numpy(q.doc_len).pin_memory(), pin(q.x0)) for q in qs]
+    outs = [torch.empty(4, base.n_docs, dtype=torch.float32).pin_memory() for _ in qs]
+    sc.score_stream(inputs, outs)
+    torch.cuda.synchronize()
+    kalm.kalm_check_device_errors()
+    for k in range(len(qs)):
+        np.testing.assert_array_equal(outs[k].numpy(), singles[k])
