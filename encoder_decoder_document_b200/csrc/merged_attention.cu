@@ -5,10 +5,12 @@
 // concatenation of its own (causal) self-attention K/V and the cross-attention
 // K/V of the document's cached pooled vectors.  One softmax covers both parts.
 //
-// Design (sm_100a), one CTA per (query tile, KV head, document):
+// Design (sm_100a): a persistent kernel, one CTA per SM, each CTA walking a list
+// of work items (query tile, KV head, document), heaviest tiles first:
 //   * 128 packed rows = (128 / G) decoder positions x G query heads of one KV
 //     head (GQA), so every K/V tile is fetched once for the G heads sharing it.
-//     The Q tile (128 x 256 bf16) is fetched once by a 3-D TMA box.
+//     The Q tile (128 x 256 bf16) is one 4-D TMA box (64 columns x heads x
+//     positions x 4 column slabs).
 //   * The KV loop walks the self segment (64-key tiles up to the tile's last
 //     position, causal mask inside) and then the cross segment (64-key tiles,
 //     only the ragged tail masked).  The concatenation exists only as this
@@ -21,18 +23,17 @@
 //     each then exponentiates (ex2 on the fused scale) and writes its own 32
 //     columns of P as bf16 into a 128-byte-swizzled shared tile (the A operand
 //     of PV), and keeps its own partial row sum.  The two partial sums meet
-//     once, in the epilogue, which again splits the 256 O columns in halves.
-//     The running max is only raised when it grows by more than 2^8 in the
-//     exponent; otherwise P keeps the stale max (values stay below 256), so the
-//     O accumulator is rescaled in tensor memory only on such rare jumps.  The
-//     final O / l is exact either way.
+//     once per item, in the epilogue, which again splits the 256 O columns in
+//     halves.  The running max is only raised when it grows by more than 2^8 in
+//     the exponent; otherwise P keeps the stale max (values stay below 256), so
+//     the O accumulator is rescaled in tensor memory only on such rare jumps.
+//     The final O / l is exact either way.
+//   * The K/V rings, S/P buffers and their barriers run over one tile counter
+//     for all items of the CTA, so the next item's Q copy (as soon as the last S
+//     of the current item is done) and its first S product overlap the current
+//     item's last softmax, P V and O write-out.
 //   * Warp roles: warps 0-7 softmax + epilogue, warp 8 TMA producer of Q and K,
 //     warp 10 TMA producer of V, warp 9 tensor-memory allocation and MMA issue.
-//     K, V and P are double-buffered.  Each tile is one TMA box: a 64-key K or V
-//     tile is a 3-D box (64 columns x 64 keys x 4 column slabs) and the Q tile a
-//     4-D box (64 columns x heads x positions x 4 slabs), because a warp's tile
-//     copies are served one after another and few large boxes keep the copy
-//     engine busy where many small ones would not.
 #include <cmath>
 
 #include "kalm.h"
@@ -51,11 +52,12 @@ constexpr int kTmaWarp = 8;
 constexpr int kMmaWarp = 9;
 constexpr int kTmaWarpV = 10;
 constexpr int kQBytes = kBM * kD * 2;          // 4 slabs of 128 rows x 128 B
-constexpr int kQSlab = kBM * 128;              // 16 KB
 constexpr int kKVBytes = kBKV * kD * 2;        // 4 slabs of 64 rows x 128 B
+constexpr int kQSlab = kBM * 128;              // 16 KB
 constexpr int kKVSlab = kBKV * 128;            // 8 KB
 constexpr int kPBytes = kBM * kBKV * 2;        // 1 slab of 128 rows x 128 B
-constexpr int kSmem = 1024 + kQBytes + 2 * kKVBytes + 2 * kKVBytes + 2 * kPBytes + 128 + 2 * 128 * 4;
+constexpr int kBarBytes = 256;
+constexpr int kSmem = 1024 + kQBytes + 2 * kKVBytes + 2 * kKVBytes + 2 * kPBytes + kBarBytes + 2 * 128 * 4;
 constexpr uint32_t kTmemCols = 512;            // O: [0,256), S0: [256,320), S1: [320,384)
 constexpr uint32_t kIdescS = idesc_bf16_f32(kBM, kBKV, false, false);
 constexpr uint32_t kIdescPV = idesc_bf16_f32(kBM, kD, false, true);
@@ -75,10 +77,36 @@ struct AttnParams {
   int G;            // query heads per KV head
   int P;            // decoder positions per tile = 128 / G
   int tiles_per_doc;
+  int n_items;
   float scale_log2;  // scale * log2(e)
   uint64_t wait_ns;
   uint32_t* err;
 };
+
+// One work item: query tile t of KV head g of document d, with its extents.
+struct Item {
+  int t, g, d, Lq, Nc, pos0, pos1, n_self, nt;
+  int64_t q0, qi, c0;
+};
+
+__device__ __forceinline__ Item make_item(const AttnParams& p, int w) {
+  Item it;
+  const int per_t = p.n_docs * p.n_kv;
+  const int rem = w % per_t;
+  it.g = rem % p.n_kv;
+  it.d = rem / p.n_kv;
+  it.q0 = p.q_off[it.d];
+  it.Lq = static_cast<int>(p.q_off[it.d + 1] - it.q0);
+  it.qi = p.in_off ? p.in_off[it.d] : it.q0;
+  it.t = p.last_only ? (it.Lq > 0 ? (it.Lq - 1) / p.P : 0) : p.tiles_per_doc - 1 - w / per_t;
+  it.c0 = p.pool_off[it.d];
+  it.Nc = static_cast<int>(p.pool_off[it.d + 1] - it.c0);
+  it.pos0 = it.t * p.P;
+  it.pos1 = min(it.pos0 + p.P, it.Lq);
+  it.n_self = it.pos0 < it.Lq ? (it.pos1 + kBKV - 1) / kBKV : 0;
+  it.nt = it.pos0 < it.Lq ? it.n_self + (it.Nc + kBKV - 1) / kBKV : 0;  // 0: nothing to do
+  return it;
+}
 
 __global__ void __launch_bounds__(kThreads, 1)
     merged_attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_ks,
@@ -86,25 +114,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                             const __grid_constant__ CUtensorMap tm_vc, const __grid_constant__ CUtensorMap tm_o,
                             const AttnParams p) {
   pdl_launch_dependents();
-  pdl_wait_predecessor();  // q/K/V come from the previous kernel; offsets are read right below
-  // ---- work item: heaviest query tiles (largest t) first
-  const int per_t = p.n_docs * p.n_kv;
-  const int rem = static_cast<int>(blockIdx.x) % per_t;
-  const int g = rem % p.n_kv;
-  const int d = rem / p.n_kv;
-  const int64_t q0 = p.q_off[d];                      // output rows
-  const int Lq = static_cast<int>(p.q_off[d + 1] - q0);
-  const int64_t qi = p.in_off ? p.in_off[d] : q0;     // input (q, self K/V) rows
-  const int t = p.last_only ? (Lq > 0 ? (Lq - 1) / p.P : 0)
-                            : p.tiles_per_doc - 1 - static_cast<int>(blockIdx.x) / per_t;
-  const int64_t c0 = p.pool_off[d];
-  const int Nc = static_cast<int>(p.pool_off[d + 1] - c0);
-  const int pos0 = t * p.P;
-  if (pos0 >= Lq) return;  // uniform across the CTA, before any set-up
-  const int pos1 = min(pos0 + p.P, Lq);
-  const int n_self = (pos1 + kBKV - 1) / kBKV;
-  const int n_cross = (Nc + kBKV - 1) / kBKV;
-  const int nt = n_self + n_cross;
+  pdl_wait_predecessor();  // q/K/V come from the previous kernel; offsets are read by every role
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -113,20 +123,23 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* sV = sK + 2 * kKVBytes;
   uint8_t* sP = sV + 2 * kKVBytes;
   uint64_t* bars = reinterpret_cast<uint64_t*>(sP + 2 * kPBytes);
-  uint64_t* bar_q = bars;
-  uint64_t* bar_k = bars + 1;   // [2]
-  uint64_t* bar_v = bars + 3;   // [2]
-  uint64_t* bar_s = bars + 5;   // [2]
-  uint64_t* bar_p = bars + 7;   // [2]
-  uint64_t* bar_pv = bars + 9;  // [2]
-  uint64_t* bar_l = bars + 11;  // partial row sums published
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 12);
+  uint64_t* bar_q = bars;        // Q landed (per item)
+  uint64_t* bar_qfree = bars + 1;  // last S of an item done: Q tile reusable (per item)
+  uint64_t* bar_k = bars + 2;    // [2] K tile landed
+  uint64_t* bar_v = bars + 4;    // [2] V tile landed
+  uint64_t* bar_s = bars + 6;    // [2] S ready
+  uint64_t* bar_p = bars + 8;    // [2] P written (and O rescaled)
+  uint64_t* bar_pv = bars + 10;  // [2] P V done
+  uint64_t* bar_l = bars + 12;   // partial row sums published (per item)
+  uint64_t* bar_ofree = bars + 13;  // O read out by the epilogue (per item)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 14);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  float* l_part = reinterpret_cast<float*>(bars + 16);  // [2][128]
+  float* l_part = reinterpret_cast<float*>(sP + 2 * kPBytes + kBarBytes);  // [2][128]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
     mbar_init(bar_q, 1);
+    mbar_init(bar_qfree, 1);
     for (int i = 0; i < 2; ++i) {
       mbar_init(&bar_k[i], 1);
       mbar_init(&bar_v[i], 1);
@@ -135,6 +148,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&bar_pv[i], 1);
     }
     mbar_init(bar_l, kSoftmaxThreads);
+    mbar_init(bar_ofree, kSoftmaxThreads);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -147,40 +161,56 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
+  auto fail_wait = [&]() {
+    record_error(p.err, kErrTimeout | kSiteAttention);
+    *abort_flag = 1;
+  };
+
   if (warp == kTmaWarp || warp == kTmaWarpV) {
     // ------------------------------------------------------------ TMA producers (Q+K, V)
     if (lane == 0) {
       const bool is_v = warp == kTmaWarpV;
-      if (!is_v) {
-        mbar_arrive_expect_tx(bar_q, kQBytes);
-        tma_load_4d(sQ, &tm_q, bar_q, 0, g * p.G, static_cast<int32_t>(qi + pos0), 0);
-      }
       uint64_t* bar_free = is_v ? bar_pv : bar_s;   // slot reusable once S (for K) / PV (for V) is done
       uint64_t* bar_full = is_v ? bar_v : bar_k;
       uint8_t* ring = is_v ? sV : sK;
-      for (int j = 0; j < nt && !*abort_flag; ++j) {
-        const int s = j & 1;
-        const bool self = j < n_self;
-        const int32_t row = self ? static_cast<int32_t>(qi + j * kBKV)
-                                 : static_cast<int32_t>(c0 + (j - n_self) * kBKV);
-        const CUtensorMap* m = is_v ? (self ? &tm_vs : &tm_vc) : (self ? &tm_ks : &tm_kc);
-        if (j >= 2 && !mbar_wait(&bar_free[s], ((j - 2) >> 1) & 1, p.wait_ns)) {
-          record_error(p.err, kErrTimeout | kSiteAttention);
-          *abort_flag = 1;
-          break;
+      uint32_t J = 0;  // tile counter over all items of this CTA
+      int n_it = 0;
+      bool ok = true;
+      for (int w = blockIdx.x; w < p.n_items && ok && !*abort_flag; w += gridDim.x) {
+        const Item it = make_item(p, w);
+        if (it.nt == 0) continue;
+        if (!is_v) {
+          if (n_it >= 1 && !mbar_wait(bar_qfree, (n_it - 1) & 1, p.wait_ns)) {
+            fail_wait();
+            break;
+          }
+          mbar_arrive_expect_tx(bar_q, kQBytes);
+          tma_load_4d(sQ, &tm_q, bar_q, 0, it.g * p.G, static_cast<int32_t>(it.qi + it.pos0), 0);
         }
-        mbar_arrive_expect_tx(&bar_full[s], kKVBytes);
-        tma_load_3d(ring + s * kKVBytes, m, &bar_full[s], 0, row, g * 4);
+        for (int j = 0; j < it.nt; ++j, ++J) {
+          const int s = J & 1;
+          const bool self = j < it.n_self;
+          const int32_t row = self ? static_cast<int32_t>(it.qi + j * kBKV)
+                                   : static_cast<int32_t>(it.c0 + (j - it.n_self) * kBKV);
+          const CUtensorMap* m = is_v ? (self ? &tm_vs : &tm_vc) : (self ? &tm_ks : &tm_kc);
+          if (J >= 2 && !mbar_wait(&bar_free[s], ((J - 2) >> 1) & 1, p.wait_ns)) {
+            fail_wait();
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&bar_full[s], kKVBytes);
+          tma_load_3d(ring + s * kKVBytes, m, &bar_full[s], 0, row, it.g * 4);
+        }
+        ++n_it;
       }
     }
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       const uint32_t q_base = smem_u32(sQ), k_base = smem_u32(sK), v_base = smem_u32(sV), p_base = smem_u32(sP);
-      bool ok = mbar_wait(bar_q, 0, p.wait_ns);
-      auto issue_s = [&](int j) -> bool {
-        const int s = j & 1;
-        if (!mbar_wait(&bar_k[s], (j >> 1) & 1, p.wait_ns)) return false;
+      auto issue_s = [&](uint32_t J) -> bool {
+        const int s = J & 1;
+        if (!mbar_wait(&bar_k[s], (J >> 1) & 1, p.wait_ns)) return false;
         tc_fence_after();
         const uint32_t d_s = tmem + 256u + static_cast<uint32_t>(s * kBKV);
 #pragma unroll
@@ -193,194 +223,238 @@ __global__ void __launch_bounds__(kThreads, 1)
         umma_commit(&bar_s[s]);
         return true;
       };
-      if (ok) ok = issue_s(0);
-      for (int j = 0; j < nt && ok && !*abort_flag; ++j) {
-        const int s = j & 1;
-        if (j + 1 < nt) {
-          ok = issue_s(j + 1);
-          if (!ok) break;
-        }
-        if (!mbar_wait(&bar_p[s], (j >> 1) & 1, p.wait_ns) || !mbar_wait(&bar_v[s], (j >> 1) & 1, p.wait_ns)) {
-          ok = false;
-          break;
-        }
+      uint32_t J = 0;
+      int n_it = 0;
+      bool ok = true;
+      for (int w = blockIdx.x; w < p.n_items && ok && !*abort_flag; w += gridDim.x) {
+        const Item it = make_item(p, w);
+        if (it.nt == 0) continue;
+        ok = mbar_wait(bar_q, n_it & 1, p.wait_ns);
+        if (!ok) break;
         tc_fence_after();
+        ok = issue_s(J);
+        for (int j = 0; j < it.nt && ok && !*abort_flag; ++j) {
+          const uint32_t Jc = J + j;
+          const int s = Jc & 1;
+          if (j + 1 < it.nt) {
+            ok = issue_s(Jc + 1);
+            if (!ok) break;
+          } else {
+            umma_commit(bar_qfree);  // fires once every S of this item (and all before) is done
+          }
+          if (!mbar_wait(&bar_p[s], (Jc >> 1) & 1, p.wait_ns) ||
+              !mbar_wait(&bar_v[s], (Jc >> 1) & 1, p.wait_ns) ||
+              (j == 0 && n_it >= 1 && !mbar_wait(bar_ofree, (n_it - 1) & 1, p.wait_ns))) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
 #pragma unroll
-        for (int kk = 0; kk < kBKV / 16; ++kk) {
-          const uint64_t ad = sdesc_sw128(p_base + s * kPBytes + kk * 32, 16, 1024);
-          // V is MN-major: 64-column slabs kKVSlab apart (LBO), 8-key groups 1024 B apart (SBO)
-          const uint64_t bd = sdesc_sw128(v_base + s * kKVBytes + kk * 16 * 128, kKVSlab, 1024);
-          umma_bf16_ss(tmem, ad, bd, kIdescPV, (j | kk) != 0 ? 1u : 0u);
+          for (int kk = 0; kk < kBKV / 16; ++kk) {
+            const uint64_t ad = sdesc_sw128(p_base + s * kPBytes + kk * 32, 16, 1024);
+            // V is MN-major: 64-column slabs kKVSlab apart (LBO), 8-key groups 1024 B apart (SBO)
+            const uint64_t bd = sdesc_sw128(v_base + s * kKVBytes + kk * 16 * 128, kKVSlab, 1024);
+            umma_bf16_ss(tmem, ad, bd, kIdescPV, (j | kk) != 0 ? 1u : 0u);
+          }
+          umma_commit(&bar_pv[s]);
         }
-        umma_commit(&bar_pv[s]);
+        J += it.nt;
+        ++n_it;
       }
-      if (!ok) {
-        record_error(p.err, kErrTimeout | kSiteAttention);
-        *abort_flag = 1;
-      }
+      if (!ok) fail_wait();
     }
   } else {
     // ------------------------------------------------------------ softmax warps 0..7
     const int quarter = warp & 3;             // TMEM lane quarter
     const int half = warp >> 2;               // which 32 of the 64 keys / 128 of the 256 O columns
     const int r = quarter * 32 + lane;        // packed row = TMEM lane
-    const int pos = pos0 + r / p.G;           // decoder position of this row
-    const int hh = r % p.G;                   // query head within the KV group
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
     const float c2 = p.scale_log2;
-    float m_run = -INFINITY, l_run = 0.f;     // running max (log2 units) and this half's sum
+    uint32_t J = 0;
+    int n_it = 0;
     bool ok = true;
-    for (int j = 0; j < nt; ++j) {
-      const int s = j & 1;
-      bool w = mbar_wait(&bar_s[s], (j >> 1) & 1, p.wait_ns);
-      if (!__all_sync(0xffffffffu, w) || *abort_flag) {
+    for (int w = blockIdx.x; w < p.n_items && ok; w += gridDim.x) {
+      const Item it = make_item(p, w);
+      if (it.nt == 0) continue;
+      const int pos = it.pos0 + r / p.G;      // decoder position of this row
+      const int hh = r % p.G;                 // query head within the KV group
+      float m_run = -INFINITY, l_run = 0.f;   // running max (log2 units) and this half's sum
+      for (int j = 0; j < it.nt; ++j) {
+        const uint32_t Jc = J + j;
+        const int s = Jc & 1;
+        bool wt = mbar_wait(&bar_s[s], (Jc >> 1) & 1, p.wait_ns);
+        if (!__all_sync(0xffffffffu, wt) || *abort_flag) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        uint32_t sr[64];
+        tmem_ld32(lane_base + 256u + s * kBKV, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
+        tmem_ld32(lane_base + 256u + s * kBKV + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
+        tmem_ld_wait();
+        // visible keys of this tile: self keys k <= pos, cross keys k < Nc
+        int n_vis = (j < it.n_self) ? pos + 1 - j * kBKV : it.Nc - (j - it.n_self) * kBKV;
+        n_vis = max(0, min(kBKV, n_vis));
+        const bool masked = !__all_sync(0xffffffffu, n_vis == kBKV);
+        if (masked) {
+#pragma unroll
+          for (int k = 0; k < 64; ++k)
+            if (k >= n_vis) sr[k] = __float_as_uint(-INFINITY);
+        }
+        // row max of the raw scores (scale > 0 keeps the order), as a tree
+        float t32[32];
+#pragma unroll
+        for (int k = 0; k < 32; ++k) t32[k] = fmaxf(__uint_as_float(sr[k]), __uint_as_float(sr[k + 32]));
+#pragma unroll
+        for (int w2 = 16; w2 > 0; w2 >>= 1)
+#pragma unroll
+          for (int k = 0; k < w2; ++k) t32[k] = fmaxf(t32[k], t32[k + w2]);
+        const float mx = t32[0] * c2;
+        float alpha = 1.f;
+        bool rescale = false;
+        if (j == 0) {
+          m_run = mx;  // every row sees self key 0, so mx is finite
+        } else if (mx > m_run + kRescaleThreshold) {
+          alpha = ex2_approx(m_run - mx);
+          m_run = mx;
+          rescale = true;
+        }
+        // this half's 32 probabilities: 2^(s * scale_log2 - m_run)
+        const float neg_m = -m_run;
+        float acc[4] = {0.f, 0.f, 0.f, 0.f};
+        uint32_t pk[16];
+#pragma unroll
+        for (int k = 0; k < 32; k += 2) {
+          const float s0 = __uint_as_float(half ? sr[32 + k] : sr[k]);
+          const float s1 = __uint_as_float(half ? sr[33 + k] : sr[k + 1]);
+          const float e0 = ex2_approx(fmaf(s0, c2, neg_m));
+          const float e1 = ex2_approx(fmaf(s1, c2, neg_m));
+          acc[(k >> 1) & 3] += e0 + e1;
+          pk[k >> 1] = pack_bf16x2(e0, e1);
+        }
+        l_run = l_run * alpha + ((acc[0] + acc[1]) + (acc[2] + acc[3]));
+        // the previous item's epilogue staged O in the P buffers
+        if (j == 0 && n_it >= 1) {
+          const bool wo = mbar_wait(bar_ofree, (n_it - 1) & 1, p.wait_ns);
+          if (!__all_sync(0xffffffffu, wo)) {
+            ok = false;
+            break;
+          }
+        }
+        // P stage s is free once PV_{j-2} has completed
+        if (Jc >= 2) {
+          const bool wp = mbar_wait(&bar_pv[s], ((Jc - 2) >> 1) & 1, p.wait_ns);
+          if (!__all_sync(0xffffffffu, wp)) {
+            ok = false;
+            break;
+          }
+        }
+        // 128-byte swizzled K-major row: 16-byte unit u of row r sits at unit u ^ (r & 7)
+        uint8_t* prow = sP + s * kPBytes + r * 128;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          uint4 v;
+          v.x = pk[4 * c + 0];
+          v.y = pk[4 * c + 1];
+          v.z = pk[4 * c + 2];
+          v.w = pk[4 * c + 3];
+          *reinterpret_cast<uint4*>(prow + (((half * 4 + c) ^ (r & 7)) << 4)) = v;
+        }
+        fence_proxy_async_smem();
+        if (__any_sync(0xffffffffu, rescale)) {
+          // O must hold the result of PV_{j-1} before it is rescaled in place
+          const bool wr = mbar_wait(&bar_pv[(Jc - 1) & 1], ((Jc - 1) >> 1) & 1, p.wait_ns);
+          if (!__all_sync(0xffffffffu, wr)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+#pragma unroll 1
+          for (int c = half * 128; c < half * 128 + 128; c += 32) {
+            uint32_t o[32];
+            tmem_ld32(lane_base + c, o);
+            tmem_ld_wait();
+#pragma unroll
+            for (int k = 0; k < 32; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * alpha);
+            tmem_st32(lane_base + c, o);
+          }
+          tmem_st_wait();
+        }
+        tc_fence_before();
+        mbar_arrive(&bar_p[s]);
+      }
+      if (!ok) break;
+      // ---- epilogue of this item: O / l -> bf16, this half's 128 columns
+      l_part[half * 128 + r] = l_run;
+      mbar_arrive(bar_l);
+      const uint32_t Jl = J + it.nt - 1;
+      bool wt = mbar_wait(&bar_pv[Jl & 1], (Jl >> 1) & 1, p.wait_ns) && mbar_wait(bar_l, n_it & 1, p.wait_ns);
+      if (!__all_sync(0xffffffffu, wt)) {
         ok = false;
         break;
       }
       tc_fence_after();
-      uint32_t sr[64];
-      tmem_ld32(lane_base + 256u + s * kBKV, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
-      tmem_ld32(lane_base + 256u + s * kBKV + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
-      tmem_ld_wait();
-      // visible keys of this tile: self keys k <= pos, cross keys k < Nc
-      int n_vis = (j < n_self) ? pos + 1 - j * kBKV : Nc - (j - n_self) * kBKV;
-      n_vis = max(0, min(kBKV, n_vis));
-      const bool masked = !__all_sync(0xffffffffu, n_vis == kBKV);
-      if (masked) {
-#pragma unroll
-        for (int k = 0; k < 64; ++k)
-          if (k >= n_vis) sr[k] = __float_as_uint(-INFINITY);
-      }
-      // row max of the raw scores (scale > 0 keeps the order), as a tree
-      float t32[32];
-#pragma unroll
-      for (int k = 0; k < 32; ++k) t32[k] = fmaxf(__uint_as_float(sr[k]), __uint_as_float(sr[k + 32]));
-#pragma unroll
-      for (int w2 = 16; w2 > 0; w2 >>= 1)
-#pragma unroll
-        for (int k = 0; k < w2; ++k) t32[k] = fmaxf(t32[k], t32[k + w2]);
-      const float mx = t32[0] * c2;
-      float alpha = 1.f;
-      bool rescale = false;
-      if (j == 0) {
-        m_run = mx;  // every row sees self key 0, so mx is finite
-      } else if (mx > m_run + kRescaleThreshold) {
-        alpha = ex2_approx(m_run - mx);
-        m_run = mx;
-        rescale = true;
-      }
-      // this half's 32 probabilities: 2^(s * scale_log2 - m_run)
-      const float neg_m = -m_run;
-      float acc[4] = {0.f, 0.f, 0.f, 0.f};
-      uint32_t pk[16];
-#pragma unroll
-      for (int k = 0; k < 32; k += 2) {
-        const float s0 = __uint_as_float(half ? sr[32 + k] : sr[k]);
-        const float s1 = __uint_as_float(half ? sr[33 + k] : sr[k + 1]);
-        const float e0 = ex2_approx(fmaf(s0, c2, neg_m));
-        const float e1 = ex2_approx(fmaf(s1, c2, neg_m));
-        acc[(k >> 1) & 3] += e0 + e1;
-        pk[k >> 1] = pack_bf16x2(e0, e1);
-      }
-      l_run = l_run * alpha + ((acc[0] + acc[1]) + (acc[2] + acc[3]));
-      // P stage s is free once PV_{j-2} has completed
-      if (j >= 2) {
-        w = mbar_wait(&bar_pv[s], ((j - 2) >> 1) & 1, p.wait_ns);
-        if (!__all_sync(0xffffffffu, w)) {
-          ok = false;
-          break;
-        }
-      }
-      // 128-byte swizzled K-major row: 16-byte unit u of row r sits at unit u ^ (r & 7)
-      uint8_t* prow = sP + s * kPBytes + r * 128;
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint4 v;
-        v.x = pk[4 * c + 0];
-        v.y = pk[4 * c + 1];
-        v.z = pk[4 * c + 2];
-        v.w = pk[4 * c + 3];
-        *reinterpret_cast<uint4*>(prow + (((half * 4 + c) ^ (r & 7)) << 4)) = v;
-      }
-      fence_proxy_async_smem();
-      if (__any_sync(0xffffffffu, rescale)) {
-        // O must hold the result of PV_{j-1} before it is rescaled in place
-        w = mbar_wait(&bar_pv[(j - 1) & 1], ((j - 1) >> 1) & 1, p.wait_ns);
-        if (!__all_sync(0xffffffffu, w)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
+      const float l_tot = l_part[r] + l_part[128 + r];
+      const float inv_l = 1.f / l_tot;
+      const bool valid = pos < it.pos1;
+      const int head = it.g * p.G + hh;
+      // This warp's 32 rows go out through its own 4 KB staging tile in the (now idle)
+      // P buffers, one 64-column slab at a time, with a 3-D TMA box (64 columns x
+      // heads x positions) -- unless some of its rows lie past the document's end.
+      const int r0 = quarter * 32;
+      const int rows_g = p.G < 32 ? p.G : 32;        // heads per box
+      const int pos_a = it.pos0 + r0 / p.G;
+      const bool warp_full = pos_a + (32 / rows_g) <= it.pos1;
+      uint8_t* stage = sP + warp * 4096;
+      __nv_bfloat16* orow = p.out + (it.q0 + pos) * p.ldo + static_cast<int64_t>(head) * kD;
 #pragma unroll 1
-        for (int c = half * 128; c < half * 128 + 128; c += 32) {
+      for (int sl = 2 * half; sl < 2 * half + 2; ++sl) {
+        uint4 v[8];
+#pragma unroll
+        for (int c2 = 0; c2 < 2; ++c2) {
           uint32_t o[32];
-          tmem_ld32(lane_base + c, o);
+          tmem_ld32(lane_base + sl * 64 + c2 * 32, o);
           tmem_ld_wait();
 #pragma unroll
-          for (int k = 0; k < 32; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * alpha);
-          tmem_st32(lane_base + c, o);
+          for (int q = 0; q < 4; ++q) {
+            v[c2 * 4 + q].x = pack_bf16x2(__uint_as_float(o[8 * q + 0]) * inv_l, __uint_as_float(o[8 * q + 1]) * inv_l);
+            v[c2 * 4 + q].y = pack_bf16x2(__uint_as_float(o[8 * q + 2]) * inv_l, __uint_as_float(o[8 * q + 3]) * inv_l);
+            v[c2 * 4 + q].z = pack_bf16x2(__uint_as_float(o[8 * q + 4]) * inv_l, __uint_as_float(o[8 * q + 5]) * inv_l);
+            v[c2 * 4 + q].w = pack_bf16x2(__uint_as_float(o[8 * q + 6]) * inv_l, __uint_as_float(o[8 * q + 7]) * inv_l);
+          }
         }
-        tmem_st_wait();
+        if (warp_full) {
+          uint8_t* row = stage + lane * 128;
+#pragma unroll
+          for (int u = 0; u < 8; ++u) *reinterpret_cast<uint4*>(row + ((u ^ (lane & 7)) << 4)) = v[u];
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_3d(&tm_o, stage, sl * 64, it.g * p.G + (r0 % p.G), static_cast<int32_t>(it.q0 + pos_a));
+            bulk_commit_group();
+            bulk_wait_group_read<0>();  // staging tile read before it is refilled
+          }
+          __syncwarp();
+        } else if (valid) {
+          uint4* dst = reinterpret_cast<uint4*>(orow + sl * 64);
+#pragma unroll
+          for (int u = 0; u < 8; ++u) dst[u] = v[u];
+        }
       }
       tc_fence_before();
-      mbar_arrive(&bar_p[s]);
+      // O read out and the staging tiles free: the next item may overwrite O and P
+      mbar_arrive(bar_ofree);
+      if (valid && half == 0 && p.lse) {
+        // natural-log softmax denominator in scaled-logit units
+        p.lse[(it.q0 + pos) * p.n_q + head] = (m_run + log2f(l_tot)) * 0.69314718055994531f;
+      }
+      J += it.nt;
+      ++n_it;
     }
-    // publish this half's row sum (every softmax thread arrives, also on failure)
-    l_part[half * 128 + r] = l_run;
-    mbar_arrive(bar_l);
+    if (lane == 0) bulk_wait_group<0>();
     if (!ok) {
       if (lane == 0) record_error(p.err, kErrTimeout | kSiteAttention);
       *abort_flag = 1;
-    } else {
-      // ---- epilogue: O / l -> bf16, this half's 128 columns
-      const int jl = nt - 1;
-      bool w = mbar_wait(&bar_pv[jl & 1], (jl >> 1) & 1, p.wait_ns) && mbar_wait(bar_l, 0, p.wait_ns);
-      if (!__all_sync(0xffffffffu, w)) {
-        if (lane == 0) record_error(p.err, kErrTimeout | kSiteAttention);
-        *abort_flag = 1;
-      } else {
-        tc_fence_after();
-        const float l_tot = l_part[r] + l_part[128 + r];
-        const float inv_l = 1.f / l_tot;
-        const bool valid = pos < pos1;
-        const int head = g * p.G + hh;
-        const bool full_tile = pos0 + p.P <= Lq;
-        __nv_bfloat16* orow = p.out + (q0 + pos) * p.ldo + static_cast<int64_t>(head) * kD;
-#pragma unroll 1
-        for (int c = half * 128; c < half * 128 + 128; c += 32) {
-          uint32_t o[32];
-          tmem_ld32(lane_base + c, o);
-          tmem_ld_wait();
-          uint4 v[4];
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            v[q].x = pack_bf16x2(__uint_as_float(o[8 * q + 0]) * inv_l, __uint_as_float(o[8 * q + 1]) * inv_l);
-            v[q].y = pack_bf16x2(__uint_as_float(o[8 * q + 2]) * inv_l, __uint_as_float(o[8 * q + 3]) * inv_l);
-            v[q].z = pack_bf16x2(__uint_as_float(o[8 * q + 4]) * inv_l, __uint_as_float(o[8 * q + 5]) * inv_l);
-            v[q].w = pack_bf16x2(__uint_as_float(o[8 * q + 6]) * inv_l, __uint_as_float(o[8 * q + 7]) * inv_l);
-          }
-          if (full_tile) {
-            // Full tile: stage O in the (now idle) Q tile, in the same 128-byte
-            // swizzled slabs; four 3-D TMA stores whose boxes match the Q boxes
-            // (positions x heads x 64 columns) write it after the CTA barrier.
-            uint8_t* row = sQ + (c >> 6) * kQSlab + r * 128;
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              const int unit = ((c & 63) >> 3) + q;  // 16-byte unit inside the 128-byte row
-              *reinterpret_cast<uint4*>(row + ((unit ^ (r & 7)) << 4)) = v[q];
-            }
-          } else if (valid) {
-            uint4* dst = reinterpret_cast<uint4*>(orow + c);
-#pragma unroll
-            for (int q = 0; q < 4; ++q) dst[q] = v[q];
-          }
-        }
-        if (full_tile) fence_proxy_async_smem();
-        if (valid && half == 0 && p.lse) {
-          // natural-log softmax denominator in scaled-logit units
-          p.lse[(q0 + pos) * p.n_q + head] = (m_run + log2f(l_tot)) * 0.69314718055994531f;
-        }
-      }
     }
   }
   tc_fence_before();
@@ -388,10 +462,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == kMmaWarp) {
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
-  } else if (threadIdx.x == 0 && pos0 + p.P <= Lq && !*abort_flag) {
-    tma_store_4d(&tm_o, sQ, 0, g * p.G, static_cast<int32_t>(q0 + pos0), 0);
-    bulk_commit_group();
-    bulk_wait_group<0>();
   }
 }
 
@@ -446,9 +516,12 @@ extern "C" kalm_status kalm_merged_attention(const kalm_bf16* q, int64_t ldq, co
     const uint64_t strides[3] = {kD * 2, static_cast<uint64_t>(ldq) * 2, 128};
     const uint32_t box[4] = {64, static_cast<uint32_t>(G), static_cast<uint32_t>(kBM / G), 4};
     if ((st = make_tmap_bf16(&tq, q, 4, dims, strides, box)) != KALM_OK) return st;
-    const uint64_t odims[4] = {64, static_cast<uint64_t>(n_q), static_cast<uint64_t>(total_q), 4};
-    const uint64_t ostrides[3] = {kD * 2, static_cast<uint64_t>(ldo) * 2, 128};
-    if ((st = make_tmap_bf16(&to, out, 4, odims, ostrides, box)) != KALM_OK) return st;
+    // O: 3-D view (256 columns, head, row); a box is one warp's 32 packed rows x 64 columns
+    const int gb = G < 32 ? G : 32;
+    const uint64_t odims[3] = {kD, static_cast<uint64_t>(n_q), static_cast<uint64_t>(total_q)};
+    const uint64_t ostrides[2] = {kD * 2, static_cast<uint64_t>(ldo) * 2};
+    const uint32_t obox[3] = {64, static_cast<uint32_t>(gb), static_cast<uint32_t>(32 / gb)};
+    if ((st = make_tmap_bf16(&to, out, 3, odims, ostrides, obox)) != KALM_OK) return st;
   }
   // K and V: 3-D views (64 columns, row, 64-column slab over all KV heads); a box is
   // one 64-key x 256-column tile of one KV head.
@@ -485,8 +558,14 @@ extern "C" kalm_status kalm_merged_attention(const kalm_bf16* q, int64_t ldq, co
   prm.scale_log2 = scale * 1.4426950408889634f;
   prm.wait_ns = kWaitNs;
   prm.err = device_error_word();
-  const int64_t grid = static_cast<int64_t>(last_tile_only ? 1 : prm.tiles_per_doc) * n_docs * n_kv;
-  if (grid > INT32_MAX) return fail(KALM_ERR_INVALID_ARG, "kalm_merged_attention: grid too large");
+  const int64_t items = static_cast<int64_t>(last_tile_only ? 1 : prm.tiles_per_doc) * n_docs * n_kv;
+  if (items > INT32_MAX) return fail(KALM_ERR_INVALID_ARG, "kalm_merged_attention: too many work items");
+  prm.n_items = static_cast<int>(items);
+  int sms = 0, dev = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (sms <= 0) sms = 148;
+  const int64_t grid = items < sms ? items : sms;  // persistent: one CTA per SM
   return check_cuda(launch_pdl(merged_attention_kernel, dim3(static_cast<unsigned>(grid)), dim3(kThreads), kSmem,
                                 static_cast<cudaStream_t>(stream), tq, tks, tvs, tkc, tvc, to, prm),
                     "launch merged_attention_kernel");
