@@ -32,6 +32,7 @@
 //     for all items of the CTA, so the next item's Q copy (as soon as the last S
 //     of the current item is done) and its first S product overlap the current
 //     item's last softmax, P V and O write-out.
+//   * Every role loads the next item's offsets while it works on the current one.
 //   * Warp roles: warps 0-7 softmax + epilogue, warp 8 TMA producer of Q and K,
 //     warp 10 TMA producer of V, warp 9 tensor-memory allocation and MMA issue.
 #include <cmath>
@@ -176,8 +177,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t J = 0;  // tile counter over all items of this CTA
       int n_it = 0;
       bool ok = true;
+      Item nxt = make_item(p, blockIdx.x);
       for (int w = blockIdx.x; w < p.n_items && ok && !*abort_flag; w += gridDim.x) {
-        const Item it = make_item(p, w);
+        const Item it = nxt;  // offsets are loaded one item ahead
+        if (w + static_cast<int>(gridDim.x) < p.n_items) nxt = make_item(p, w + gridDim.x);
         if (it.nt == 0) continue;
         if (!is_v) {
           if (n_it >= 1 && !mbar_wait(bar_qfree, (n_it - 1) & 1, p.wait_ns)) {
@@ -226,8 +229,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t J = 0;
       int n_it = 0;
       bool ok = true;
+      Item nxt = make_item(p, blockIdx.x);
       for (int w = blockIdx.x; w < p.n_items && ok && !*abort_flag; w += gridDim.x) {
-        const Item it = make_item(p, w);
+        const Item it = nxt;  // offsets are loaded one item ahead
+        if (w + static_cast<int>(gridDim.x) < p.n_items) nxt = make_item(p, w + gridDim.x);
         if (it.nt == 0) continue;
         ok = mbar_wait(bar_q, n_it & 1, p.wait_ns);
         if (!ok) break;
@@ -273,8 +278,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t J = 0;
     int n_it = 0;
     bool ok = true;
+    Item nxt = make_item(p, blockIdx.x);
     for (int w = blockIdx.x; w < p.n_items && ok; w += gridDim.x) {
-      const Item it = make_item(p, w);
+      const Item it = nxt;
+      if (w + static_cast<int>(gridDim.x) < p.n_items) nxt = make_item(p, w + gridDim.x);
       if (it.nt == 0) continue;
       const int pos = it.pos0 + r / p.G;      // decoder position of this row
       const int hh = r % p.G;                 // query head within the KV group
