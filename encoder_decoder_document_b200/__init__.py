@@ -17,7 +17,8 @@ from ._abi import KalmError, call, load, library_path  # noqa: F401
 __all__ = [
     "KalmError", "load", "library_path", "kalm_version", "kalm_device_check", "kalm_check_device_errors",
     "kalm_ragged_offsets", "kalm_chunk_pool", "kalm_linear", "kalm_cross_kv_proj", "kalm_merged_attention",
-    "kalm_yes_no_score", "kalm_broadcast_rows", "kalm_selftest_wait_timeout",
+    "kalm_yes_no_score", "kalm_broadcast_rows", "kalm_selftest_wait_timeout", "kalm_attention_items",
+    "kalm_attention_schedule",
 ]
 
 HEAD_DIM = 256
@@ -100,10 +101,11 @@ def kalm_merged_attention(q: torch.Tensor, k_self: torch.Tensor, v_self: torch.T
                           n_q: int, n_kv: int, out: torch.Tensor, scale: Optional[float] = None,
                           lse: Optional[torch.Tensor] = None, head_dim: int = HEAD_DIM,
                           in_off: Optional[torch.Tensor] = None, last_tile_only: bool = False,
-                          total_q: Optional[int] = None, stream=None) -> None:
+                          total_q: Optional[int] = None, order: Optional[torch.Tensor] = None, stream=None) -> None:
     """2-D row views: q/k/v self [input rows][...], out [q_off[-1] rows][>= n_q*D],
     k/v cross [pooled rows][>= n_kv*D].  ``in_off`` (optional) gives each document's
-    first input row; by default it is q_off."""
+    first input row; by default it is q_off.  ``order`` (optional) is a work order
+    from ``kalm_attention_schedule`` for the same offsets and sizes."""
     if scale is None:
         scale = head_dim ** -0.5
     if _ld(k_self) != _ld(v_self) or _ld(k_cross) != _ld(v_cross):
@@ -114,7 +116,20 @@ def kalm_merged_attention(q: torch.Tensor, k_self: torch.Tensor, v_self: torch.T
          _p(v_self, torch.bfloat16), _ld(k_self), _p(k_cross, torch.bfloat16), _p(v_cross, torch.bfloat16),
          _ld(k_cross), _p(q_off, torch.int64), _p(in_off, torch.int64), q.shape[0], _p(pool_off, torch.int64),
          n_docs, int(max_q), int(total_q), k_cross.shape[0], n_q, n_kv, head_dim, float(scale),
-         1 if last_tile_only else 0, _p(out, torch.bfloat16), _ld(out), _p(lse, torch.float32), _stream(stream))
+         1 if last_tile_only else 0, _p(order, torch.int32), _p(out, torch.bfloat16), _ld(out), _p(lse, torch.float32),
+         _stream(stream))
+
+
+def kalm_attention_items(n_docs: int, max_q: int, n_q: int, n_kv: int, last_tile_only: bool = False) -> int:
+    """Work items of one kalm_merged_attention call (-1 for rejected sizes)."""
+    return int(load().kalm_attention_items(n_docs, max_q, n_q, n_kv, 1 if last_tile_only else 0))
+
+
+def kalm_attention_schedule(q_off: torch.Tensor, pool_off: torch.Tensor, max_q: int, n_q: int, n_kv: int,
+                            order: torch.Tensor, last_tile_only: bool = False, stream=None) -> None:
+    """Write a heaviest-first work order for kalm_merged_attention into ``order`` (int32)."""
+    call("kalm_attention_schedule", _p(q_off, torch.int64), _p(pool_off, torch.int64), q_off.numel() - 1, int(max_q),
+         n_q, n_kv, 1 if last_tile_only else 0, _p(order, torch.int32), order.numel(), _stream(stream))
 
 
 def kalm_yes_no_score(hidden: torch.Tensor, q_off: torch.Tensor, w_yes: torch.Tensor, w_no: torch.Tensor,

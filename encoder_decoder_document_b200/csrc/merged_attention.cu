@@ -79,6 +79,7 @@ struct AttnParams {
   int P;            // decoder positions per tile = 128 / G
   int tiles_per_doc;
   int n_items;
+  const int32_t* order;  // work items sorted heaviest first (kalm_attention_schedule); NULL: index order
   float scale_log2;  // scale * log2(e)
   uint64_t wait_ns;
   uint32_t* err;
@@ -106,6 +107,35 @@ __device__ __forceinline__ Item make_item(const AttnParams& p, int w) {
   it.pos1 = min(it.pos0 + p.P, it.Lq);
   it.n_self = it.pos0 < it.Lq ? (it.pos1 + kBKV - 1) / kBKV : 0;
   it.nt = it.pos0 < it.Lq ? it.n_self + (it.Nc + kBKV - 1) / kBKV : 0;  // 0: nothing to do
+  return it;
+}
+
+constexpr int kNoMore = -2;  // item_at: this CTA has no further items
+constexpr int kSkip = -1;    // item_at: no item at this pass
+
+// Work item of this CTA's k-th pass.  Without a work order CTA c takes items
+// c, c + grid, c + 2 grid, ...  With one (items sorted heaviest first), it takes
+// positions in snake order -- c in even passes, grid - 1 - c in odd ones -- so
+// every CTA gets a similar mix of heavy and light items.
+__device__ __forceinline__ int item_at(const AttnParams& p, int k) {
+  const int64_t base = static_cast<int64_t>(k) * gridDim.x;
+  if (base >= p.n_items) return kNoMore;
+  const int c = static_cast<int>(blockIdx.x);
+  const int64_t idx = base + ((p.order && (k & 1)) ? static_cast<int>(gridDim.x) - 1 - c : c);
+  if (idx >= p.n_items) return kSkip;
+  if (!p.order) return static_cast<int>(idx);
+  const int w = p.order[idx];
+  if (w < 0 || w >= p.n_items) {  // not a work order of this launch: flag it, skip the entry
+    record_error(p.err, kErrDeviceArg | kSiteAttention);
+    return kSkip;
+  }
+  return w;
+}
+
+__device__ __forceinline__ Item load_item(const AttnParams& p, int w) {
+  if (w >= 0) return make_item(p, w);
+  Item it{};
+  it.nt = 0;
   return it;
 }
 
@@ -177,10 +207,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t J = 0;  // tile counter over all items of this CTA
       int n_it = 0;
       bool ok = true;
-      Item nxt = make_item(p, blockIdx.x);
-      for (int w = blockIdx.x; w < p.n_items && ok && !*abort_flag; w += gridDim.x) {
+      int wc = item_at(p, 0);
+      Item nxt = load_item(p, wc);
+      for (int pass = 0; wc != kNoMore && ok && !*abort_flag; ++pass) {
         const Item it = nxt;  // offsets are loaded one item ahead
-        if (w + static_cast<int>(gridDim.x) < p.n_items) nxt = make_item(p, w + gridDim.x);
+        wc = item_at(p, pass + 1);
+        nxt = load_item(p, wc);
         if (it.nt == 0) continue;
         if (!is_v) {
           if (n_it >= 1 && !mbar_wait(bar_qfree, (n_it - 1) & 1, p.wait_ns)) {
@@ -229,10 +261,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t J = 0;
       int n_it = 0;
       bool ok = true;
-      Item nxt = make_item(p, blockIdx.x);
-      for (int w = blockIdx.x; w < p.n_items && ok && !*abort_flag; w += gridDim.x) {
+      int wc = item_at(p, 0);
+      Item nxt = load_item(p, wc);
+      for (int pass = 0; wc != kNoMore && ok && !*abort_flag; ++pass) {
         const Item it = nxt;  // offsets are loaded one item ahead
-        if (w + static_cast<int>(gridDim.x) < p.n_items) nxt = make_item(p, w + gridDim.x);
+        wc = item_at(p, pass + 1);
+        nxt = load_item(p, wc);
         if (it.nt == 0) continue;
         ok = mbar_wait(bar_q, n_it & 1, p.wait_ns);
         if (!ok) break;
@@ -278,10 +312,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t J = 0;
     int n_it = 0;
     bool ok = true;
-    Item nxt = make_item(p, blockIdx.x);
-    for (int w = blockIdx.x; w < p.n_items && ok; w += gridDim.x) {
+    int wc = item_at(p, 0);
+    Item nxt = load_item(p, wc);
+    for (int pass = 0; wc != kNoMore && ok; ++pass) {
       const Item it = nxt;
-      if (w + static_cast<int>(gridDim.x) < p.n_items) nxt = make_item(p, w + gridDim.x);
+      wc = item_at(p, pass + 1);
+      nxt = load_item(p, wc);
       if (it.nt == 0) continue;
       const int pos = it.pos0 + r / p.G;      // decoder position of this row
       const int hh = r % p.G;                 // query head within the KV group
@@ -472,6 +508,40 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
+// Work order for the persistent kernel: every item's cost (its K/V tiles plus one
+// for the per-item Q copy and epilogue) is computed from the offsets, and the
+// items are counting-sorted by cost, heaviest first.  One CTA; the order of equal
+// costs is whatever the atomics give (each item's result does not depend on
+// which CTA computes it).
+constexpr int kSchedThreads = 1024;
+constexpr int kSchedBins = 64;
+
+__device__ __forceinline__ int item_cost_bin(const AttnParams& p, int w) {
+  const Item it = make_item(p, w);
+  const int cost = it.nt > 0 ? it.nt + 1 : 0;
+  return kSchedBins - 1 - min(cost, kSchedBins - 1);  // bin 0 = heaviest
+}
+
+__global__ void __launch_bounds__(kSchedThreads) attention_schedule_kernel(const AttnParams p, int32_t* order) {
+  __shared__ int hist[kSchedBins];
+  __shared__ int next[kSchedBins];
+  pdl_launch_dependents();
+  pdl_wait_predecessor();
+  if (threadIdx.x < kSchedBins) hist[threadIdx.x] = 0;
+  __syncthreads();
+  for (int w = threadIdx.x; w < p.n_items; w += kSchedThreads) atomicAdd(&hist[item_cost_bin(p, w)], 1);
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int run = 0;
+    for (int b = 0; b < kSchedBins; ++b) {
+      next[b] = run;
+      run += hist[b];
+    }
+  }
+  __syncthreads();
+  for (int w = threadIdx.x; w < p.n_items; w += kSchedThreads) order[atomicAdd(&next[item_cost_bin(p, w)], 1)] = w;
+}
+
 }  // namespace
 
 kalm_status setup_attention_kernels() {
@@ -489,8 +559,8 @@ extern "C" kalm_status kalm_merged_attention(const kalm_bf16* q, int64_t ldq, co
                                              const int64_t* in_off, int64_t total_in, const int64_t* pool_off,
                                              int32_t n_docs, int32_t max_q, int64_t total_q, int64_t total_pool,
                                              int32_t n_q, int32_t n_kv, int32_t head_dim, float scale,
-                                             int32_t last_tile_only, kalm_bf16* out, int64_t ldo, float* lse,
-                                             kalm_stream_t stream) {
+                                             int32_t last_tile_only, const int32_t* order, kalm_bf16* out,
+                                             int64_t ldo, float* lse, kalm_stream_t stream) {
   kalm_status st = ensure_device(nullptr);
   if (st != KALM_OK) return st;
   if (head_dim != kD) return fail(KALM_ERR_UNSUPPORTED, "kalm_merged_attention: head_dim=%d (only 256)", head_dim);
@@ -562,6 +632,7 @@ extern "C" kalm_status kalm_merged_attention(const kalm_bf16* q, int64_t ldq, co
   prm.G = G;
   prm.P = kBM / G;
   prm.tiles_per_doc = (max_q + prm.P - 1) / prm.P;
+  prm.order = order;
   prm.scale_log2 = scale * 1.4426950408889634f;
   prm.wait_ns = kWaitNs;
   prm.err = device_error_word();
@@ -576,4 +647,47 @@ extern "C" kalm_status kalm_merged_attention(const kalm_bf16* q, int64_t ldq, co
   return check_cuda(launch_pdl(merged_attention_kernel, dim3(static_cast<unsigned>(grid)), dim3(kThreads), kSmem,
                                 static_cast<cudaStream_t>(stream), tq, tks, tvs, tkc, tvc, to, prm),
                     "launch merged_attention_kernel");
+}
+
+extern "C" int64_t kalm_attention_items(int32_t n_docs, int32_t max_q, int32_t n_q, int32_t n_kv,
+                                        int32_t last_tile_only) {
+  if (n_docs < 0 || n_q <= 0 || n_kv <= 0 || n_q % n_kv || max_q < 0 || max_q > KALM_MAX_QUERY_TOKENS) return -1;
+  const int G = n_q / n_kv;
+  if (kBM % G) return -1;
+  const int P = kBM / G;
+  const int64_t tiles = last_tile_only ? 1 : (max_q + P - 1) / P;
+  return max_q == 0 ? 0 : tiles * n_docs * n_kv;
+}
+
+extern "C" kalm_status kalm_attention_schedule(const int64_t* q_off, const int64_t* pool_off, int32_t n_docs,
+                                               int32_t max_q, int32_t n_q, int32_t n_kv, int32_t last_tile_only,
+                                               int32_t* order, int64_t order_len, kalm_stream_t stream) {
+  kalm_status st = ensure_device(nullptr);
+  if (st != KALM_OK) return st;
+  const int64_t items = kalm_attention_items(n_docs, max_q, n_q, n_kv, last_tile_only);
+  if (items < 0)
+    return fail(KALM_ERR_INVALID_ARG, "kalm_attention_schedule: bad sizes (n_docs=%d n_q=%d n_kv=%d max_q=%d)", n_docs,
+                n_q, n_kv, max_q);
+  if (items > INT32_MAX) return fail(KALM_ERR_INVALID_ARG, "kalm_attention_schedule: too many work items");
+  if (order_len < items)
+    return fail(KALM_ERR_INVALID_ARG, "kalm_attention_schedule: order_len=%lld < %lld work items",
+                (long long)order_len, (long long)items);
+  if (items == 0) return KALM_OK;
+  if (!q_off || !pool_off || !order) return fail(KALM_ERR_INVALID_ARG, "kalm_attention_schedule: NULL pointer");
+  AttnParams prm{};
+  prm.q_off = q_off;
+  prm.in_off = nullptr;
+  prm.last_only = last_tile_only ? 1 : 0;
+  prm.pool_off = pool_off;
+  prm.n_docs = n_docs;
+  prm.n_q = n_q;
+  prm.n_kv = n_kv;
+  prm.G = n_q / n_kv;
+  prm.P = kBM / prm.G;
+  prm.tiles_per_doc = (max_q + prm.P - 1) / prm.P;
+  prm.n_items = static_cast<int>(items);
+  prm.err = device_error_word();
+  return check_cuda(launch_pdl(attention_schedule_kernel, dim3(1), dim3(kSchedThreads), 0,
+                               static_cast<cudaStream_t>(stream), prm, order),
+                    "launch attention_schedule_kernel");
 }

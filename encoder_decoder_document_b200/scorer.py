@@ -25,7 +25,8 @@ import numpy as np
 import torch
 
 from . import (kalm_broadcast_rows, kalm_chunk_pool, kalm_cross_kv_proj, kalm_device_check, kalm_linear,
-               kalm_merged_attention, kalm_ragged_offsets, kalm_yes_no_score)
+               kalm_merged_attention, kalm_ragged_offsets, kalm_yes_no_score, kalm_attention_items,
+               kalm_attention_schedule)
 
 HEAD_DIM = 256
 
@@ -103,6 +104,9 @@ class FBNLScorer:
         self.x = torch.empty(rows, H, dtype=torch.bfloat16, **kw)
         # (yes, no, margin, score) rows of one buffer: one device->host copy per query
         self.result = torch.empty(4, n_docs, dtype=torch.float32, **kw)
+        # work order of the full-layer attention launches (same costs in every layer)
+        self.order = torch.empty(max(kalm_attention_items(n_docs, lq, self.n_q, self.n_kv), 1), dtype=torch.int32,
+                                 **kw)
         self.yes, self.no, self.margin, self.score = self.result[0], self.result[1], self.result[2], self.result[3]
         self.graphs = None
 
@@ -124,6 +128,8 @@ class FBNLScorer:
         self._mark("offsets")
         kalm_ragged_offsets(self.q_len, self.q_off, None, 1)
         self._mark("offsets")
+        kalm_attention_schedule(self.q_off, self.pool_off, self.lq, self.n_q, self.n_kv, self.order)
+        self._mark("schedule")
         kalm_chunk_pool(self.enc, self.tok_off, self.doc_len, self.pooled, self.pool_off, self.total_pooled,
                         self.chunk)
         self._mark("chunk_pool")
@@ -151,7 +157,7 @@ class FBNLScorer:
         q, ks, vs = self.qkv_views()
         kc, vc = self.cross_views(l)
         kalm_merged_attention(q, ks, vs, kc, vc, self.q_off, self.pool_off, self.lq, self.n_q, self.n_kv, self.o,
-                              self.scale)
+                              self.scale, order=self.order)
         self._mark("merged_attention")
 
     def layer_out(self, l: int) -> None:
@@ -179,7 +185,7 @@ class FBNLScorer:
             q, ks, vs = self.qkv_views()
             in_off = None
         kalm_merged_attention(q, ks, vs, kc, vc, self.q_off, self.pool_off, Lq, self.n_q, self.n_kv, self.o,
-                              self.scale, in_off=in_off, last_tile_only=last)
+                              self.scale, in_off=in_off, last_tile_only=last, order=None if last else self.order)
         self._mark("merged_attention")
         if last:
             # only each document's final row reaches the readout

@@ -189,6 +189,11 @@ kalm_status kalm_cross_kv_proj(const kalm_bf16* pooled, int64_t pooled_ld, int64
  *         positions) that holds each document's last decoder row; the other
  *         rows of `out` are left untouched.  Enough when only the final
  *         position is read afterwards (the yes/no readout of the last layer).
+ * order   int32[kalm_attention_items(...)] written by kalm_attention_schedule
+ *         for the same offsets and sizes, or NULL.  Only the order in which the
+ *         persistent CTAs take the work items changes (heaviest first, spread
+ *         over the CTAs); the results are the same.  An entry outside the item
+ *         range is skipped and flagged in the device error word.
  * out     [total_q][ldo] bf16, head h at element h*head_dim
  * lse     fp32 [total_q][n_q] or NULL: natural log of each row's softmax
  *         denominator, in scaled-logit units.
@@ -201,8 +206,27 @@ kalm_status kalm_merged_attention(const kalm_bf16* q, int64_t ldq,
                                   const int64_t* pool_off, int32_t n_docs, int32_t max_q,
                                   int64_t total_q, int64_t total_pool,
                                   int32_t n_q, int32_t n_kv, int32_t head_dim, float scale,
-                                  int32_t last_tile_only, kalm_bf16* out, int64_t ldo, float* lse,
-                                  kalm_stream_t stream);
+                                  int32_t last_tile_only, const int32_t* order,
+                                  kalm_bf16* out, int64_t ldo, float* lse, kalm_stream_t stream);
+
+/* Work items of one kalm_merged_attention call (one query tile of 128/(n_q/n_kv)
+ * decoder positions x one KV head x one document): ceil(max_q / (128 n_kv / n_q))
+ * * n_docs * n_kv, or n_docs * n_kv with last_tile_only.  Host-only
+ * arithmetic; returns -1 for sizes kalm_merged_attention rejects.  Scheduling
+ * aid for the step-3 kernel; the pages have no counterpart (they describe what
+ * the attention computes, not how a GPU divides it). */
+int64_t kalm_attention_items(int32_t n_docs, int32_t max_q, int32_t n_q, int32_t n_kv, int32_t last_tile_only);
+
+/* Work order for kalm_merged_attention: writes order[0 .. items-1], a
+ * permutation of the work items sorted by cost (the item's K/V tiles, from
+ * q_off and pool_off), heaviest first.  The costs are the same for every layer
+ * of a query, so one order serves all its layers.  order is caller-owned device
+ * memory of at least order_len >= kalm_attention_items(...) entries; stream-
+ * ordered, one single-CTA kernel; nothing allocated.  Errors: sizes as
+ * kalm_merged_attention, order_len too small -> KALM_ERR_INVALID_ARG. */
+kalm_status kalm_attention_schedule(const int64_t* q_off, const int64_t* pool_off, int32_t n_docs,
+                                    int32_t max_q, int32_t n_q, int32_t n_kv, int32_t last_tile_only,
+                                    int32_t* order, int64_t order_len, kalm_stream_t stream);
 
 /* Step 4 - yes/no readout at each document's final decoder position.
  * "What this is": score = softmax([logit_yes, logit_no])[yes] at the final

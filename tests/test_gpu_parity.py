@@ -180,7 +180,7 @@ def _attn_arrays(rng, lq, nc, n_q, n_kv, q_std=0.5, k_std=0.5, kc_mult=1.0):
                 vc=rand_bf16(rng, (C, n_kv, D)), q_off=q_off, p_off=p_off, n_q=n_q, n_kv=n_kv)
 
 
-def _attn_run(kalm, a, p_off=None, scale=1.0 / 16):
+def _attn_run(kalm, a, p_off=None, scale=1.0 / 16, order=None):
     """Run the kernel on fused row layouts as the scorer uses them: [q | k | v] and [k_cross | v_cross]."""
     D, n_q, n_kv = 256, a["n_q"], a["n_kv"]
     q_off = a["q_off"]
@@ -196,7 +196,7 @@ def _attn_run(kalm, a, p_off=None, scale=1.0 / 16):
     lse = torch.full((R, n_q), float("nan"), dtype=torch.float32, device="cuda")
     kalm.kalm_merged_attention(qkv[:, : n_q * D], qkv[:, n_q * D: n_q * D + w], qkv[:, n_q * D + w:],
                                kvc[:, :w], kvc[:, w:], i64(q_off), i64(p_off), int(np.diff(q_off).max()), n_q,
-                               n_kv, out, scale, lse)
+                               n_kv, out, scale, lse, order=order)
     kalm.kalm_check_device_errors()
     return from_dev(out).reshape(R, n_q, D), lse.cpu().numpy().astype(np.float64)
 
@@ -571,3 +571,77 @@ def test_score_stream_matches_single_queries(kalm):
     kalm.kalm_check_device_errors()
     for k in range(len(qs)):
         np.testing.assert_array_equal(outs[k].numpy(), singles[k])
+
+
+def _item_costs(q_off, p_off, max_q, n_q, n_kv):
+    """Host restatement of the work items' costs (K/V tiles + 1, 0 for an empty tile),
+    in the kernel's item numbering: item w = tile t (heaviest first), KV head, document."""
+    G = n_q // n_kv
+    P = 128 // G
+    n = len(q_off) - 1
+    tiles = -(-max_q // P)
+    costs = []
+    for w in range(tiles * n * n_kv):
+        rem = w % (n * n_kv)
+        d = rem // n_kv
+        t = tiles - 1 - w // (n * n_kv)
+        lq, nc = int(q_off[d + 1] - q_off[d]), int(p_off[d + 1] - p_off[d])
+        pos0 = t * P
+        if pos0 >= lq:
+            costs.append(0)
+            continue
+        pos1 = min(pos0 + P, lq)
+        costs.append(-(-pos1 // 64) + -(-nc // 64) + 1)
+    return np.array(costs)
+
+
+@pytest.mark.parametrize("lq,nc,n_q,n_kv", [
+    ([128] * 100, list(range(16, 256, 2))[:100], 4, 1),
+    ([1, 2, 31, 33, 65, 130, 512], [0, 5, 64, 65, 128, 129, 256], 4, 1),
+    ([256, 100, 17], [75, 256, 3], 8, 4),
+])
+def test_attention_schedule_sorted_permutation(kalm, lq, nc, n_q, n_kv):
+    """The work order is a permutation of the items, heaviest first by the host cost."""
+    q_off = np.concatenate([[0], np.cumsum(lq)])
+    p_off = np.concatenate([[0], np.cumsum(nc)])
+    max_q = max(lq)
+    n_items = kalm.kalm_attention_items(len(lq), max_q, n_q, n_kv)
+    order = torch.full((n_items + 3,), -7, dtype=torch.int32, device="cuda")
+    kalm.kalm_attention_schedule(i64(q_off), i64(p_off), max_q, n_q, n_kv, order)
+    kalm.kalm_check_device_errors()
+    got = order.cpu().numpy()
+    assert sorted(got[:n_items].tolist()) == list(range(n_items))
+    assert got[n_items:].tolist() == [-7, -7, -7]          # nothing written past the items
+    costs = _item_costs(q_off, p_off, max_q, n_q, n_kv)
+    assert (np.diff(costs[got[:n_items]]) <= 0).all()
+
+
+def test_attention_order_gives_identical_results(kalm):
+    """Following a work order changes only which CTA computes an item: outputs and
+    log-sum-exps are bit-identical to the index order, and both match the oracle."""
+    rng = np.random.default_rng(71)
+    lq = [int(x) for x in rng.integers(1, 300, 37)]
+    nc = [int(x) for x in rng.integers(0, 257, 37)]
+    a = _attn_arrays(rng, lq, nc, 4, 1)
+    n_items = kalm.kalm_attention_items(len(lq), max(lq), 4, 1)
+    order = torch.empty(n_items, dtype=torch.int32, device="cuda")
+    kalm.kalm_attention_schedule(i64(a["q_off"]), i64(a["p_off"]), max(lq), 4, 1, order)
+    o1, l1 = _attn_run(kalm, a)
+    o2, l2 = _attn_run(kalm, a, order=order)
+    assert np.array_equal(o1, o2) and np.array_equal(l1, l2)
+    want, _ = _attn_oracle(a)
+    _check_attn(o2, want)
+
+
+def test_attention_order_out_of_range_is_flagged(kalm):
+    """Entries outside the item range are skipped (nothing written) and flagged."""
+    from encoder_decoder_document_b200 import KalmError
+    rng = np.random.default_rng(72)
+    a = _attn_arrays(rng, [64, 64], [10, 20], 4, 1)
+    n_items = kalm.kalm_attention_items(2, 64, 4, 1)
+    order = torch.tensor([n_items, -1] * n_items, dtype=torch.int32, device="cuda")[:n_items]
+    with pytest.raises(KalmError) as e:
+        _attn_run(kalm, a, order=order)
+    assert e.value.name == "KALM_ERR_DEVICE_ARG"
+    with pytest.raises(KalmError):
+        kalm.kalm_attention_schedule(i64(a["q_off"]), i64(a["p_off"]), 64, 4, 1, order[:1])  # too short
