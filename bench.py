@@ -47,6 +47,7 @@ def parse():
     ap.add_argument("--impl", default="kalm", choices=["kalm", "reference"])
     ap.add_argument("--cpu-sample-docs", type=int, default=0, help="documents in the oracle sample (0 = auto)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-pool-sweep", action="store_true", help="skip the pooling-only sweep at 1024/4096 docs")
     return ap.parse_args()
 
 
@@ -108,7 +109,56 @@ def workload(q):
     w["merged_attention"] = int(full_attn * (L - 1) + last_attn)
     w["o_proj"] = int(2 * nq * D * H * (rows * (L - 1) + n))
     w["total_flops"] = w["cross_kv_proj"] + w["qkv_proj"] + w["merged_attention"] + w["o_proj"]
+    # unfused algorithmic bytes (each operand read once, each result written once), for the
+    # arithmetic-intensity bound min(peak, AI * HBM)
+    P_ = int(nc.sum())
+    w["bytes"] = {
+        "cross_kv_proj": 2 * (P_ * H + L * 2 * nkv * D * H + P_ * L * 2 * nkv * D),
+        "qkv_proj": 2 * ((lq + rows * (L - 1)) * (H + (nq + 2 * nkv) * D) + L * (nq + 2 * nkv) * D * H),
+        "merged_attention": 2 * (L - 1) * (rows * (2 * nq + 2 * nkv) * D + P_ * 2 * nkv * D)
+                            + 2 * (n * P * 2 * nq * D + rows * 2 * nkv * D + P_ * 2 * nkv * D),
+        "o_proj": 2 * ((rows * (L - 1) + n) * (nq * D + 2 * H) + L * H * nq * D),
+    }
     return w
+
+
+def pool_sweep(doc_counts=(1024, 4096), reps=10):
+    """The pooling kernel alone at the throughput-sweep shapes with many documents
+    (hidden 640, log-normal lengths, median 200, clipped to [1, 1024]): bytes moved,
+    median time of `reps` calls (L2 flushed before each, CUDA events), GB/s."""
+    import torch
+    import synthetic
+    from encoder_decoder_document_b200 import kalm_chunk_pool, kalm_ragged_offsets
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device="cuda")
+    gen = torch.Generator(device="cuda")
+    out = []
+    for n in doc_counts:
+        lens = synthetic.draw_lengths(synthetic.CONFIGS["sweep"]["len"], n, np.random.default_rng([4, n]))
+        H = synthetic.CONFIGS["sweep"]["hidden"]
+        total = int(lens.sum())
+        nc = (lens.astype(np.int64) + 3) // 4
+        gen.manual_seed(4 * 100003 + n)
+        enc = torch.randn(total, H, device="cuda", generator=gen).to(torch.bfloat16)
+        len_d = torch.from_numpy(lens).cuda()
+        tok_off = torch.empty(n + 1, dtype=torch.int64, device="cuda")
+        pool_off = torch.empty(n + 1, dtype=torch.int64, device="cuda")
+        kalm_ragged_offsets(len_d, tok_off, pool_off, 4)
+        pooled = torch.empty(int(nc.sum()), H, dtype=torch.bfloat16, device="cuda")
+        ts = []
+        for i in range(reps + 2):
+            flush.fill_(1.0)
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            kalm_chunk_pool(enc, tok_off, len_d, pooled, pool_off, pooled.shape[0], 4)
+            b.record()
+            b.synchronize()
+            if i >= 2:
+                ts.append(a.elapsed_time(b))
+        us = 1e3 * statistics.median(ts)
+        byts = int((total + int(nc.sum())) * H * 2 + 8 * n)
+        out.append({"docs": n, "encoder_tokens": total, "bytes": byts, "us": us, "gbs": byts / (us * 1e-6) / 1e9})
+        del enc, pooled
+    return out
 
 
 class Clocks:
@@ -239,6 +289,7 @@ def main():
     out_h = torch.empty(4, q.n_docs, dtype=torch.float32).pin_memory()
     sc.load_inputs(enc_h, len_h, x0_h)
     sc.capture(instrument=True)
+    launches_per_step = sc.launches
     stream = torch.cuda.current_stream()
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device="cuda")
 
@@ -315,10 +366,32 @@ def main():
         b.synchronize()
         serial_ms.append(a.elapsed_time(b))
     serial_total = sum(serial_ms[max(args.warmup, 3):])
+
+    # ---------------- persistent-cache regime: the same documents against many queries; the
+    # documents' pooled vectors and cross K/V are built once, each query runs the decoder only
+    sc.cache_documents(enc_h, len_h)
+    dec_graph = sc.graphs_decode[sc.slot]
+    dec_ms = []
+    for i in range(max(args.warmup, 3) + args.steps):
+        a, b = step_timed(dec_graph)
+        b.synchronize()
+        if i >= max(args.warmup, 3):
+            dec_ms.append(a.elapsed_time(b))
+    x0s = [x0_h] * n_e2e
+    sc.score_cached_stream(x0s[: max(args.warmup, 3)], [outs[k % 2] for k in range(max(args.warmup, 3))])
+    torch.cuda.synchronize()
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    sc.score_cached_stream(x0s, [outs[k % 2] for k in range(n_e2e)])
+    b.record(stream)
+    b.synchronize()
+    dec_e2e_total = a.elapsed_time(b)
+    dec_total = sum(dec_ms)
     if world > 1:
-        t = torch.tensor([e2e_total, serial_total], device="cuda", dtype=torch.float64)
+        t = torch.tensor([e2e_total, serial_total, dec_total, dec_e2e_total], device="cuda", dtype=torch.float64)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_total, serial_total = float(t[0].item()), float(t[1].item())
+        e2e_total, serial_total, dec_total, dec_e2e_total = (float(x) for x in t.tolist())
     kalm_check_device_errors()
     h2d = enc_h.numel() * 2 + len_h.numel() * 4 + x0_h.numel() * 2
     d2h = out_h.numel() * 4
@@ -334,9 +407,19 @@ def main():
         kern[k]["tflops"] = w[k] / (kern[k]["us_per_step"] * 1e-6) / 1e12
     dom = max(tensor_kernels, key=lambda k: kern[k]["share"])
     dom_ach = kern[dom]["tflops"]
+    ai = w[dom] / w["bytes"][dom]
+    ai_bound = min(pk["bf16"], ai * pk["hbm"] / 1e3)
     roofline = {"kernel": dom, "bound": "tensor", "achieved": dom_ach, "peak": pk["bf16"], "unit": "TFLOP/s",
                 "frac": dom_ach / pk["bf16"], "traffic": traffic(dom),
-                "peak_source": f"{pk['source']} dense bf16 burst (cuBLAS), of measured"}
+                "peak_source": f"{pk['source']} dense bf16 burst (cuBLAS), of measured",
+                "frac_sustained": dom_ach / pk["bf16_sustained"], "peak_sustained": pk["bf16_sustained"],
+                "ai_flop_per_byte": ai, "ai_bound": ai_bound, "frac_of_ai_bound": dom_ach / ai_bound}
+    for k in tensor_kernels:
+        ai_k = w[k] / w["bytes"][k]
+        kern[k]["frac_burst"] = kern[k]["tflops"] / pk["bf16"]
+        kern[k]["frac_sustained"] = kern[k]["tflops"] / pk["bf16_sustained"]
+        kern[k]["ai_flop_per_byte"] = ai_k
+        kern[k]["frac_of_ai_bound"] = kern[k]["tflops"] / min(pk["bf16"], ai_k * pk["hbm"] / 1e3)
     pool_gbs = w["pool_bytes"] / (kern["chunk_pool"]["avg_us"] * 1e-6) / 1e9
     attn_proj_us = sum(kern[k]["us_per_step"] for k in ("merged_attention", "cross_kv_proj") if k in kern)
     attn_proj_flops = w["cross_kv_proj"] + w["merged_attention"]
@@ -345,6 +428,8 @@ def main():
 
     if rank == 0:
         cb = None
+        sweep = None if args.no_pool_sweep else [dict(x, peak_gbs=pk["hbm"], frac=x["gbs"] / pk["hbm"])
+                                                 for x in pool_sweep()]
         if not args.no_cpu_baseline and world == 1:
             cb = cpu_baseline(q, args.cpu_sample_docs or q.n_docs)
         line = {
@@ -377,7 +462,17 @@ def main():
                     "serial": {"value": world * q.n_docs * args.steps / (serial_total / 1e3),
                                "ms_per_step": serial_total / args.steps,
                                "how": "copy in, replay, copy out, one step at a time"}},
-            "gpu_launches": sc.launches * args.steps,
+            "decode_only": {"value": world * q.n_docs * args.steps / (dec_total / 1e3), "unit": UNIT,
+                            "ms_per_step": dec_total / args.steps,
+                            "e2e": {"value": world * q.n_docs * n_e2e / (dec_e2e_total / 1e3), "unit": UNIT,
+                                    "h2d_bytes_per_step": x0_h.numel() * 2, "d2h_bytes_per_step": d2h},
+                            "how": "persistent-cache regime: the documents' pooled vectors and every layer's cross "
+                                   "K/V built once (FBNLScorer.cache_documents); each step is one query through "
+                                   "the decoder-only graph (L2 flushed before each step); e2e through "
+                                   "FBNLScorer.score_cached_stream with the query input copied in and scores read "
+                                   "back"},
+            "pool_sweep": sweep,
+            "gpu_launches": launches_per_step * args.steps,
             "clocks": clk,
             "cpu_baseline": cb,
         }

@@ -71,6 +71,8 @@ class FBNLScorer:
         self.prune = prune
         self._shape = None
         self.graph: Optional[torch.cuda.CUDAGraph] = None
+        self.graphs = None
+        self.graphs_decode = None
         # optional per-launch timing: (label, event) recorded after every entry-point call
         self.marks: Optional[list] = None
         self.launches = 0  # kernel launches issued by the last forward()
@@ -109,6 +111,7 @@ class FBNLScorer:
                                  **kw)
         self.yes, self.no, self.margin, self.score = self.result[0], self.result[1], self.result[2], self.result[3]
         self.graphs = None
+        self.graphs_decode = None
 
     def use_slot(self, i: int) -> None:
         """Point the input buffers at slot i (for the next forward() or capture)."""
@@ -200,14 +203,13 @@ class FBNLScorer:
                           self.margin)
         self._mark("yes_no_score")
 
-    def forward(self) -> None:
-        """All steps on the current stream, from the inputs in self.enc / doc_len / x0."""
-        self.launches = 0
-        if self.marks is not None:
-            self._mark("start")
-            self.launches = 0
+    def documents(self) -> None:
+        """The document side: offsets, the pooled document cache and every layer's cross K/V."""
         self.pool()
         self.cross_kv()
+
+    def decode(self) -> None:
+        """The query side: the decoder stack over the cached cross K/V, then the readout."""
         kalm_broadcast_rows(self.x0, self.q_off, self.x)
         self._mark("broadcast")
         for l in range(self.L):
@@ -216,6 +218,20 @@ class FBNLScorer:
             else:
                 self.layer(l)
         self.readout()
+
+    def forward(self, cached: bool = False) -> None:
+        """All steps on the current stream, from the inputs in self.enc / doc_len / x0.
+
+        With ``cached`` only decode() runs: the documents' offsets, work order and
+        cross K/V from the last full forward over the same documents are reused
+        (the persistent-cache regime: one document set, many queries)."""
+        self.launches = 0
+        if self.marks is not None:
+            self._mark("start")
+            self.launches = 0
+        if not cached:
+            self.documents()
+        self.decode()
 
     def capture(self, instrument: bool = False) -> None:
         """Record forward() as a CUDA graph (buffers must stay allocated).
@@ -240,6 +256,13 @@ class FBNLScorer:
             with torch.cuda.graph(g):
                 self.forward()
             self.graphs.append(g)
+        self.graphs_decode = []
+        for i in range(2):  # decode-only graphs (persistent-cache regime), one per input slot
+            self.use_slot(i)
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                self.forward(cached=True)
+            self.graphs_decode.append(g)
         self.use_slot(slot)
         self.graph = self.graphs[slot]
         self.graph_inst = None
@@ -318,6 +341,51 @@ class FBNLScorer:
             i = k % 2
             comp.wait_event(self._ready[i])
             self.graphs[i].replay()
+            self._free[i].record(comp)
+            outs[k].copy_(self.result, non_blocking=True)
+
+    def cache_documents(self, enc_host: torch.Tensor, doc_len_host: torch.Tensor) -> None:
+        """Build the document cache (pooled vectors and every layer's cross K/V) for a
+        document set that many queries will be scored against; stream-ordered.  Both
+        input slots share the cache, so score_cached_stream can use either."""
+        for slot in self.slots:
+            slot["enc"][: enc_host.shape[0]].copy_(enc_host, non_blocking=True)
+            slot["doc_len"].copy_(doc_len_host, non_blocking=True)
+        self.documents()
+
+    def score_cached_stream(self, x0s, outs) -> None:
+        """Score queries against the cached documents (decode-only graphs), overlapping
+        each query's decoder-input copy with the previous query's compute.
+
+        x0s[k]: pinned host bf16 [lq][H] decoder input of query k; outs[k]: pinned
+        [4][n_docs] fp32 host tensor for (yes, no, margin, score).  Requires
+        cache_documents() (or a full forward over the same documents) and capture()."""
+        if not getattr(self, "graphs_decode", None):
+            raise RuntimeError("score_cached_stream needs capture() first")
+        comp = torch.cuda.current_stream()
+        if getattr(self, "_copy_stream", None) is None:
+            self._copy_stream = torch.cuda.Stream()
+            self._ready = [torch.cuda.Event(), torch.cuda.Event()]
+            self._free = [torch.cuda.Event(), torch.cuda.Event()]
+        cs = self._copy_stream
+        cs.wait_stream(comp)
+
+        def h2d(k):
+            i = k % 2
+            with torch.cuda.stream(cs):
+                if k >= 2:
+                    cs.wait_event(self._free[i])
+                self.slots[i]["x0"].copy_(x0s[k], non_blocking=True)
+                self._ready[i].record(cs)
+
+        if x0s:
+            h2d(0)
+        for k in range(len(x0s)):
+            if k + 1 < len(x0s):
+                h2d(k + 1)
+            i = k % 2
+            comp.wait_event(self._ready[i])
+            self.graphs_decode[i].replay()
             self._free[i].record(comp)
             outs[k].copy_(self.result, non_blocking=True)
 

@@ -573,6 +573,28 @@ def test_score_stream_matches_single_queries(kalm):
         np.testing.assert_array_equal(outs[k].numpy(), singles[k])
 
 
+def test_cached_documents_match_full_queries(kalm):
+    """Persistent-cache regime: scoring queries against documents cached once
+    (decode-only graphs) gives, bit for bit, the scores of full runs."""
+    from encoder_decoder_document_b200.scorer import DeviceWeights, FBNLScorer
+    base = synthetic.make_query("tiny")
+    qs = [synthetic.make_query("tiny", seed=s, doc_len=base.doc_len) for s in range(1, 6)]
+    sc = FBNLScorer(DeviceWeights.from_bits(base.weights), base.n_q, base.n_kv)
+    full = []
+    for q in qs:
+        sc.rerank(q.x0, base.enc, base.doc_len)   # every query against the same documents
+        full.append(sc.scores_to_host().numpy().copy())
+    sc.capture()
+    pin = lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).pin_memory()
+    sc.cache_documents(pin(base.enc), torch.from_numpy(base.doc_len).pin_memory())
+    outs = [torch.empty(4, base.n_docs, dtype=torch.float32).pin_memory() for _ in qs]
+    sc.score_cached_stream([pin(q.x0) for q in qs], outs)
+    torch.cuda.synchronize()
+    kalm.kalm_check_device_errors()
+    for k in range(len(qs)):
+        np.testing.assert_array_equal(outs[k].numpy(), full[k])
+
+
 def _item_costs(q_off, p_off, max_q, n_q, n_kv):
     """Host restatement of the work items' costs (K/V tiles + 1, 0 for an empty tile),
     in the kernel's item numbering: item w = tile t (heaviest first), KV head, document."""
