@@ -48,6 +48,8 @@ def parse():
     ap.add_argument("--cpu-sample-docs", type=int, default=0, help="documents in the oracle sample (0 = auto)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-pool-sweep", action="store_true", help="skip the pooling-only sweep at 1024/4096 docs")
+    ap.add_argument("--pool-sweep-only", action="store_true",
+                    help="run only the pooling sweep at 1024/4096 documents and print it as one JSON line")
     return ap.parse_args()
 
 
@@ -252,6 +254,11 @@ def run_reference(args):
 
 def main():
     args = parse()
+    if args.pool_sweep_only:
+        pk = peaks()
+        sweep = [dict(x, peak_gbs=pk["hbm"], frac=x["gbs"] / pk["hbm"]) for x in pool_sweep()]
+        print(json.dumps({"pool_sweep": sweep}), flush=True)
+        return
     if args.impl == "reference":
         run_reference(args)
         return

@@ -27,7 +27,7 @@ __device__ __forceinline__ int find_doc(const int64_t* __restrict__ pool_off, in
 }
 
 template <int CHUNK>
-__global__ void __launch_bounds__(256) chunk_pool_kernel(const uint4* __restrict__ enc, int64_t enc_ld_v,
+__global__ void __launch_bounds__(256, 8) chunk_pool_kernel(const uint4* __restrict__ enc, int64_t enc_ld_v,
                                                          const int64_t* __restrict__ tok_off,
                                                          const int32_t* __restrict__ len, int n_docs, int vec_per_row,
                                                          int chunk_rt, uint4* __restrict__ pooled,
