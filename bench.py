@@ -124,6 +124,38 @@ def workload(q):
     return w
 
 
+def pool_chunks(enc, len_d, chunks=(1, 2, 4, 8), reps=10):
+    """The pooling kernel alone on one query's encoder states at each chunk size
+    (Matryoshka granularities): median time of `reps` calls with the L2 flushed before
+    each (CUDA events), algorithmic bytes, GB/s."""
+    import torch
+    from encoder_decoder_document_b200 import kalm_chunk_pool, kalm_ragged_offsets
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device="cuda")
+    n, H = len_d.numel(), enc.shape[1]
+    lens = len_d.cpu().numpy().astype(np.int64)
+    out = []
+    for c in chunks:
+        nc = (lens + c - 1) // c
+        tok_off = torch.empty(n + 1, dtype=torch.int64, device="cuda")
+        pool_off = torch.empty(n + 1, dtype=torch.int64, device="cuda")
+        kalm_ragged_offsets(len_d, tok_off, pool_off, c)
+        pooled = torch.empty(int(nc.sum()), H, dtype=torch.bfloat16, device="cuda")
+        ts = []
+        for i in range(reps + 2):
+            flush.fill_(1.0)
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            kalm_chunk_pool(enc, tok_off, len_d, pooled, pool_off, pooled.shape[0], c)
+            b.record()
+            b.synchronize()
+            if i >= 2:
+                ts.append(a.elapsed_time(b))
+        us = 1e3 * statistics.median(ts)
+        byts = int((lens.sum() + nc.sum()) * H * 2 + 8 * n)
+        out.append({"chunk": c, "bytes": byts, "us": us, "gbs": byts / (us * 1e-6) / 1e9})
+    return out
+
+
 def pool_sweep(doc_counts=(1024, 4096), reps=10):
     """The pooling kernel alone at the throughput-sweep shapes with many documents
     (hidden 640, log-normal lengths, median 200, clipped to [1, 1024]): bytes moved,
@@ -437,6 +469,8 @@ def main():
         cb = None
         sweep = None if args.no_pool_sweep else [dict(x, peak_gbs=pk["hbm"], frac=x["gbs"] / pk["hbm"])
                                                  for x in pool_sweep()]
+        chunks = None if args.no_pool_sweep else [dict(x, frac=x["gbs"] / pk["hbm"])
+                                                  for x in pool_chunks(sc.enc[: int(q.doc_len.sum())], sc.doc_len)]
         if not args.no_cpu_baseline and world == 1:
             cb = cpu_baseline(q, args.cpu_sample_docs or q.n_docs)
         line = {
@@ -479,6 +513,7 @@ def main():
                                    "FBNLScorer.score_cached_stream with the query input copied in and scores read "
                                    "back"},
             "pool_sweep": sweep,
+            "pool_chunks": chunks,
             "gpu_launches": launches_per_step * args.steps,
             "clocks": clk,
             "cpu_baseline": cb,

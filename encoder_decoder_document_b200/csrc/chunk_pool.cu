@@ -128,10 +128,13 @@ extern "C" kalm_status kalm_chunk_pool(const kalm_bf16* enc, int64_t enc_ld, con
   uint32_t* err = device_error_word();
   const uint4* e = reinterpret_cast<const uint4*>(enc);
   uint4* p = reinterpret_cast<uint4*>(pooled);
+  // chunk 4 (the runtime contract) and 2 have unrolled kernels; other sizes take the generic loop
   const cudaError_t ce =
-      chunk == 4 ? launch_pdl(chunk_pool_kernel<4>, dim3((unsigned)blocks), dim3(256), 0, s, e, enc_ld / 8, tok_off,
-                              len, n_docs, vpr, chunk, p, pooled_ld / 8, pool_off, total_vec, err)
-                 : launch_pdl(chunk_pool_kernel<0>, dim3((unsigned)blocks), dim3(256), 0, s, e, enc_ld / 8, tok_off,
-                              len, n_docs, vpr, chunk, p, pooled_ld / 8, pool_off, total_vec, err);
+      chunk == 4   ? launch_pdl(chunk_pool_kernel<4>, dim3((unsigned)blocks), dim3(256), 0, s, e, enc_ld / 8, tok_off,
+                                len, n_docs, vpr, chunk, p, pooled_ld / 8, pool_off, total_vec, err)
+      : chunk == 2 ? launch_pdl(chunk_pool_kernel<2>, dim3((unsigned)blocks), dim3(256), 0, s, e, enc_ld / 8, tok_off,
+                                len, n_docs, vpr, chunk, p, pooled_ld / 8, pool_off, total_vec, err)
+                   : launch_pdl(chunk_pool_kernel<0>, dim3((unsigned)blocks), dim3(256), 0, s, e, enc_ld / 8, tok_off,
+                                len, n_docs, vpr, chunk, p, pooled_ld / 8, pool_off, total_vec, err);
   return check_cuda(ce, "launch chunk_pool_kernel");
 }

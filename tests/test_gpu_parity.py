@@ -93,8 +93,8 @@ def test_chunk_pool_edge_lengths_padded_and_strided(kalm):
     got, _ = _run_pool(kalm, oracle.f64_to_bf16_bits(enc), tok, lens, H, ld=H + 40)
     want, _ = oracle.chunk_pool(enc, tok, lens, 4)
     assert np.abs(got - want).max() <= POOL_TOL
-    # chunk 1 is the identity; a chunk of 3 exercises the generic path
-    for chunk in (1, 3):
+    # chunk 1 is the identity; 2 has its own unrolled kernel; 3 and 8 take the generic loop
+    for chunk in (1, 2, 3, 8):
         got, _ = _run_pool(kalm, oracle.f64_to_bf16_bits(enc), tok, lens, H, chunk=chunk)
         want, _ = oracle.chunk_pool(enc, tok, lens, chunk)
         assert np.abs(got - want).max() <= POOL_TOL

@@ -111,24 +111,25 @@ def test_pooled_counts_bounds():
     assert c.max() == 256
 
 
-def test_chunk_pool_vs_bruteforce_padded_mask():
-    rng = np.random.default_rng(11)
+@pytest.mark.parametrize("chunk", [1, 2, 4, 8])
+def test_chunk_pool_vs_bruteforce_padded_mask(chunk):
+    rng = np.random.default_rng(11 + chunk)
     lens = [0, 1, 2, 3, 4, 5, 8, 9, 13]
     H, Lmax = 3, 16
     padded = rng.standard_normal((len(lens), Lmax, H))
     # packed copy of the valid rows with a row offset per document
     tok_off = np.concatenate([[0], np.cumsum(lens)])
     packed = np.concatenate([padded[d, :lens[d]] for d in range(len(lens))])
-    pooled, off = O.chunk_pool(packed, tok_off, lens, 4, round_out=False)
+    pooled, off = O.chunk_pool(packed, tok_off, lens, chunk, round_out=False)
     for d, n in enumerate(lens):
         mask = [1] * n + [0] * (Lmax - n)
-        want = brute.pool_padded(padded[d].tolist(), mask, 4)
+        want = brute.pool_padded(padded[d].tolist(), mask, chunk)
         got = pooled[off[d]:off[d + 1]]
         assert len(want) == got.shape[0]
         if want:
             np.testing.assert_allclose(got, np.array(want), rtol=0, atol=1e-12)
     # the padded layout (row stride Lmax) gives the same result
-    pooled2, _ = O.chunk_pool(padded.reshape(-1, H), np.arange(len(lens)) * Lmax, lens, 4,
+    pooled2, _ = O.chunk_pool(padded.reshape(-1, H), np.arange(len(lens)) * Lmax, lens, chunk,
                               round_out=False)
     np.testing.assert_array_equal(pooled2, pooled)
 
