@@ -21,6 +21,11 @@ tensors.  Sources, by page title and section:
   score = sigmoid(yes_logit - no_logit).
 * "KaLM-Reranker-V1-Small-Q4_K_M-GGUF", "Score a pair": margin = yes - no,
   score = sigmoid(margin), larger margins rank first.
+* "KaLM-Reranker-V1-Nano - MLX (Apple Silicon)", "Derivation": rotary
+  position parameters and inverse-frequency tables come from the model
+  config; the rotation itself (pairing element i with i + D/2, angle
+  position * theta^(-2i/D)) is the standard form, a reading the pages leave
+  open, as is which segments are rotated (here: the decoder's self Q and K).
 
 Readings taken where the pages are silent are listed with each function.
 Parity is pinned by ``tests/test_oracle_pins.py`` (brute force, closed forms,
@@ -28,6 +33,8 @@ library special cases, invariants); nothing here is "parity unpinned".
 """
 from .kalm_oracle import (  # noqa: F401
     bf16_round,
+    rope_inv_freq,
+    apply_rope,
     bf16_bits_to_f64,
     f64_to_bf16_bits,
     pooled_counts,

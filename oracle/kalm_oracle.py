@@ -235,19 +235,52 @@ def yes_no_score(x_last: np.ndarray, w_yes: np.ndarray, w_no: np.ndarray):
 
 
 # ----------------------------------------------------------------------------
+# Rotary position embedding of the decoder's self Q and K
+# ----------------------------------------------------------------------------
+def rope_inv_freq(head_dim: int, theta: float) -> np.ndarray:
+    """Inverse frequencies theta^(-2i/head_dim), i = 0 .. head_dim/2 - 1: the table a
+    model config's rope parameters define ("KaLM-Reranker-V1-Nano - MLX",
+    "Derivation": the inverse-frequency tables are computed from the config)."""
+    i = np.arange(head_dim // 2, dtype=np.float64)
+    return float(theta) ** (-2.0 * i / head_dim)
+
+
+def apply_rope(x: np.ndarray, positions: Sequence[int], theta: float, round_out: bool = True) -> np.ndarray:
+    """Rotate each head vector of row r by its decoder position ``positions[r]``.
+
+    x: [rows][heads][D].  Element i (< D/2) pairs with element i + D/2 and the pair
+    (a, b) turns by the angle pos * inv_freq[i]: (a cos - b sin, b cos + a sin).
+    Rounded to bf16 (the rotated Q and K are stored)."""
+    D = x.shape[-1]
+    h = D // 2
+    ang = np.asarray(positions, np.float64)[:, None] * rope_inv_freq(D, theta)[None, :]
+    c = np.cos(ang)[:, None, :]
+    s = np.sin(ang)[:, None, :]
+    a, b = x[..., :h], x[..., h:]
+    out = np.concatenate([a * c - b * s, b * c + a * s], axis=-1)
+    return bf16_round(out) if round_out else out
+
+
+# ----------------------------------------------------------------------------
 # End to end (oracle mode (ii): the oracle chains its own rounded outputs)
 # ----------------------------------------------------------------------------
 def decoder_layer(X: np.ndarray, pooled: np.ndarray, w_qkv_l, w_o_l, w_kv_l, n_q: int, n_kv: int,
-                  head_dim: int, scale: float, trace: Optional[dict] = None) -> np.ndarray:
+                  head_dim: int, scale: float, trace: Optional[dict] = None,
+                  rope_theta: Optional[float] = None) -> np.ndarray:
     """One layer of the synthetic attention-only decoder for one document.
 
     Reading of the synthetic stack (the pages name no MLP/norm on this path):
     ``X <- X + MergedAttn(X Wq, X Wk, X Wv, P Wk_c, P Wv_c) Wo`` with P the
-    document's pooled vectors.  Returns the new X (bf16-rounded)."""
+    document's pooled vectors.  With ``rope_theta`` the self Q and K are rotated
+    by decoder position 0 .. Lq-1 before the attention (the cross keys have no
+    decoder position and are not rotated).  Returns the new X (bf16-rounded)."""
     D = head_dim
     Lq = X.shape[0]
     kv = linear(pooled, w_kv_l).reshape(-1, 2, n_kv, D)
     qkv = linear(X, w_qkv_l)
+    if rope_theta is not None:
+        qk = apply_rope(qkv[:, :(n_q + n_kv) * D].reshape(Lq, n_q + n_kv, D), np.arange(Lq), rope_theta)
+        qkv = np.concatenate([qk.reshape(Lq, -1), qkv[:, (n_q + n_kv) * D:]], axis=1)
     q = qkv[:, : n_q * D].reshape(Lq, n_q, D)
     ks = qkv[:, n_q * D:(n_q + n_kv) * D].reshape(Lq, n_kv, D)
     vs = qkv[:, (n_q + n_kv) * D:].reshape(Lq, n_kv, D)
@@ -261,7 +294,7 @@ def decoder_layer(X: np.ndarray, pooled: np.ndarray, w_qkv_l, w_o_l, w_kv_l, n_q
 def forward_doc(enc_doc: np.ndarray, x0: np.ndarray, w_qkv, w_o, w_kv_cross,
                 w_yes, w_no, n_q: int, n_kv: int, head_dim: int, scale: float,
                 chunk: int = 4, layers: Optional[Sequence[int]] = None,
-                trace: Optional[dict] = None):
+                trace: Optional[dict] = None, rope_theta: Optional[float] = None):
     """Score one document with the synthetic attention-only decoder stack
     (``decoder_layer`` per layer, X0 = the query's decoder input).
     Returns ``(yes, no, margin, score)`` as floats.  ``trace`` (a dict), if
@@ -271,7 +304,8 @@ def forward_doc(enc_doc: np.ndarray, x0: np.ndarray, w_qkv, w_o, w_kv_cross,
     X = np.asarray(x0, np.float64)
     lay = range(len(w_qkv)) if layers is None else layers
     for l in lay:
-        X = decoder_layer(X, pooled, w_qkv[l], w_o[l], w_kv_cross[l], n_q, n_kv, head_dim, scale, trace)
+        X = decoder_layer(X, pooled, w_qkv[l], w_o[l], w_kv_cross[l], n_q, n_kv, head_dim, scale, trace,
+                          rope_theta)
     if trace is not None:
         trace["pooled"] = pooled
         trace["x_final"] = X
@@ -280,7 +314,7 @@ def forward_doc(enc_doc: np.ndarray, x0: np.ndarray, w_qkv, w_o, w_kv_cross,
 
 
 def forward_query(query, docs: Optional[Sequence[int]] = None, chunk: int = 4,
-                  scale: Optional[float] = None):
+                  scale: Optional[float] = None, rope_theta: Optional[float] = None):
     """End-to-end oracle scores for documents ``docs`` (default: all) of a
     ``synthetic.Query``.  Returns fp64 arrays (yes, no, margin, score)."""
     D = query.head_dim
@@ -298,6 +332,6 @@ def forward_query(query, docs: Optional[Sequence[int]] = None, chunk: int = 4,
         a, b = int(query.tok_off[d]), int(query.tok_off[d + 1])
         enc = bf16_bits_to_f64(query.enc[a:b])
         res.append(forward_doc(enc, x0, w_qkv, w_o, w_kv, w_yes, w_no,
-                               query.n_q, query.n_kv, D, scale, chunk))
+                               query.n_q, query.n_kv, D, scale, chunk, rope_theta=rope_theta))
     r = np.array(res, dtype=np.float64).reshape(-1, 4)
     return r[:, 0], r[:, 1], r[:, 2], r[:, 3]

@@ -396,3 +396,79 @@ def test_forward_query_doc_independence():
     for d in range(qy.n_docs):
         s = O.forward_query(qy, docs=[d])[3]
         assert s[0] == all_scores[d]
+
+
+# ---------------------------------------------------------------------------
+# Rotary position embedding of the decoder's self Q and K
+# ---------------------------------------------------------------------------
+def test_rope_matches_complex_rotation():
+    """Each pair (x[i], x[i + D/2]) read as the complex number x[i] + j x[i + D/2] is
+    multiplied by exp(j * pos * theta^(-2i/D)) (numpy complex arithmetic)."""
+    rng = np.random.default_rng(21)
+    D, theta = 16, 10000.0
+    x = rng.standard_normal((5, 3, D))
+    pos = [0, 1, 7, 100, 511]
+    got = O.apply_rope(x, pos, theta, round_out=False)
+    z = x[..., : D // 2] + 1j * x[..., D // 2:]
+    freq = np.array([theta ** (-(2 * i) / D) for i in range(D // 2)])
+    rot = np.exp(1j * np.outer(pos, freq))[:, None, :]
+    want = z * rot
+    np.testing.assert_allclose(got[..., : D // 2], want.real, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(got[..., D // 2:], want.imag, rtol=0, atol=1e-12)
+
+
+def test_rope_special_cases():
+    rng = np.random.default_rng(22)
+    x = rng.standard_normal((4, 2, 8))
+    # position 0 is the identity; the rotation keeps every pair's length
+    np.testing.assert_array_equal(O.apply_rope(x, [0] * 4, 500.0, round_out=False), x)
+    y = O.apply_rope(x, [3, 9, 27, 81], 500.0, round_out=False)
+    np.testing.assert_allclose(y[..., :4] ** 2 + y[..., 4:] ** 2, x[..., :4] ** 2 + x[..., 4:] ** 2, rtol=1e-13)
+    # D = 2: one pair at frequency 1, so position p rotates (1, 0) to (cos p, sin p)
+    e = np.array([[[1.0, 0.0]]])
+    np.testing.assert_allclose(O.apply_rope(e, [2], 1e4, round_out=False)[0, 0], [math.cos(2), math.sin(2)],
+                               atol=1e-15)
+    # composing two shifts is one shift by the sum (rotation angles add)
+    a = O.apply_rope(O.apply_rope(x, [5] * 4, 500.0, round_out=False), [6] * 4, 500.0, round_out=False)
+    np.testing.assert_allclose(a, O.apply_rope(x, [11] * 4, 500.0, round_out=False), atol=1e-12)
+
+
+def test_rope_scores_depend_on_relative_position_only():
+    """q_m . k_n after rotation depends on m - n only (the point of the embedding)."""
+    rng = np.random.default_rng(23)
+    D = 32
+    q = rng.standard_normal((1, 1, D))
+    k = rng.standard_normal((1, 1, D))
+    dots = []
+    for m, n in [(10, 3), (17, 10), (507, 500)]:
+        qm = O.apply_rope(q, [m], 1e4, round_out=False)[0, 0]
+        kn = O.apply_rope(k, [n], 1e4, round_out=False)[0, 0]
+        dots.append(float(qm @ kn))
+    np.testing.assert_allclose(dots, dots[0], rtol=0, atol=1e-11)
+    # and a different offset gives a different score
+    q0 = O.apply_rope(q, [4], 1e4, round_out=False)[0, 0]
+    k0 = O.apply_rope(k, [0], 1e4, round_out=False)[0, 0]
+    assert abs(float(q0 @ k0) - dots[0]) > 1e-6
+
+
+def test_decoder_layer_rope_rotates_self_qk_only():
+    """With RoPE the layer equals the plain layer run on rotated Q/K weights' outputs:
+    checked by rotating the oracle's own projections and comparing attention inputs."""
+    import synthetic
+    qy = synthetic.make_query("tiny", layers=1, hidden=64, n_docs=1)
+    w = qy.weights
+    enc = O.bf16_bits_to_f64(qy.enc)
+    x0 = O.bf16_bits_to_f64(qy.x0)
+    pooled, _ = O.chunk_pool(enc, [0], [enc.shape[0]], 4)
+    args = (O.bf16_bits_to_f64(w.w_qkv[0]), O.bf16_bits_to_f64(w.w_o[0]), O.bf16_bits_to_f64(w.w_kv_cross[0]),
+            qy.n_q, qy.n_kv, qy.head_dim, 1 / 16)
+    tr = {}
+    O.decoder_layer(x0, pooled, *args, trace=tr, rope_theta=1e4)
+    tr0 = {}
+    O.decoder_layer(x0, pooled, *args, trace=tr0)
+    D, nq, nkv, Lq = qy.head_dim, qy.n_q, qy.n_kv, x0.shape[0]
+    qkv_rot, qkv = tr["layers"][0]["qkv"], tr0["layers"][0]["qkv"]
+    want = O.apply_rope(qkv[:, :(nq + nkv) * D].reshape(Lq, nq + nkv, D), np.arange(Lq), 1e4).reshape(Lq, -1)
+    np.testing.assert_array_equal(qkv_rot[:, :(nq + nkv) * D], want)
+    np.testing.assert_array_equal(qkv_rot[:, (nq + nkv) * D:], qkv[:, (nq + nkv) * D:])   # V untouched
+    np.testing.assert_array_equal(tr["layers"][0]["kv_cross"], tr0["layers"][0]["kv_cross"])  # cross untouched
