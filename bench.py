@@ -48,6 +48,8 @@ def parse():
     ap.add_argument("--cpu-sample-docs", type=int, default=0, help="documents in the oracle sample (0 = auto)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-pool-sweep", action="store_true", help="skip the pooling-only sweep at 1024/4096 docs")
+    ap.add_argument("--rope-theta", type=float, default=None,
+                    help="rotate the decoder's self Q/K with this rotary base in every layer (default: off)")
     ap.add_argument("--pool-sweep-only", action="store_true",
                     help="run only the pooling sweep at 1024/4096 documents and print it as one JSON line")
     return ap.parse_args()
@@ -154,6 +156,30 @@ def pool_chunks(enc, len_d, chunks=(1, 2, 4, 8), reps=10):
         byts = int((lens.sum() + nc.sum()) * H * 2 + 8 * n)
         out.append({"chunk": c, "bytes": byts, "us": us, "gbs": byts / (us * 1e-6) / 1e9})
     return out
+
+
+def rope_alone(sc, theta=1e4, reps=10):
+    """The rotary-embedding kernel alone on one layer's Q|K|V buffer (all documents'
+    rows, Q and self-K heads): median time (L2 flushed before each call), bytes
+    read + written, GB/s."""
+    import torch
+    from encoder_decoder_document_b200 import kalm_rope
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device="cuda")
+    heads = sc.n_q + sc.n_kv
+    ts = []
+    for i in range(reps + 2):
+        flush.fill_(1.0)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        kalm_rope(sc.qkv, sc.q_off, heads, theta, sc.D)
+        b.record()
+        b.synchronize()
+        if i >= 2:
+            ts.append(a.elapsed_time(b))
+    us = 1e3 * statistics.median(ts)
+    byts = 2 * sc.qkv.shape[0] * heads * sc.D * 2
+    return {"rows": sc.qkv.shape[0], "heads": heads, "theta": theta, "bytes": byts, "us": us,
+            "gbs": byts / (us * 1e-6) / 1e9}
 
 
 def pool_sweep(doc_counts=(1024, 4096), reps=10):
@@ -319,7 +345,7 @@ def main():
     q = synthetic.make_query(args.config, seed=base if rank == 0 else base + 1000 * rank)
     w = workload(q)
     pk = peaks()
-    sc = FBNLScorer(DeviceWeights.from_bits(q.weights), q.n_q, q.n_kv)
+    sc = FBNLScorer(DeviceWeights.from_bits(q.weights), q.n_q, q.n_kv, rope_theta=args.rope_theta)
     total_pooled = int(((q.doc_len.astype(np.int64) + 3) // 4).sum())
     sc.prepare(q.n_docs, int(q.doc_len.sum()), total_pooled, q.lq)
     enc_h = torch.from_numpy(q.enc.view(np.int16)).view(torch.bfloat16).pin_memory()
@@ -471,6 +497,9 @@ def main():
                                                  for x in pool_sweep()]
         chunks = None if args.no_pool_sweep else [dict(x, frac=x["gbs"] / pk["hbm"])
                                                   for x in pool_chunks(sc.enc[: int(q.doc_len.sum())], sc.doc_len)]
+        rope = None if args.no_pool_sweep else dict(rope_alone(sc), frac=None)
+        if rope is not None:
+            rope["frac"] = rope["gbs"] / pk["hbm"]
         if not args.no_cpu_baseline and world == 1:
             cb = cpu_baseline(q, args.cpu_sample_docs or q.n_docs)
         line = {
@@ -485,7 +514,8 @@ def main():
                        "graph": "one CUDA graph per step (launches overlap through programmatic dependent "
                                 "launch); per-kernel times come from a second graph with a timing event "
                                 "after every launch, replayed once after each timed step",
-                       "instrumented_ms_per_step": sum(sum(v) for v in per_kernel.values()) / args.steps},
+                       "instrumented_ms_per_step": sum(sum(v) for v in per_kernel.values()) / args.steps,
+                       "rope_theta": args.rope_theta},
             "roofline": roofline,
             "algorithmic_flops_per_step": step_flops,
             "pool": {"bytes": w["pool_bytes"], "avg_us": kern["chunk_pool"]["avg_us"], "achieved_gbs": pool_gbs,
@@ -514,6 +544,7 @@ def main():
                                    "back"},
             "pool_sweep": sweep,
             "pool_chunks": chunks,
+            "rope": rope,
             "gpu_launches": launches_per_step * args.steps,
             "clocks": clk,
             "cpu_baseline": cb,

@@ -18,7 +18,7 @@ __all__ = [
     "KalmError", "load", "library_path", "kalm_version", "kalm_device_check", "kalm_check_device_errors",
     "kalm_ragged_offsets", "kalm_chunk_pool", "kalm_linear", "kalm_cross_kv_proj", "kalm_merged_attention",
     "kalm_yes_no_score", "kalm_broadcast_rows", "kalm_selftest_wait_timeout", "kalm_attention_items",
-    "kalm_attention_schedule",
+    "kalm_attention_schedule", "kalm_rope",
 ]
 
 HEAD_DIM = 256
@@ -143,6 +143,14 @@ def kalm_yes_no_score(hidden: torch.Tensor, q_off: torch.Tensor, w_yes: torch.Te
 def kalm_broadcast_rows(src: torch.Tensor, q_off: torch.Tensor, dst: torch.Tensor, stream=None) -> None:
     call("kalm_broadcast_rows", _p(src, torch.bfloat16), _ld(src), src.shape[0], src.shape[1],
          _p(q_off, torch.int64), q_off.numel() - 1, _p(dst, torch.bfloat16), _ld(dst), _stream(stream))
+
+
+def kalm_rope(x: torch.Tensor, q_off: torch.Tensor, n_heads: int, theta: float, head_dim: int = HEAD_DIM,
+              stream=None) -> None:
+    """Rotate the first n_heads head vectors of every row of x in place by the row's
+    decoder position (row - q_off[d] for the document d owning the row)."""
+    call("kalm_rope", _p(x, torch.bfloat16), _ld(x), x.shape[0], n_heads, head_dim, _p(q_off, torch.int64),
+         q_off.numel() - 1, float(theta), _stream(stream))
 
 
 def kalm_selftest_wait_timeout(wait_ns: int, stream=None) -> None:

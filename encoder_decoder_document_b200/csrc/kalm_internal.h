@@ -20,6 +20,9 @@ kalm_status ensure_device(int* device_out);
 // Device address of the current device's error word (valid after ensure_device).
 uint32_t* device_error_word();
 
+// Streaming multiprocessors of the current device (cached at set-up).
+int num_sms();
+
 // Map a CUDA runtime error to KALM_ERR_CUDA with its message; KALM_OK if none.
 kalm_status check_cuda(cudaError_t e, const char* what);
 

@@ -19,6 +19,7 @@ constexpr uint32_t kSiteAttention = 3u << 8;
 constexpr uint32_t kSiteReadout = 4u << 8;
 constexpr uint32_t kSiteOffsets = 5u << 8;
 constexpr uint32_t kSiteSelftest = 6u << 8;
+constexpr uint32_t kSiteRope = 7u << 8;
 
 // Default bound of one wait: 1 s.  No wait of a healthy launch comes close.
 constexpr uint64_t kWaitNs = 1000000000ull;

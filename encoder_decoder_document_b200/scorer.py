@@ -26,7 +26,7 @@ import torch
 
 from . import (kalm_broadcast_rows, kalm_chunk_pool, kalm_cross_kv_proj, kalm_device_check, kalm_linear,
                kalm_merged_attention, kalm_ragged_offsets, kalm_yes_no_score, kalm_attention_items,
-               kalm_attention_schedule)
+               kalm_attention_schedule, kalm_rope)
 
 HEAD_DIM = 256
 
@@ -61,7 +61,7 @@ class FBNLScorer:
     (the readout reads nothing else)."""
 
     def __init__(self, weights: DeviceWeights, n_q: int, n_kv: int, chunk: int = 4, head_dim: int = HEAD_DIM,
-                 prune: bool = True):
+                 prune: bool = True, rope_theta: Optional[float] = None):
         kalm_device_check()
         self.w = weights
         self.L, qkv_rows, self.H = weights.w_qkv.shape
@@ -69,6 +69,7 @@ class FBNLScorer:
         assert qkv_rows == (n_q + 2 * n_kv) * head_dim
         self.scale = head_dim ** -0.5
         self.prune = prune
+        self.rope_theta = rope_theta  # rotary base for the decoder's self Q/K, or None (no rotation)
         self._shape = None
         self.graph: Optional[torch.cuda.CUDAGraph] = None
         self.graphs = None
@@ -99,6 +100,7 @@ class FBNLScorer:
         self.pool_off = torch.empty(n_docs + 1, dtype=torch.int64, **kw)
         self.q_off = torch.empty(n_docs + 1, dtype=torch.int64, **kw)
         self.zero_off = torch.zeros(n_docs, dtype=torch.int64, **kw)
+        self.one_doc_off = torch.tensor([0, lq], dtype=torch.int64, **kw)  # the query's common rows
         self.pooled = torch.empty(max(total_pooled, 1), H, dtype=torch.bfloat16, **kw)
         self.kv_cross = torch.empty(max(total_pooled, 1), L * 2 * self.n_kv * D, dtype=torch.bfloat16, **kw)
         self.qkv = torch.empty(rows, (self.n_q + 2 * self.n_kv) * D, dtype=torch.bfloat16, **kw)
@@ -152,9 +154,15 @@ class FBNLScorer:
         D, nq, nkv = self.D, self.n_q, self.n_kv
         return (self.qkv[:, : nq * D], self.qkv[:, nq * D:(nq + nkv) * D], self.qkv[:, (nq + nkv) * D:])
 
+    def rope(self, qkv: torch.Tensor, q_off: torch.Tensor) -> None:
+        if self.rope_theta is not None:
+            kalm_rope(qkv, q_off, self.n_q + self.n_kv, self.rope_theta, self.D)
+            self._mark("rope")
+
     def layer_qkv(self, l: int) -> None:
         kalm_linear(self.x, self.w.w_qkv[l], self.qkv)
         self._mark("qkv_proj")
+        self.rope(self.qkv, self.q_off)
 
     def layer_attention(self, l: int) -> None:
         q, ks, vs = self.qkv_views()
@@ -181,6 +189,7 @@ class FBNLScorer:
             # every document's decoder input is the query's common input: one Q|K|V for all
             kalm_linear(self.x0, self.w.w_qkv[l], self.qkv[:Lq])
             self._mark("qkv_proj")
+            self.rope(self.qkv[:Lq], self.one_doc_off)
             q, ks, vs = (t[:Lq] for t in self.qkv_views())
             in_off = self.zero_off
         else:

@@ -252,6 +252,29 @@ kalm_status kalm_broadcast_rows(const kalm_bf16* src, int64_t ld_src, int32_t ro
                                 int32_t width, const int64_t* q_off, int32_t n_docs,
                                 kalm_bf16* dst, int64_t ld_dst, kalm_stream_t stream);
 
+/* Rotary position embedding of the decoder's self Q and K, in place ("next"
+ * step after the four above).  "KaLM-Reranker-V1-Nano - MLX (Apple Silicon)",
+ * "Derivation": the rotary parameters and inverse-frequency tables are read
+ * from the model config.  Reading taken (the pages give neither the pairing
+ * nor which segments are rotated): element i < head_dim/2 of each head vector
+ * pairs with element i + head_dim/2 and (a, b) turns by the angle
+ * pos * theta^(-2i/head_dim): (a cos - b sin, b cos + a sin); the decoder's
+ * self Q and K are rotated, the cross keys (pooled passage vectors, no decoder
+ * position) are not.
+ *
+ * x       [rows][ldx] bf16, n_heads head vectors of head_dim elements at the
+ *         start of each row (Q heads then self-K heads of the fused Q|K|V
+ *         layout: one call covers both); rotated in place, one bf16 rounding.
+ * q_off   int64[n_docs+1]: row r belongs to the document d with
+ *         q_off[d] <= r < q_off[d+1] and sits at position r - q_off[d]
+ *         (< KALM_MAX_QUERY_TOKENS; rows = q_off[n_docs]).
+ * theta   rotary base (> 1).
+ * Requirements: head_dim % 16 == 0, ldx % 8 == 0, x 16-byte aligned.  A row
+ * whose position falls outside [0, KALM_MAX_QUERY_TOKENS) is left unchanged and
+ * flagged in the device error word. */
+kalm_status kalm_rope(kalm_bf16* x, int64_t ldx, int64_t rows, int32_t n_heads, int32_t head_dim,
+                      const int64_t* q_off, int32_t n_docs, float theta, kalm_stream_t stream);
+
 /* Failure-detection self-test: one CTA waits on a shared-memory barrier that
  * nothing completes, with a bound of `wait_ns` nanoseconds; on expiry it
  * records a timeout in the device error word and returns.  Lets tests check

@@ -667,3 +667,56 @@ def test_attention_order_out_of_range_is_flagged(kalm):
     assert e.value.name == "KALM_ERR_DEVICE_ARG"
     with pytest.raises(KalmError):
         kalm.kalm_attention_schedule(i64(a["q_off"]), i64(a["p_off"]), 64, 4, 1, order[:1])  # too short
+
+
+# ---------------------------------------------------------------------------
+# rotary position embedding of the decoder's self Q/K
+# ---------------------------------------------------------------------------
+def _bf16_ulp(v):
+    """Spacing of bf16 values at |v| (2^-133 below the normal range)."""
+    a = np.maximum(np.abs(v), 2.0 ** -126)
+    return 2.0 ** (np.floor(np.log2(a)) - 7)
+
+
+@pytest.mark.parametrize("theta", [1e4, 1e6])
+def test_rope_parity(kalm, theta):
+    """GPU rotation vs the oracle on a fused Q|K|V buffer with ragged documents:
+    one bf16 step plus the fp32 angle error; V columns and padding untouched."""
+    rng = np.random.default_rng(81)
+    D, n_q, n_kv = 256, 4, 1
+    lq = np.array([1, 2, 31, 129, 512, 64], np.int64)
+    q_off = np.concatenate([[0], np.cumsum(lq)])
+    R, W = int(q_off[-1]), (n_q + 2 * n_kv) * D
+    x = rand_bf16(rng, (R, W + 8))
+    dev = f64_to_dev(x)
+    kalm.kalm_rope(dev[:, :W], i64(q_off), n_q + n_kv, theta)
+    kalm.kalm_check_device_errors()
+    got = from_dev(dev)
+    pos = np.concatenate([np.arange(n) for n in lq])
+    qk = x[:, :(n_q + n_kv) * D].reshape(R, n_q + n_kv, D)
+    want = oracle.apply_rope(qk, pos, theta).reshape(R, -1)
+    a, b = qk[..., : D // 2], qk[..., D // 2:]
+    mag = np.concatenate([np.abs(a) + np.abs(b)] * 2, axis=-1).reshape(R, -1)
+    bound = _bf16_ulp(want) + 1e-4 * mag   # fp32 angle (pos * freq) error ~3e-5 rad at pos 511
+    assert (np.abs(got[:, :(n_q + n_kv) * D] - want) <= bound).all()
+    np.testing.assert_array_equal(got[:, (n_q + n_kv) * D:], x[:, (n_q + n_kv) * D:])
+    # position 0 rows are returned bit for bit
+    np.testing.assert_array_equal(got[q_off[:-1]], x[q_off[:-1]])
+
+
+def test_end_to_end_tiny_with_rope(kalm):
+    """The stack with rotated self Q/K matches the oracle's, pruned or not."""
+    from encoder_decoder_document_b200.scorer import DeviceWeights, FBNLScorer
+    q = synthetic.make_query("tiny", layers=3)
+    res = []
+    for prune in (False, True):
+        sc = FBNLScorer(DeviceWeights.from_bits(q.weights), q.n_q, q.n_kv, prune=prune, rope_theta=1e4)
+        sc.rerank(q.x0, q.enc, q.doc_len)
+        kalm.kalm_check_device_errors()
+        res.append(sc.scores_to_host().numpy())
+    assert np.abs(res[0] - res[1]).max() <= 1e-6
+    y, n, m, s = oracle.forward_query(q, rope_theta=1e4)
+    _check_scores(res[1][3], s, m)
+    # and the rotation matters: without it the scores differ
+    y0, n0, m0, s0 = oracle.forward_query(q)
+    assert np.abs(m0 - m).max() > 1e-3
