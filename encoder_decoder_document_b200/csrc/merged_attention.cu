@@ -33,6 +33,8 @@
 //     of the current item is done) and its first S product overlap the current
 //     item's last softmax, P V and O write-out.
 //   * Every role loads the next item's offsets while it works on the current one.
+//   * Epilogue: each warp stages its 32 rows x 64 columns of O / l as bf16 in the idle
+//     P buffers and copies them out row-major, so every store writes whole lines.
 //   * Warp roles: warps 0-7 softmax + epilogue, warp 8 TMA producer of Q and K,
 //     warp 10 TMA producer of V, warp 9 tensor-memory allocation and MMA issue.
 #include <cmath>
@@ -142,8 +144,7 @@ __device__ __forceinline__ Item load_item(const AttnParams& p, int w) {
 __global__ void __launch_bounds__(kThreads, 1)
     merged_attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_ks,
                             const __grid_constant__ CUtensorMap tm_vs, const __grid_constant__ CUtensorMap tm_kc,
-                            const __grid_constant__ CUtensorMap tm_vc, const __grid_constant__ CUtensorMap tm_o,
-                            const AttnParams p) {
+                            const __grid_constant__ CUtensorMap tm_vc, const AttnParams p) {
   pdl_launch_dependents();
   pdl_wait_predecessor();  // q/K/V come from the previous kernel; offsets are read by every role
 
@@ -442,14 +443,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool valid = pos < it.pos1;
       const int head = it.g * p.G + hh;
       // This warp's 32 rows go out through its own 4 KB staging tile in the (now idle)
-      // P buffers, one 64-column slab at a time, with a 3-D TMA box (64 columns x
-      // heads x positions) -- unless some of its rows lie past the document's end.
+      // P buffers, one 64-column slab at a time: each lane writes its row (swizzled,
+      // so the writes are bank-conflict free), then reads it back row-major, 8 lanes
+      // per 128-byte row, so every global store instruction writes 4 whole lines.
       const int r0 = quarter * 32;
-      const int rows_g = p.G < 32 ? p.G : 32;        // heads per box
-      const int pos_a = it.pos0 + r0 / p.G;
-      const bool warp_full = pos_a + (32 / rows_g) <= it.pos1;
       uint8_t* stage = sP + warp * 4096;
-      __nv_bfloat16* orow = p.out + (it.q0 + pos) * p.ldo + static_cast<int64_t>(head) * kD;
 #pragma unroll 1
       for (int sl = 2 * half; sl < 2 * half + 2; ++sl) {
         uint4 v[8];
@@ -466,23 +464,24 @@ __global__ void __launch_bounds__(kThreads, 1)
             v[c2 * 4 + q].w = pack_bf16x2(__uint_as_float(o[8 * q + 6]) * inv_l, __uint_as_float(o[8 * q + 7]) * inv_l);
           }
         }
-        if (warp_full) {
-          uint8_t* row = stage + lane * 128;
+        uint8_t* row = stage + lane * 128;
 #pragma unroll
-          for (int u = 0; u < 8; ++u) *reinterpret_cast<uint4*>(row + ((u ^ (lane & 7)) << 4)) = v[u];
-          fence_proxy_async_smem();
-          __syncwarp();
-          if (lane == 0) {
-            tma_store_3d(&tm_o, stage, sl * 64, it.g * p.G + (r0 % p.G), static_cast<int32_t>(it.q0 + pos_a));
-            bulk_commit_group();
-            bulk_wait_group_read<0>();  // staging tile read before it is refilled
+        for (int u = 0; u < 8; ++u) *reinterpret_cast<uint4*>(row + ((u ^ (lane & 7)) << 4)) = v[u];
+        __syncwarp();
+        const int cu = lane & 7;  // 16-byte unit of the row this lane copies
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          const int rr = (lane >> 3) + 4 * k;  // row of the warp's 32
+          const uint4 val = *reinterpret_cast<const uint4*>(stage + rr * 128 + ((cu ^ (rr & 7)) << 4));
+          const int prow = r0 + rr;            // packed row = position x head
+          const int ppos = it.pos0 + prow / p.G;
+          if (ppos < it.pos1) {
+            __nv_bfloat16* dst = p.out + (it.q0 + ppos) * p.ldo +
+                                 static_cast<int64_t>(it.g * p.G + prow % p.G) * kD + sl * 64 + cu * 8;
+            *reinterpret_cast<uint4*>(dst) = val;
           }
-          __syncwarp();
-        } else if (valid) {
-          uint4* dst = reinterpret_cast<uint4*>(orow + sl * 64);
-#pragma unroll
-          for (int u = 0; u < 8; ++u) dst[u] = v[u];
         }
+        __syncwarp();  // staging tile read before it is refilled
       }
       tc_fence_before();
       // O read out and the staging tiles free: the next item may overwrite O and P
@@ -494,7 +493,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       J += it.nt;
       ++n_it;
     }
-    if (lane == 0) bulk_wait_group<0>();
     if (!ok) {
       if (lane == 0) record_error(p.err, kErrTimeout | kSiteAttention);
       *abort_flag = 1;
@@ -585,20 +583,14 @@ extern "C" kalm_status kalm_merged_attention(const kalm_bf16* q, int64_t ldq, co
   if (total_q > INT32_MAX - 1024 || total_pool > INT32_MAX - 1024 || total_in > INT32_MAX - 1024)
     return fail(KALM_ERR_INVALID_ARG, "kalm_merged_attention: too many rows");
 
-  // Q and O: 4-D views (64 columns, head, row, 64-column slab) so one box moves a whole
+  // Q: a 4-D view (64 columns, head, row, 64-column slab) so one box moves a whole
   // 128-row x 256-column tile in the slab-major order the tensor-core descriptors read.
-  CUtensorMap tq, tks, tvs, tkc, tvc, to;
+  CUtensorMap tq, tks, tvs, tkc, tvc;
   {
     const uint64_t dims[4] = {64, static_cast<uint64_t>(n_q), static_cast<uint64_t>(total_in), 4};
     const uint64_t strides[3] = {kD * 2, static_cast<uint64_t>(ldq) * 2, 128};
     const uint32_t box[4] = {64, static_cast<uint32_t>(G), static_cast<uint32_t>(kBM / G), 4};
     if ((st = make_tmap_bf16(&tq, q, 4, dims, strides, box)) != KALM_OK) return st;
-    // O: 3-D view (256 columns, head, row); a box is one warp's 32 packed rows x 64 columns
-    const int gb = G < 32 ? G : 32;
-    const uint64_t odims[3] = {kD, static_cast<uint64_t>(n_q), static_cast<uint64_t>(total_q)};
-    const uint64_t ostrides[2] = {kD * 2, static_cast<uint64_t>(ldo) * 2};
-    const uint32_t obox[3] = {64, static_cast<uint32_t>(gb), static_cast<uint32_t>(32 / gb)};
-    if ((st = make_tmap_bf16(&to, out, 3, odims, ostrides, obox)) != KALM_OK) return st;
   }
   // K and V: 3-D views (64 columns, row, 64-column slab over all KV heads); a box is
   // one 64-key x 256-column tile of one KV head.
@@ -645,7 +637,7 @@ extern "C" kalm_status kalm_merged_attention(const kalm_bf16* q, int64_t ldq, co
   if (sms <= 0) sms = 148;
   const int64_t grid = items < sms ? items : sms;  // persistent: one CTA per SM
   return check_cuda(launch_pdl(merged_attention_kernel, dim3(static_cast<unsigned>(grid)), dim3(kThreads), kSmem,
-                                static_cast<cudaStream_t>(stream), tq, tks, tvs, tkc, tvc, to, prm),
+                                static_cast<cudaStream_t>(stream), tq, tks, tvs, tkc, tvc, prm),
                     "launch merged_attention_kernel");
 }
 
