@@ -17,21 +17,23 @@
 //     loop order; nothing is materialised in memory.
 //   * S = Q K^T and O += P V run on the tensor cores (tcgen05.mma, fp32
 //     accumulators in tensor memory: O = 256 columns, S double-buffered 2 x 64).
-//   * Softmax: two threads per row (warps w and w+4 share TMEM lane quarter
-//     w % 4).  Both read the row's 64 scores with tcgen05.ld and take the same
-//     row max, so they agree on the running max without talking to each other;
-//     each then exponentiates (ex2 on the fused scale) and writes its own 32
-//     columns of P as bf16 into a 128-byte-swizzled shared tile (the A operand
-//     of PV), and keeps its own partial row sum.  The two partial sums meet
-//     once per item, in the epilogue, which again splits the 256 O columns in
-//     halves.  The running max is only raised when it grows by more than 2^8 in
-//     the exponent; otherwise P keeps the stale max (values stay below 256), so
-//     the O accumulator is rescaled in tensor memory only on such rare jumps.
-//     The final O / l is exact either way.
+//     The Q tile is copied once per item from shared memory into the last 128
+//     tensor-memory columns (tcgen05.cp) and the S products read it from there,
+//     so each S product reads only the 64-key K tile from shared memory and the
+//     shared-memory Q tile is free for the next item's copy right away.
+//   * Softmax: the two warp groups (warps 0-3, 4-7) take alternate tiles, one
+//     thread per row with all 64 scores, so two tiles' exponentials overlap.  A
+//     tile's running max goes to the next tile's group through shared memory as
+//     soon as its row max is known.  The running max is only raised when it grows
+//     by more than 2^8 in the exponent; otherwise P keeps the stale max (values
+//     stay below 256), so O is rescaled in tensor memory only on such rare jumps.
+//     Each group keeps its partial row sum relative to the max it last used; the
+//     epilogue brings both to the final max.  P goes as bf16 into a 128-byte-
+//     swizzled shared tile (the A operand of P V).
 //   * The K/V rings, S/P buffers and their barriers run over one tile counter
-//     for all items of the CTA, so the next item's Q copy (as soon as the last S
-//     of the current item is done) and its first S product overlap the current
-//     item's last softmax, P V and O write-out.
+//     for all items of the CTA, so the next item's Q load (issued as soon as the
+//     current Q is in tensor memory) and its first S product overlap the current
+//     item's tiles, last softmax, P V and O write-out.
 //   * Every role loads the next item's offsets while it works on the current one.
 //   * Epilogue: each warp stages its 32 rows x 64 columns of O / l as bf16 in the idle
 //     P buffers and copies them out row-major, so every store writes whole lines.
@@ -60,8 +62,10 @@ constexpr int kQSlab = kBM * 128;              // 16 KB
 constexpr int kKVSlab = kBKV * 128;            // 8 KB
 constexpr int kPBytes = kBM * kBKV * 2;        // 1 slab of 128 rows x 128 B
 constexpr int kBarBytes = 256;
-constexpr int kSmem = 1024 + kQBytes + 2 * kKVBytes + 2 * kKVBytes + 2 * kPBytes + kBarBytes + 2 * 128 * 4;
-constexpr uint32_t kTmemCols = 512;            // O: [0,256), S0: [256,320), S1: [320,384)
+constexpr int kSmem = 1024 + kQBytes + 2 * kKVBytes + 2 * kKVBytes + 2 * kPBytes + kBarBytes + 2 * 128 * 4 + 128 * 4;
+static_assert(kSmem <= 227 * 1024, "attention shared memory");
+constexpr uint32_t kTmemCols = 512;            // O: [0,256), S0: [256,320), S1: [320,384), Q: [384,512)
+constexpr uint32_t kTmemQ = 384;               // the Q tile as bf16 pairs (A operand of S = Q K^T)
 constexpr uint32_t kIdescS = idesc_bf16_f32(kBM, kBKV, false, false);
 constexpr uint32_t kIdescPV = idesc_bf16_f32(kBM, kD, false, true);
 constexpr float kRescaleThreshold = 8.0f;      // log2 units
@@ -156,7 +160,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* sP = sV + 2 * kKVBytes;
   uint64_t* bars = reinterpret_cast<uint64_t*>(sP + 2 * kPBytes);
   uint64_t* bar_q = bars;        // Q landed (per item)
-  uint64_t* bar_qfree = bars + 1;  // last S of an item done: Q tile reusable (per item)
+  uint64_t* bar_qfree = bars + 1;  // Q copied into tensor memory: shared-memory Q tile reusable (per item)
   uint64_t* bar_k = bars + 2;    // [2] K tile landed
   uint64_t* bar_v = bars + 4;    // [2] V tile landed
   uint64_t* bar_s = bars + 6;    // [2] S ready
@@ -164,9 +168,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* bar_pv = bars + 10;  // [2] P V done
   uint64_t* bar_l = bars + 12;   // partial row sums published (per item)
   uint64_t* bar_ofree = bars + 13;  // O read out by the epilogue (per item)
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 14);
+  uint64_t* bar_m = bars + 14;   // [2] running max after a tile published (one per tile parity)
+  uint64_t* bar_sdone = bars + 16;  // every S of an item done: the Q columns of tensor memory reusable
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 17);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   float* l_part = reinterpret_cast<float*>(sP + 2 * kPBytes + kBarBytes);  // [2][128]
+  // running max after the latest tile, per row: written by the tile's group, read by the next
+  // tile's group after bar_m; the bar_m waits order every write after the previous read
+  float* m_pub = l_part + 2 * 128;                                         // [128]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
@@ -176,11 +185,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&bar_k[i], 1);
       mbar_init(&bar_v[i], 1);
       mbar_init(&bar_s[i], 1);
-      mbar_init(&bar_p[i], kSoftmaxThreads);
+      mbar_init(&bar_p[i], kSoftmaxThreads / 2);  // one warp group writes each tile's P
       mbar_init(&bar_pv[i], 1);
+      mbar_init(&bar_m[i], 4);                    // the four warps of that group
     }
     mbar_init(bar_l, kSoftmaxThreads);
     mbar_init(bar_ofree, kSoftmaxThreads);
+    mbar_init(bar_sdone, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -252,9 +263,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int kk = 0; kk < kD / 16; ++kk) {
           const uint32_t off = static_cast<uint32_t>((kk & 3) * 32);  // 16-element step inside a swizzle row
-          const uint64_t ad = sdesc_sw128(q_base + (kk >> 2) * kQSlab + off, 16, 1024);
           const uint64_t bd = sdesc_sw128(k_base + s * kKVBytes + (kk >> 2) * kKVSlab + off, 16, 1024);
-          umma_bf16_ss(d_s, ad, bd, kIdescS, kk != 0 ? 1u : 0u);
+          // Q from tensor memory: only the K tile is read from shared memory
+          umma_bf16_ts(d_s, tmem + kTmemQ + static_cast<uint32_t>(kk * 8), bd, kIdescS, kk != 0 ? 1u : 0u);
         }
         umma_commit(&bar_s[s]);
         return true;
@@ -269,9 +280,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         wc = item_at(p, pass + 1);
         nxt = load_item(p, wc);
         if (it.nt == 0) continue;
-        ok = mbar_wait(bar_q, n_it & 1, p.wait_ns);
+        // Q of this item: landed in shared memory, and the previous item's S products
+        // no longer read the Q columns -> copy it into tensor memory, then release the
+        // shared-memory tile so the next item's Q can load during this whole item
+        ok = mbar_wait(bar_q, n_it & 1, p.wait_ns) && (n_it == 0 || mbar_wait(bar_sdone, (n_it - 1) & 1, p.wait_ns));
         if (!ok) break;
         tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < kD / 16; ++kk)
+          tmem_cp_128x256b(tmem + kTmemQ + static_cast<uint32_t>(kk * 8),
+                           sdesc_sw128(q_base + (kk >> 2) * kQSlab + static_cast<uint32_t>((kk & 3) * 32), 16, 1024));
+        umma_commit(bar_qfree);
         ok = issue_s(J);
         for (int j = 0; j < it.nt && ok && !*abort_flag; ++j) {
           const uint32_t Jc = J + j;
@@ -280,7 +299,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             ok = issue_s(Jc + 1);
             if (!ok) break;
           } else {
-            umma_commit(bar_qfree);  // fires once every S of this item (and all before) is done
+            umma_commit(bar_sdone);  // fires once every S of this item (and all before) is done
           }
           if (!mbar_wait(&bar_p[s], (Jc >> 1) & 1, p.wait_ns) ||
               !mbar_wait(&bar_v[s], (Jc >> 1) & 1, p.wait_ns) ||
@@ -305,8 +324,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // ------------------------------------------------------------ softmax warps 0..7
+    // Two warp groups take alternate tiles (group = tile parity = S and P buffer), one
+    // thread per row with all 64 scores, so two tiles' exponentials run at once.  The
+    // running max passes from each tile to the next through shared memory as soon as
+    // the tile's row max is known; each group keeps its partial row sum relative to the
+    // max it last used, and the epilogue brings both to the final max.
     const int quarter = warp & 3;             // TMEM lane quarter
-    const int half = warp >> 2;               // which 32 of the 64 keys / 128 of the 256 O columns
+    const int half = warp >> 2;               // warp group; in the epilogue, which 128 O columns
     const int r = quarter * 32 + lane;        // packed row = TMEM lane
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
     const float c2 = p.scale_log2;
@@ -322,10 +346,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (it.nt == 0) continue;
       const int pos = it.pos0 + r / p.G;      // decoder position of this row
       const int hh = r % p.G;                 // query head within the KV group
-      float m_run = -INFINITY, l_run = 0.f;   // running max (log2 units) and this half's sum
+      float m_ref = -INFINITY, l_own = 0.f;   // this group's partial sum and the max it is relative to
       for (int j = 0; j < it.nt; ++j) {
         const uint32_t Jc = J + j;
         const int s = Jc & 1;
+        if (s != half) continue;              // the other group's tile
         bool wt = mbar_wait(&bar_s[s], (Jc >> 1) & 1, p.wait_ns);
         if (!__all_sync(0xffffffffu, wt) || *abort_flag) {
           ok = false;
@@ -354,38 +379,40 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int k = 0; k < w2; ++k) t32[k] = fmaxf(t32[k], t32[k + w2]);
         const float mx = t32[0] * c2;
-        float alpha = 1.f;
-        bool rescale = false;
-        if (j == 0) {
-          m_run = mx;  // every row sees self key 0, so mx is finite
-        } else if (mx > m_run + kRescaleThreshold) {
-          alpha = ex2_approx(m_run - mx);
-          m_run = mx;
-          rescale = true;
-        }
-        // this half's 32 probabilities: 2^(s * scale_log2 - m_run)
-        const float neg_m = -m_run;
-        float acc[4] = {0.f, 0.f, 0.f, 0.f};
-        uint32_t pk[16];
-#pragma unroll
-        for (int k = 0; k < 32; k += 2) {
-          const float s0 = __uint_as_float(half ? sr[32 + k] : sr[k]);
-          const float s1 = __uint_as_float(half ? sr[33 + k] : sr[k + 1]);
-          const float e0 = ex2_approx(fmaf(s0, c2, neg_m));
-          const float e1 = ex2_approx(fmaf(s1, c2, neg_m));
-          acc[(k >> 1) & 3] += e0 + e1;
-          pk[k >> 1] = pack_bf16x2(e0, e1);
-        }
-        l_run = l_run * alpha + ((acc[0] + acc[1]) + (acc[2] + acc[3]));
-        // the previous item's epilogue staged O in the P buffers
-        if (j == 0 && n_it >= 1) {
-          const bool wo = mbar_wait(bar_ofree, (n_it - 1) & 1, p.wait_ns);
-          if (!__all_sync(0xffffffffu, wo)) {
+        // running max after the previous tile (the other group's), or none at an item's start
+        float m_prev = -INFINITY;
+        if (j > 0) {
+          const bool wm = mbar_wait(&bar_m[s ^ 1], ((Jc - 1) >> 1) & 1, p.wait_ns);
+          if (!__all_sync(0xffffffffu, wm)) {
             ok = false;
             break;
           }
+          m_prev = m_pub[r];
         }
-        // P stage s is free once PV_{j-2} has completed
+        // lazy max: raised only when it grows by more than 2^8 (j == 0: every row sees self key 0)
+        const bool rescale = j > 0 && mx > m_prev + kRescaleThreshold;
+        const float m_run = (j == 0 || rescale) ? mx : m_prev;
+        m_pub[r] = m_run;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bar_m[s]);
+        if (m_ref != m_run) {  // this group's sum so far was relative to an older max
+          l_own = (m_ref == -INFINITY) ? 0.f : l_own * ex2_approx(m_ref - m_run);
+          m_ref = m_run;
+        }
+        // the row's 64 probabilities: 2^(s * scale_log2 - m_run)
+        const float neg_m = -m_run;
+        float acc[4] = {0.f, 0.f, 0.f, 0.f};
+        uint32_t pk[32];
+#pragma unroll
+        for (int k = 0; k < 64; k += 2) {
+          const float e0 = ex2_approx(fmaf(__uint_as_float(sr[k]), c2, neg_m));
+          const float e1 = ex2_approx(fmaf(__uint_as_float(sr[k + 1]), c2, neg_m));
+          acc[(k >> 1) & 3] += e0 + e1;
+          pk[k >> 1] = pack_bf16x2(e0, e1);
+        }
+        l_own += (acc[0] + acc[1]) + (acc[2] + acc[3]);
+        // P buffer s is free once PV_{Jc-2} has completed (also when this warp's epilogue
+        // staging, which lives in the same rows of the same buffer, is done: program order)
         if (Jc >= 2) {
           const bool wp = mbar_wait(&bar_pv[s], ((Jc - 2) >> 1) & 1, p.wait_ns);
           if (!__all_sync(0xffffffffu, wp)) {
@@ -396,25 +423,26 @@ __global__ void __launch_bounds__(kThreads, 1)
         // 128-byte swizzled K-major row: 16-byte unit u of row r sits at unit u ^ (r & 7)
         uint8_t* prow = sP + s * kPBytes + r * 128;
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
+        for (int c = 0; c < 8; ++c) {
           uint4 v;
           v.x = pk[4 * c + 0];
           v.y = pk[4 * c + 1];
           v.z = pk[4 * c + 2];
           v.w = pk[4 * c + 3];
-          *reinterpret_cast<uint4*>(prow + (((half * 4 + c) ^ (r & 7)) << 4)) = v;
+          *reinterpret_cast<uint4*>(prow + ((c ^ (r & 7)) << 4)) = v;
         }
         fence_proxy_async_smem();
         if (__any_sync(0xffffffffu, rescale)) {
-          // O must hold the result of PV_{j-1} before it is rescaled in place
-          const bool wr = mbar_wait(&bar_pv[(Jc - 1) & 1], ((Jc - 1) >> 1) & 1, p.wait_ns);
+          // O must hold the result of PV_{Jc-1} before it is rescaled in place
+          const bool wr = mbar_wait(&bar_pv[s ^ 1], ((Jc - 1) >> 1) & 1, p.wait_ns);
           if (!__all_sync(0xffffffffu, wr)) {
             ok = false;
             break;
           }
           tc_fence_after();
+          const float alpha = rescale ? ex2_approx(m_prev - m_run) : 1.f;
 #pragma unroll 1
-          for (int c = half * 128; c < half * 128 + 128; c += 32) {
+          for (int c = 0; c < kD; c += 32) {
             uint32_t o[32];
             tmem_ld32(lane_base + c, o);
             tmem_ld_wait();
@@ -428,10 +456,22 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_arrive(&bar_p[s]);
       }
       if (!ok) break;
+      // both groups' sums relative to the final running max (published by the last tile)
+      const uint32_t Jl = J + it.nt - 1;
+      float m_fin = m_ref;
+      if (static_cast<int>(Jl & 1) != half) {
+        const bool wm = mbar_wait(&bar_m[Jl & 1], (Jl >> 1) & 1, p.wait_ns);
+        if (!__all_sync(0xffffffffu, wm)) {
+          ok = false;
+          break;
+        }
+        m_fin = m_pub[r];
+      }
+      const float l_run = (m_ref == -INFINITY) ? 0.f : l_own * ex2_approx(m_ref - m_fin);
+      const float m_run = m_fin;
       // ---- epilogue of this item: O / l -> bf16, this half's 128 columns
       l_part[half * 128 + r] = l_run;
       mbar_arrive(bar_l);
-      const uint32_t Jl = J + it.nt - 1;
       bool wt = mbar_wait(&bar_pv[Jl & 1], (Jl >> 1) & 1, p.wait_ns) && mbar_wait(bar_l, n_it & 1, p.wait_ns);
       if (!__all_sync(0xffffffffu, wt)) {
         ok = false;
