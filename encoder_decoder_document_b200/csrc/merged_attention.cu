@@ -399,18 +399,6 @@ __global__ void __launch_bounds__(kThreads, 1)
           l_own = (m_ref == -INFINITY) ? 0.f : l_own * ex2_approx(m_ref - m_run);
           m_ref = m_run;
         }
-        // the row's 64 probabilities: 2^(s * scale_log2 - m_run)
-        const float neg_m = -m_run;
-        float acc[4] = {0.f, 0.f, 0.f, 0.f};
-        uint32_t pk[32];
-#pragma unroll
-        for (int k = 0; k < 64; k += 2) {
-          const float e0 = ex2_approx(fmaf(__uint_as_float(sr[k]), c2, neg_m));
-          const float e1 = ex2_approx(fmaf(__uint_as_float(sr[k + 1]), c2, neg_m));
-          acc[(k >> 1) & 3] += e0 + e1;
-          pk[k >> 1] = pack_bf16x2(e0, e1);
-        }
-        l_own += (acc[0] + acc[1]) + (acc[2] + acc[3]);
         // P buffer s is free once PV_{Jc-2} has completed (also when this warp's epilogue
         // staging, which lives in the same rows of the same buffer, is done: program order)
         if (Jc >= 2) {
@@ -420,17 +408,33 @@ __global__ void __launch_bounds__(kThreads, 1)
             break;
           }
         }
-        // 128-byte swizzled K-major row: 16-byte unit u of row r sits at unit u ^ (r & 7)
+        // the row's 64 probabilities 2^(s * scale_log2 - m_run), written as bf16 into the
+        // 128-byte swizzled K-major row (16-byte unit u of row r sits at unit u ^ (r & 7)),
+        // 32 at a time
+        const float neg_m = -m_run;
+        float acc[4] = {0.f, 0.f, 0.f, 0.f};
         uint8_t* prow = sP + s * kPBytes + r * 128;
 #pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          uint4 v;
-          v.x = pk[4 * c + 0];
-          v.y = pk[4 * c + 1];
-          v.z = pk[4 * c + 2];
-          v.w = pk[4 * c + 3];
-          *reinterpret_cast<uint4*>(prow + ((c ^ (r & 7)) << 4)) = v;
+        for (int hp = 0; hp < 2; ++hp) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int k = 0; k < 32; k += 2) {
+            const float e0 = ex2_approx(fmaf(__uint_as_float(sr[32 * hp + k]), c2, neg_m));
+            const float e1 = ex2_approx(fmaf(__uint_as_float(sr[32 * hp + k + 1]), c2, neg_m));
+            acc[(k >> 1) & 3] += e0 + e1;
+            pk[k >> 1] = pack_bf16x2(e0, e1);
+          }
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            uint4 v;
+            v.x = pk[4 * c + 0];
+            v.y = pk[4 * c + 1];
+            v.z = pk[4 * c + 2];
+            v.w = pk[4 * c + 3];
+            *reinterpret_cast<uint4*>(prow + (((4 * hp + c) ^ (r & 7)) << 4)) = v;
+          }
         }
+        l_own += (acc[0] + acc[1]) + (acc[2] + acc[3]);
         fence_proxy_async_smem();
         if (__any_sync(0xffffffffu, rescale)) {
           // O must hold the result of PV_{Jc-1} before it is rescaled in place
