@@ -19,6 +19,7 @@ on a bounded sample of the same workload on the host cores.
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import json
 import math
 import os
@@ -50,6 +51,8 @@ def parse():
     ap.add_argument("--no-pool-sweep", action="store_true", help="skip the pooling-only sweep at 1024/4096 docs")
     ap.add_argument("--rope-theta", type=float, default=None,
                     help="rotate the decoder's self Q/K with this rotary base in every layer (default: off)")
+    ap.add_argument("--sweep", action="store_true",
+                    help="end-to-end throughput at the sweep shapes (1..4096 documents per query), one JSON line")
     ap.add_argument("--pool-sweep-only", action="store_true",
                     help="run only the pooling sweep at 1024/4096 documents and print it as one JSON line")
     return ap.parse_args()
@@ -182,6 +185,62 @@ def rope_alone(sc, theta=1e4, reps=10):
             "gbs": byts / (us * 1e-6) / 1e9}
 
 
+def run_sweep(args, doc_counts=(1, 16, 100, 1024, 4096)):
+    """End-to-end throughput at the sweep shapes (Nano model, log-normal lengths with
+    median 200 clipped to [1, 1024], one seeded query per point with Lq drawn from
+    [32, 512]): K steps of the captured graph per point, L2 flushed before each step,
+    plus the pooling and attention kernels' own times from the instrumented graph."""
+    import torch
+    import synthetic
+    from encoder_decoder_document_b200 import _build, kalm_check_device_errors
+    from encoder_decoder_document_b200.scorer import DeviceWeights, FBNLScorer
+    _build.build()
+    pk = peaks()
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device="cuda")
+    weights = None
+    out = []
+    for n in doc_counts:
+        q = synthetic.make_query("sweep", n_docs=n, seed=4, with_weights=weights is None)
+        if weights is None:
+            weights = q.weights
+        q = dataclasses.replace(q, weights=weights)
+        w = workload(q)
+        sc = FBNLScorer(DeviceWeights.from_bits(weights), q.n_q, q.n_kv)
+        total_pooled = int(((q.doc_len.astype(np.int64) + 3) // 4).sum())
+        sc.prepare(q.n_docs, int(q.doc_len.sum()), total_pooled, q.lq)
+        sc.load_inputs(torch.from_numpy(q.enc.view(np.int16)).view(torch.bfloat16),
+                       torch.from_numpy(q.doc_len), torch.from_numpy(q.x0.view(np.int16)).view(torch.bfloat16))
+        sc.capture(instrument=True)
+        ts, per = [], {}
+        for i in range(args.warmup + args.steps):
+            for g in (sc.graph, sc.graph_inst):
+                flush.fill_(1.0)
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record()
+                g.replay()
+                b.record()
+                b.synchronize()
+                if i >= args.warmup:
+                    if g is sc.graph:
+                        ts.append(a.elapsed_time(b))
+                    else:
+                        for label, v in sc.kernel_times().items():
+                            per.setdefault(label, []).extend(v)
+        kalm_check_device_errors()
+        ms = statistics.median(ts)
+        attn_us = 1e3 * sum(per["merged_attention"]) / args.steps
+        pool_us = 1e3 * statistics.mean(per["chunk_pool"])
+        out.append({"docs": n, "lq": q.lq, "encoder_tokens": int(q.doc_len.sum()), "ms_per_query": ms,
+                    "pairs_per_s": n / (ms * 1e-3), "step_tflops": w["total_flops"] / (ms * 1e-3) / 1e12,
+                    "attention_us": attn_us, "attention_tflops": w["merged_attention"] / (attn_us * 1e-6) / 1e12,
+                    "pool_us": pool_us, "pool_gbs": w["pool_bytes"] / (pool_us * 1e-6) / 1e9,
+                    "pool_frac": w["pool_bytes"] / (pool_us * 1e-6) / 1e9 / pk["hbm"]})
+        print(json.dumps(out[-1]), flush=True)
+        del sc
+        torch.cuda.empty_cache()
+    return out
+
+
 def pool_sweep(doc_counts=(1024, 4096), reps=10):
     """The pooling kernel alone at the throughput-sweep shapes with many documents
     (hidden 640, log-normal lengths, median 200, clipped to [1, 1024]): bytes moved,
@@ -312,6 +371,9 @@ def run_reference(args):
 
 def main():
     args = parse()
+    if args.sweep:
+        print(json.dumps({"sweep": run_sweep(args)}), flush=True)
+        return
     if args.pool_sweep_only:
         pk = peaks()
         sweep = [dict(x, peak_gbs=pk["hbm"], frac=x["gbs"] / pk["hbm"]) for x in pool_sweep()]
