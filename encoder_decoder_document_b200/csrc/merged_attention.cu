@@ -38,7 +38,10 @@
 //   * Epilogue: each warp stages its 32 rows x 64 columns of O / l as bf16 in the idle
 //     P buffers and copies them out row-major, so every store writes whole lines.
 //   * Warp roles: warps 0-7 softmax + epilogue, warp 8 TMA producer of Q and K,
-//     warp 10 TMA producer of V, warp 9 tensor-memory allocation and MMA issue.
+//     warp 10 TMA producer of V, warp 9 tensor-memory allocation, the Q copy and
+//     the S products, warp 11 the P V products.  With two issuing threads, S of the
+//     next tiles goes out while P V waits for the softmax, so the tensor pipe does
+//     not idle behind one thread's waits.
 #include <cmath>
 
 #include "kalm.h"
@@ -51,11 +54,12 @@ namespace {
 constexpr int kD = 256;
 constexpr int kBM = 128;
 constexpr int kBKV = 64;
-constexpr int kThreads = 352;
+constexpr int kThreads = 384;
 constexpr int kSoftmaxThreads = 256;
 constexpr int kTmaWarp = 8;
 constexpr int kMmaWarp = 9;
 constexpr int kTmaWarpV = 10;
+constexpr int kMmaWarpPV = 11;
 constexpr int kQBytes = kBM * kD * 2;          // 4 slabs of 128 rows x 128 B
 constexpr int kKVBytes = kBKV * kD * 2;        // 4 slabs of 64 rows x 128 B
 constexpr int kQSlab = kBM * 128;              // 16 KB
@@ -219,6 +223,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t J = 0;  // tile counter over all items of this CTA
       int n_it = 0;
       bool ok = true;
+      bool q_ready = false;  // the current item's Q was issued during the previous item
       int wc = item_at(p, 0);
       Item nxt = load_item(p, wc);
       for (int pass = 0; wc != kNoMore && ok && !*abort_flag; ++pass) {
@@ -226,7 +231,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         wc = item_at(p, pass + 1);
         nxt = load_item(p, wc);
         if (it.nt == 0) continue;
-        if (!is_v) {
+        // The shared-memory Q tile is free once the previous item's Q is in tensor memory,
+        // which happens at that item's start, so the Q+K producer normally issues an
+        // item's Q during the previous item (q_ready); here only if that did not happen.
+        if (!is_v && !q_ready) {
           if (n_it >= 1 && !mbar_wait(bar_qfree, (n_it - 1) & 1, p.wait_ns)) {
             fail_wait();
             break;
@@ -234,6 +242,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           mbar_arrive_expect_tx(bar_q, kQBytes);
           tma_load_4d(sQ, &tm_q, bar_q, 0, it.g * p.G, static_cast<int32_t>(it.qi + it.pos0), 0);
         }
+        q_ready = false;
         for (int j = 0; j < it.nt; ++j, ++J) {
           const int s = J & 1;
           const bool self = j < it.n_self;
@@ -247,29 +256,27 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           mbar_arrive_expect_tx(&bar_full[s], kKVBytes);
           tma_load_3d(ring + s * kKVBytes, m, &bar_full[s], 0, row, it.g * 4);
+          if (!is_v && j == 0 && nxt.nt > 0) {
+            // next item's Q as soon as this item's Q is in tensor memory
+            if (!mbar_wait(bar_qfree, n_it & 1, p.wait_ns)) {
+              fail_wait();
+              ok = false;
+              break;
+            }
+            mbar_arrive_expect_tx(bar_q, kQBytes);
+            tma_load_4d(sQ, &tm_q, bar_q, 0, nxt.g * p.G, static_cast<int32_t>(nxt.qi + nxt.pos0), 0);
+            q_ready = true;
+          }
         }
         ++n_it;
       }
     }
   } else if (warp == kMmaWarp) {
-    // ------------------------------------------------------------ MMA issuer
+    // ------------------------------------------------------------ S issuer: Q copy and S = Q K^T
+    // S of tile J goes out as soon as K_J has landed and the softmax has read S_{J-2}
+    // (same buffer), independently of the P V products, which warp 11 issues.
     if (lane == 0) {
-      const uint32_t q_base = smem_u32(sQ), k_base = smem_u32(sK), v_base = smem_u32(sV), p_base = smem_u32(sP);
-      auto issue_s = [&](uint32_t J) -> bool {
-        const int s = J & 1;
-        if (!mbar_wait(&bar_k[s], (J >> 1) & 1, p.wait_ns)) return false;
-        tc_fence_after();
-        const uint32_t d_s = tmem + 256u + static_cast<uint32_t>(s * kBKV);
-#pragma unroll
-        for (int kk = 0; kk < kD / 16; ++kk) {
-          const uint32_t off = static_cast<uint32_t>((kk & 3) * 32);  // 16-element step inside a swizzle row
-          const uint64_t bd = sdesc_sw128(k_base + s * kKVBytes + (kk >> 2) * kKVSlab + off, 16, 1024);
-          // Q from tensor memory: only the K tile is read from shared memory
-          umma_bf16_ts(d_s, tmem + kTmemQ + static_cast<uint32_t>(kk * 8), bd, kIdescS, kk != 0 ? 1u : 0u);
-        }
-        umma_commit(&bar_s[s]);
-        return true;
-      };
+      const uint32_t q_base = smem_u32(sQ), k_base = smem_u32(sK);
       uint32_t J = 0;
       int n_it = 0;
       bool ok = true;
@@ -291,16 +298,48 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_cp_128x256b(tmem + kTmemQ + static_cast<uint32_t>(kk * 8),
                            sdesc_sw128(q_base + (kk >> 2) * kQSlab + static_cast<uint32_t>((kk & 3) * 32), 16, 1024));
         umma_commit(bar_qfree);
-        ok = issue_s(J);
         for (int j = 0; j < it.nt && ok && !*abort_flag; ++j) {
           const uint32_t Jc = J + j;
           const int s = Jc & 1;
-          if (j + 1 < it.nt) {
-            ok = issue_s(Jc + 1);
-            if (!ok) break;
-          } else {
-            umma_commit(bar_sdone);  // fires once every S of this item (and all before) is done
+          if (!mbar_wait(&bar_k[s], (Jc >> 1) & 1, p.wait_ns) ||
+              (Jc >= 2 && !mbar_wait(&bar_p[s], ((Jc - 2) >> 1) & 1, p.wait_ns))) {  // S_{Jc-2} read
+            ok = false;
+            break;
           }
+          tc_fence_after();
+          const uint32_t d_s = tmem + 256u + static_cast<uint32_t>(s * kBKV);
+#pragma unroll
+          for (int kk = 0; kk < kD / 16; ++kk) {
+            const uint32_t off = static_cast<uint32_t>((kk & 3) * 32);  // 16-element step inside a swizzle row
+            const uint64_t bd = sdesc_sw128(k_base + s * kKVBytes + (kk >> 2) * kKVSlab + off, 16, 1024);
+            // Q from tensor memory: only the K tile is read from shared memory
+            umma_bf16_ts(d_s, tmem + kTmemQ + static_cast<uint32_t>(kk * 8), bd, kIdescS, kk != 0 ? 1u : 0u);
+          }
+          umma_commit(&bar_s[s]);
+          if (j + 1 == it.nt) umma_commit(bar_sdone);  // every S of this item done
+        }
+        J += it.nt;
+        ++n_it;
+      }
+      if (!ok) fail_wait();
+    }
+  } else if (warp == kMmaWarpPV) {
+    // ------------------------------------------------------------ P V issuer
+    if (lane == 0) {
+      const uint32_t v_base = smem_u32(sV), p_base = smem_u32(sP);
+      uint32_t J = 0;
+      int n_it = 0;
+      bool ok = true;
+      int wc = item_at(p, 0);
+      Item nxt = load_item(p, wc);
+      for (int pass = 0; wc != kNoMore && ok && !*abort_flag; ++pass) {
+        const Item it = nxt;
+        wc = item_at(p, pass + 1);
+        nxt = load_item(p, wc);
+        if (it.nt == 0) continue;
+        for (int j = 0; j < it.nt && ok && !*abort_flag; ++j) {
+          const uint32_t Jc = J + j;
+          const int s = Jc & 1;
           if (!mbar_wait(&bar_p[s], (Jc >> 1) & 1, p.wait_ns) ||
               !mbar_wait(&bar_v[s], (Jc >> 1) & 1, p.wait_ns) ||
               (j == 0 && n_it >= 1 && !mbar_wait(bar_ofree, (n_it - 1) & 1, p.wait_ns))) {
