@@ -531,22 +531,32 @@ __global__ void __launch_bounds__(kThreads, 1)
       // per 128-byte row, so every global store instruction writes 4 whole lines.
       const int r0 = quarter * 32;
       uint8_t* stage = sP + warp * 4096;
-#pragma unroll 1
-      for (int sl = 2 * half; sl < 2 * half + 2; ++sl) {
-        uint4 v[8];
+      // this thread's 128 O columns, two 32-column loads per wait, packed to bf16; O is
+      // then free for the next item's P V before any store is issued
+      uint4 vv[2][8];
 #pragma unroll
-        for (int c2 = 0; c2 < 2; ++c2) {
-          uint32_t o[32];
-          tmem_ld32(lane_base + sl * 64 + c2 * 32, o);
-          tmem_ld_wait();
+      for (int hs = 0; hs < 2; ++hs) {
+        uint32_t o[2][32];
+        tmem_ld32(lane_base + half * 128 + hs * 64, o[0]);
+        tmem_ld32(lane_base + half * 128 + hs * 64 + 32, o[1]);
+        tmem_ld_wait();
+#pragma unroll
+        for (int c = 0; c < 2; ++c)
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
-            v[c2 * 4 + q].x = pack_bf16x2(__uint_as_float(o[8 * q + 0]) * inv_l, __uint_as_float(o[8 * q + 1]) * inv_l);
-            v[c2 * 4 + q].y = pack_bf16x2(__uint_as_float(o[8 * q + 2]) * inv_l, __uint_as_float(o[8 * q + 3]) * inv_l);
-            v[c2 * 4 + q].z = pack_bf16x2(__uint_as_float(o[8 * q + 4]) * inv_l, __uint_as_float(o[8 * q + 5]) * inv_l);
-            v[c2 * 4 + q].w = pack_bf16x2(__uint_as_float(o[8 * q + 6]) * inv_l, __uint_as_float(o[8 * q + 7]) * inv_l);
+            uint4& v = vv[hs][c * 4 + q];
+            v.x = pack_bf16x2(__uint_as_float(o[c][8 * q + 0]) * inv_l, __uint_as_float(o[c][8 * q + 1]) * inv_l);
+            v.y = pack_bf16x2(__uint_as_float(o[c][8 * q + 2]) * inv_l, __uint_as_float(o[c][8 * q + 3]) * inv_l);
+            v.z = pack_bf16x2(__uint_as_float(o[c][8 * q + 4]) * inv_l, __uint_as_float(o[c][8 * q + 5]) * inv_l);
+            v.w = pack_bf16x2(__uint_as_float(o[c][8 * q + 6]) * inv_l, __uint_as_float(o[c][8 * q + 7]) * inv_l);
           }
-        }
+      }
+      tc_fence_before();
+      mbar_arrive(bar_ofree);  // O read out: the next item's first P V may overwrite it
+#pragma unroll
+      for (int hs = 0; hs < 2; ++hs) {
+        const int sl = 2 * half + hs;
+        const uint4* v = vv[hs];
         uint8_t* row = stage + lane * 128;
 #pragma unroll
         for (int u = 0; u < 8; ++u) *reinterpret_cast<uint4*>(row + ((u ^ (lane & 7)) << 4)) = v[u];
@@ -566,9 +576,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         __syncwarp();  // staging tile read before it is refilled
       }
-      tc_fence_before();
-      // O read out and the staging tiles free: the next item may overwrite O and P
-      mbar_arrive(bar_ofree);
       if (valid && half == 0 && p.lse) {
         // natural-log softmax denominator in scaled-logit units
         p.lse[(it.q0 + pos) * p.n_q + head] = (m_run + log2f(l_tot)) * 0.69314718055994531f;
