@@ -162,27 +162,36 @@ def pool_chunks(enc, len_d, chunks=(1, 2, 4, 8), reps=10):
 
 
 def rope_alone(sc, theta=1e4, reps=10):
-    """The rotary-embedding kernel alone on one layer's Q|K|V buffer (all documents'
-    rows, Q and self-K heads): median time (L2 flushed before each call), bytes
-    read + written, GB/s."""
+    """Cost of the rotary embedding on one layer's Q|K|V (all documents' rows, Q and
+    self-K heads), L2 flushed before each call, medians: the standalone rotation
+    kernel (bytes read + written, GB/s), and the Q|K|V projection without and with
+    the rotation fused into its epilogue."""
     import torch
-    from encoder_decoder_document_b200 import kalm_rope
+    from encoder_decoder_document_b200 import kalm_linear, kalm_linear_rope, kalm_rope
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device="cuda")
     heads = sc.n_q + sc.n_kv
-    ts = []
-    for i in range(reps + 2):
-        flush.fill_(1.0)
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record()
-        kalm_rope(sc.qkv, sc.q_off, heads, theta, sc.D)
-        b.record()
-        b.synchronize()
-        if i >= 2:
-            ts.append(a.elapsed_time(b))
-    us = 1e3 * statistics.median(ts)
+    w = sc.w.w_qkv[1]
+
+    def timed(fn):
+        ts = []
+        for i in range(reps + 2):
+            flush.fill_(1.0)
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            fn()
+            b.record()
+            b.synchronize()
+            if i >= 2:
+                ts.append(a.elapsed_time(b))
+        return 1e3 * statistics.median(ts)
+
+    us = timed(lambda: kalm_rope(sc.qkv, sc.q_off, heads, theta, sc.D))
+    plain = timed(lambda: kalm_linear(sc.x, w, sc.qkv))
+    fused = timed(lambda: kalm_linear_rope(sc.x, w, sc.qkv, sc.q_off, heads, theta, sc.D))
     byts = 2 * sc.qkv.shape[0] * heads * sc.D * 2
     return {"rows": sc.qkv.shape[0], "heads": heads, "theta": theta, "bytes": byts, "us": us,
-            "gbs": byts / (us * 1e-6) / 1e9}
+            "gbs": byts / (us * 1e-6) / 1e9, "qkv_proj_us": plain, "qkv_proj_rope_us": fused,
+            "fused_extra_us": fused - plain}
 
 
 def run_sweep(args, doc_counts=(1, 16, 100, 1024, 4096)):

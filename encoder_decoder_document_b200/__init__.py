@@ -18,7 +18,7 @@ __all__ = [
     "KalmError", "load", "library_path", "kalm_version", "kalm_device_check", "kalm_check_device_errors",
     "kalm_ragged_offsets", "kalm_chunk_pool", "kalm_linear", "kalm_cross_kv_proj", "kalm_merged_attention",
     "kalm_yes_no_score", "kalm_broadcast_rows", "kalm_selftest_wait_timeout", "kalm_attention_items",
-    "kalm_attention_schedule", "kalm_rope",
+    "kalm_attention_schedule", "kalm_rope", "kalm_linear_rope",
 ]
 
 HEAD_DIM = 256
@@ -151,6 +151,19 @@ def kalm_rope(x: torch.Tensor, q_off: torch.Tensor, n_heads: int, theta: float, 
     decoder position (row - q_off[d] for the document d owning the row)."""
     call("kalm_rope", _p(x, torch.bfloat16), _ld(x), x.shape[0], n_heads, head_dim, _p(q_off, torch.int64),
          q_off.numel() - 1, float(theta), _stream(stream))
+
+
+def kalm_linear_rope(x: torch.Tensor, w: torch.Tensor, y: torch.Tensor, q_off: torch.Tensor, rot_heads: int,
+                     theta: float, head_dim: int = HEAD_DIM, stream=None) -> None:
+    """y = x . w^T with the first rot_heads head vectors of every row rotated by the
+    row's decoder position, in the projection's epilogue."""
+    m, k = x.shape
+    n = w.shape[0]
+    if w.shape[1] != k or y.shape[0] != m or y.shape[1] != n:
+        raise KalmError(1, "kalm_linear_rope", f"shapes x{tuple(x.shape)} w{tuple(w.shape)} y{tuple(y.shape)}")
+    call("kalm_linear_rope", _p(x, torch.bfloat16), _ld(x), _p(w, torch.bfloat16), _ld(w), _p(y, torch.bfloat16),
+         _ld(y), m, n, k, rot_heads * head_dim, head_dim, _p(q_off, torch.int64), q_off.numel() - 1, float(theta),
+         _stream(stream))
 
 
 def kalm_selftest_wait_timeout(wait_ns: int, stream=None) -> None:

@@ -352,6 +352,34 @@ __device__ __forceinline__ void umma_commit_pair_multicast(uint64_t* bar, uint16
       : "memory");
 }
 
+// ---------------------------------------------------------------- rotary embedding
+// sin and cos of an angle in [0, 512 rad]: Cody-Waite reduction by 2*pi (W. J. Cody
+// and W. Waite, "Software Manual for the Elementary Functions", 1980) with 2*pi
+// split into a short head (8 significant bits, so k * head is exact for k < 2^15)
+// and a tail, then the hardware approximation on |r| <= pi.  Error stays near
+// 1e-6 rad, far below one bf16 step of the rotated values.
+__device__ __forceinline__ void sincos_reduced(float a, float* s, float* c) {
+  constexpr float kTwoPiHead = 6.28125f;                  // 201/32
+  constexpr float kTwoPiTail = 1.935307179586232e-3f;     // 2*pi - 201/32
+  constexpr float kInvTwoPi = 0.15915494309189535f;
+  const float k = rintf(a * kInvTwoPi);
+  float r = fmaf(-k, kTwoPiHead, a);
+  r = fmaf(-k, kTwoPiTail, r);
+  __sincosf(r, s, c);
+}
+
+// Rotation of pair p (element p and element p + head_dim/2) at decoder position
+// pos: angle pos * theta^(-2p/head_dim), computed as 2^(-p * (2/head_dim) *
+// log2(theta)); (a, b) -> (a cos - b sin, b cos + a sin) with fixed rounding
+// steps, so every kernel that rotates gets the same bits.
+__device__ __forceinline__ void rope_pair(float pos, int pair, float inv_half_d, float log2_theta, float a, float b,
+                                          float* ra, float* rb) {
+  float sn, cs;
+  sincos_reduced(pos * exp2f(-static_cast<float>(pair) * inv_half_d * log2_theta), &sn, &cs);
+  *ra = fmaf(a, cs, __fmul_rn(-b, sn));
+  *rb = fmaf(b, cs, __fmul_rn(a, sn));
+}
+
 // Pack two fp32 into a bf16x2 word (round to nearest even), low half = a.
 __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
   __nv_bfloat162 v = __floats2bfloat162_rn(a, b);

@@ -23,6 +23,8 @@
 // The accumulator is double-buffered in TMEM (2 x BN columns) so the epilogue
 // of tile i overlaps the main loop of tile i+1.  Out-of-range rows/columns of
 // x and w are zero-filled by TMA; the epilogue masks their stores.
+#include <cmath>
+
 #include "kalm.h"
 #include "kalm_internal.h"
 #include "kalm_ptx.cuh"
@@ -61,13 +63,87 @@ __device__ __forceinline__ void epi_prefetch_residual(const CUtensorMap* tm_r, u
   }
 }
 
+// Optional rotary embedding applied in the epilogue of a Q|K|V projection: output
+// columns [0, rot_cols) are head vectors of 256 elements (one 256-column tile is one
+// head) rotated by the row's decoder position (row - q_off[d] for its document d).
+struct RopeArgs {
+  const int64_t* q_off;
+  int n_docs;
+  int rot_cols;  // 0: no rotation
+  float log2_theta;
+  float inv_half_d;  // 2 / head_dim
+  int64_t rows;      // M: rows past it are clipped by the store
+  uint32_t* err;     // device error word: a stored row whose position is out of range
+};
+
+// One 32-column chunk of one warp's 32 rows: bf16 into a 64-byte-swizzled staging
+// slot, then a TMA tile store.  The slot is reused once the store issued from it two
+// chunks ago has read it.
+__device__ __forceinline__ void epi_emit(const float (&v)[32], int col, int row0, const CUtensorMap* tm_y,
+                                         uint8_t* obuf, int& out_slot, int lane) {
+  // 64-byte swizzle of a 32 x 64 B chunk: 16-byte unit i of row r sits at unit i ^ ((r >> 1) & 3)
+  const uint32_t swz = static_cast<uint32_t>((lane >> 1) & 3);
+  if (lane == 0) bulk_wait_group_read<1>();
+  __syncwarp();
+  uint8_t* orow = obuf + out_slot * kChunkBytes + lane * 64;
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    uint4 o;
+    o.x = pack_bf16x2(v[q * 8 + 0], v[q * 8 + 1]);
+    o.y = pack_bf16x2(v[q * 8 + 2], v[q * 8 + 3]);
+    o.z = pack_bf16x2(v[q * 8 + 4], v[q * 8 + 5]);
+    o.w = pack_bf16x2(v[q * 8 + 6], v[q * 8 + 7]);
+    *reinterpret_cast<uint4*>(orow + ((q ^ swz) << 4)) = o;
+  }
+  fence_proxy_async_smem();
+  __syncwarp();
+  if (lane == 0) {
+    tma_store_2d(tm_y, obuf + out_slot * kChunkBytes, col, row0);
+    bulk_commit_group();
+  }
+  out_slot ^= 1;
+}
+
 // Epilogue of one tile for one warp: 32 rows (TMEM lanes of this warp) x nch
 // 32-column chunks.  fp32 accumulator (+ residual) -> bf16 -> swizzled staging
-// chunk -> TMA tile store.  Returns false if a bounded wait expired.
+// chunk -> TMA tile store.  A tile of rotated heads pairs chunk c with chunk c + 4
+// (element i with element i + 128): both are rounded to bf16 (the stored
+// projection), rotated in fp32 and rounded again.  Returns false if a bounded wait
+// expired.
 __device__ __forceinline__ bool epi_tile(uint32_t t_row, int nch, int n0, int row0, bool has_residual,
                                          const CUtensorMap* tm_y, const CUtensorMap* tm_r, uint8_t* obuf,
                                          uint8_t* rbuf, uint64_t* rbar, uint32_t& rphase, int& out_slot, int lane,
-                                         uint64_t wait_ns) {
+                                         uint64_t wait_ns, const RopeArgs& rope) {
+  if (n0 < rope.rot_cols && nch == 8) {
+    // decoder position of this lane's row
+    const int64_t m = row0 + lane;
+    int lo = 0, hi = rope.n_docs - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (__ldg(rope.q_off + mid) <= m) lo = mid; else hi = mid - 1;
+    }
+    const int64_t pos64 = m - __ldg(rope.q_off + lo);
+    if (m < rope.rows && (pos64 < 0 || pos64 >= KALM_MAX_QUERY_TOKENS))
+      record_error(rope.err, kErrDeviceArg | kSiteRope);
+    const float pos = static_cast<float>(pos64);
+#pragma unroll 1
+    for (int c = 0; c < 4; ++c) {
+      uint32_t ra[32], rb[32];
+      tmem_ld32(t_row + c * 32, ra);
+      tmem_ld32(t_row + (c + 4) * 32, rb);
+      tmem_ld_wait();
+      float va[32], vb[32];
+#pragma unroll
+      for (int j = 0; j < 32; ++j) {
+        const float a = __bfloat162float(__float2bfloat16_rn(__uint_as_float(ra[j])));
+        const float b = __bfloat162float(__float2bfloat16_rn(__uint_as_float(rb[j])));
+        rope_pair(pos, c * 32 + j, rope.inv_half_d, rope.log2_theta, a, b, &va[j], &vb[j]);
+      }
+      epi_emit(va, n0 + c * 32, row0, tm_y, obuf, out_slot, lane);
+      epi_emit(vb, n0 + (c + 4) * 32, row0, tm_y, obuf, out_slot, lane);
+    }
+    return true;
+  }
   // 64-byte swizzle of a 32 x 64 B chunk: 16-byte unit i of row r sits at unit i ^ ((r >> 1) & 3)
   const uint32_t swz = static_cast<uint32_t>((lane >> 1) & 3);
 #pragma unroll 1
@@ -101,26 +177,7 @@ __device__ __forceinline__ bool epi_tile(uint32_t t_row, int nch, int n0, int ro
         tma_load_2d(rbuf + b * kChunkBytes, tm_r, &rbar[b], n0 + (c + 2) * 32, row0);
       }
     }
-    // the staging slot is free once the store issued from it two chunks ago has read it
-    if (lane == 0) bulk_wait_group_read<1>();
-    __syncwarp();
-    uint8_t* orow = obuf + out_slot * kChunkBytes + lane * 64;
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      uint4 o;
-      o.x = pack_bf16x2(v[q * 8 + 0], v[q * 8 + 1]);
-      o.y = pack_bf16x2(v[q * 8 + 2], v[q * 8 + 3]);
-      o.z = pack_bf16x2(v[q * 8 + 4], v[q * 8 + 5]);
-      o.w = pack_bf16x2(v[q * 8 + 6], v[q * 8 + 7]);
-      *reinterpret_cast<uint4*>(orow + ((q ^ swz) << 4)) = o;
-    }
-    fence_proxy_async_smem();
-    __syncwarp();
-    if (lane == 0) {
-      tma_store_2d(tm_y, obuf + out_slot * kChunkBytes, n0 + c * 32, row0);
-      bulk_commit_group();
-    }
-    out_slot ^= 1;
+    epi_emit(v, n0 + c * 32, row0, tm_y, obuf, out_slot, lane);
   }
   return true;
 }
@@ -129,7 +186,7 @@ template <int BN>
 __global__ void __launch_bounds__(kThreads, 1)
     linear_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w,
                   const __grid_constant__ CUtensorMap tm_y, const __grid_constant__ CUtensorMap tm_r,
-                  bool has_residual, int M, int N, int K, uint64_t wait_ns, uint32_t* err) {
+                  bool has_residual, int M, int N, int K, uint64_t wait_ns, uint32_t* err, const RopeArgs rope) {
   using C = LinearCfg<BN>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -274,7 +331,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t t_row =
             tmem + (static_cast<uint32_t>(quarter * 32) << 16) + static_cast<uint32_t>(acc * BN);
         ok = epi_tile(t_row, nch, n0, row0, has_residual, &tm_y, &tm_r, obuf, rbuf, rbar, rphase, out_slot, lane,
-                      wait_ns);
+                      wait_ns, rope);
       }
       if (!ok || *abort_flag) {
         if (lane == 0) record_error(err, kErrTimeout | kSiteLinear);
@@ -323,7 +380,7 @@ template <int BN>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     linear_pair_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w,
                        const __grid_constant__ CUtensorMap tm_y, const __grid_constant__ CUtensorMap tm_r,
-                       bool has_residual, int M, int N, int K, uint64_t wait_ns, uint32_t* err) {
+                       bool has_residual, int M, int N, int K, uint64_t wait_ns, uint32_t* err, const RopeArgs rope) {
   using C = Linear2Cfg<BN>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -475,7 +532,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         const uint32_t t_row =
             tmem + (static_cast<uint32_t>(quarter * 32) << 16) + static_cast<uint32_t>(acc) * C::ACC_STRIDE;
         ok = epi_tile(t_row, nch, n0, row0, has_residual, &tm_y, &tm_r, obuf, rbuf, rbar, rphase, out_slot, lane,
-                      wait_ns);
+                      wait_ns, rope);
       }
       if (!ok || *abort_flag) {
         if (lane == 0) record_error(err, kErrTimeout | kSiteLinear);
@@ -593,7 +650,7 @@ kalm_status make_operand_maps(CUtensorMap* tx, CUtensorMap* tw, CUtensorMap* ty,
 template <int BN>
 kalm_status launch_pair(const kalm_bf16* x, int64_t ldx, const kalm_bf16* w, int64_t ldw, const kalm_bf16* residual,
                         int64_t ldr, kalm_bf16* y, int64_t ldy, int64_t m, int32_t n, int32_t k, int slots,
-                        cudaStream_t stream) {
+                        cudaStream_t stream, const RopeArgs& rope) {
   CUtensorMap tx, tw, ty, tr;
   kalm_status st = make_operand_maps(&tx, &tw, &ty, &tr, x, ldx, w, ldw, residual, ldr, y, ldy, m, n, k, BN / 2);
   if (st != KALM_OK) return st;
@@ -601,7 +658,7 @@ kalm_status launch_pair(const kalm_bf16* x, int64_t ldx, const kalm_bf16* w, int
   const int pairs = static_cast<int>(tiles < slots ? tiles : slots);
   return check_cuda(launch_pdl(linear_pair_kernel<BN>, dim3(2 * pairs), dim3(kThreads), Linear2Cfg<BN>::SMEM,
                                 stream, tx, tw, ty, tr, residual != nullptr, (int)m, n, k, kWaitNs,
-                                device_error_word()),
+                                device_error_word(), rope),
                     "launch linear_pair_kernel");
 }
 
@@ -610,7 +667,7 @@ kalm_status launch_pair(const kalm_bf16* x, int64_t ldx, const kalm_bf16* w, int
 // Shared by kalm_linear and kalm_cross_kv_proj.
 kalm_status launch_linear(const kalm_bf16* x, int64_t ldx, const kalm_bf16* w, int64_t ldw, const kalm_bf16* residual,
                           int64_t ldr, kalm_bf16* y, int64_t ldy, int64_t m, int32_t n, int32_t k,
-                          cudaStream_t stream, const char* who) {
+                          cudaStream_t stream, const char* who, const RopeArgs& rope = RopeArgs{}) {
   if (m < 0 || n <= 0 || k <= 0) return fail(KALM_ERR_INVALID_ARG, "%s: m=%lld n=%d k=%d", who, (long long)m, n, k);
   if (m == 0) return KALM_OK;
   if (m > INT32_MAX - 512) return fail(KALM_ERR_INVALID_ARG, "%s: m=%lld too large", who, (long long)m);
@@ -622,7 +679,11 @@ kalm_status launch_linear(const kalm_bf16* x, int64_t ldx, const kalm_bf16* w, i
     return fail(KALM_ERR_INVALID_ARG, "%s: strides must be multiples of 8 and >= the row width", who);
   if (!aligned16(x) || !aligned16(w) || !aligned16(y) || (residual && !aligned16(residual)))
     return fail(KALM_ERR_INVALID_ARG, "%s: bf16 pointers must be 16-byte aligned", who);
-  if (m >= 2 * kBM && n >= 128) {
+  if (rope.rot_cols > 0 && m >= 2 * kBM) {
+    // rotated heads need one head per tile: 256-column pair tiles
+    return launch_pair<256>(x, ldx, w, ldw, residual, ldr, y, ldy, m, n, k, pair_slots(0), stream, rope);
+  }
+  if (m >= 2 * kBM && n >= 128 && rope.rot_cols == 0) {
     // CTA-pair tiles of 256 x BN.  Time ~ rounds of co-resident pairs x (BN + fixed
     // per-tile cost); the fixed cost, measured at the Nano projection shapes, is worth
     // ~480 columns, so narrower tiles pay off only when they save a round.
@@ -640,9 +701,9 @@ kalm_status launch_linear(const kalm_bf16* x, int64_t ldx, const kalm_bf16* w, i
       }
     }
     const int slots = pair_slots(best);
-    if (best == 0) return launch_pair<256>(x, ldx, w, ldw, residual, ldr, y, ldy, m, n, k, slots, stream);
-    if (best == 1) return launch_pair<192>(x, ldx, w, ldw, residual, ldr, y, ldy, m, n, k, slots, stream);
-    return launch_pair<160>(x, ldx, w, ldw, residual, ldr, y, ldy, m, n, k, slots, stream);
+    if (best == 0) return launch_pair<256>(x, ldx, w, ldw, residual, ldr, y, ldy, m, n, k, slots, stream, rope);
+    if (best == 1) return launch_pair<192>(x, ldx, w, ldw, residual, ldr, y, ldy, m, n, k, slots, stream, rope);
+    return launch_pair<160>(x, ldx, w, ldw, residual, ldr, y, ldy, m, n, k, slots, stream, rope);
   }
   const bool wide = (n % 256) == 0;
   const int BN = wide ? 256 : 128;
@@ -654,9 +715,9 @@ kalm_status launch_linear(const kalm_bf16* x, int64_t ldx, const kalm_bf16* w, i
   const bool has_r = residual != nullptr;
   const cudaError_t ce =
       wide ? launch_pdl(linear_kernel<256>, dim3(grid), dim3(kThreads), LinearCfg<256>::SMEM, stream, tx, tw, ty, tr,
-                        has_r, (int)m, n, k, kWaitNs, device_error_word())
+                        has_r, (int)m, n, k, kWaitNs, device_error_word(), rope)
            : launch_pdl(linear_kernel<128>, dim3(grid), dim3(kThreads), LinearCfg<128>::SMEM, stream, tx, tw, ty, tr,
-                        has_r, (int)m, n, k, kWaitNs, device_error_word());
+                        has_r, (int)m, n, k, kWaitNs, device_error_word(), rope);
   return check_cuda(ce, "launch linear_kernel");
 }
 
@@ -684,4 +745,22 @@ extern "C" kalm_status kalm_cross_kv_proj(const kalm_bf16* pooled, int64_t poole
   if (n > INT32_MAX) return fail(KALM_ERR_INVALID_ARG, "kalm_cross_kv_proj: output width too large");
   return launch_linear(pooled, pooled_ld, w_kv, hidden, nullptr, 0, kv_cross, n, total_pooled,
                        static_cast<int32_t>(n), hidden, static_cast<cudaStream_t>(stream), "kalm_cross_kv_proj");
+}
+
+extern "C" kalm_status kalm_linear_rope(const kalm_bf16* x, int64_t ldx, const kalm_bf16* w, int64_t ldw, kalm_bf16* y,
+                                        int64_t ldy, int64_t m, int32_t n, int32_t k, int32_t rot_cols,
+                                        int32_t head_dim, const int64_t* q_off, int32_t n_docs, float theta,
+                                        kalm_stream_t stream) {
+  kalm_status st = ensure_device(nullptr);
+  if (st != KALM_OK) return st;
+  if (head_dim != 256) return fail(KALM_ERR_UNSUPPORTED, "kalm_linear_rope: head_dim=%d (only 256)", head_dim);
+  if (n % 256) return fail(KALM_ERR_UNSUPPORTED, "kalm_linear_rope: n=%d must be a multiple of 256", n);
+  if (rot_cols <= 0 || rot_cols % head_dim || rot_cols > n)
+    return fail(KALM_ERR_INVALID_ARG, "kalm_linear_rope: rot_cols=%d must be a positive multiple of %d <= n=%d",
+                rot_cols, head_dim, n);
+  if (!(theta > 1.f) || !std::isfinite(theta)) return fail(KALM_ERR_INVALID_ARG, "kalm_linear_rope: theta must be > 1");
+  if (n_docs <= 0 || !q_off) return fail(KALM_ERR_INVALID_ARG, "kalm_linear_rope: q_off/n_docs required");
+  RopeArgs rope{q_off, n_docs, rot_cols, log2f(theta), 2.0f / static_cast<float>(head_dim), m, device_error_word()};
+  return launch_linear(x, ldx, w, ldw, nullptr, 0, y, ldy, m, n, k, static_cast<cudaStream_t>(stream),
+                       "kalm_linear_rope", rope);
 }

@@ -22,21 +22,6 @@ namespace {
 
 constexpr int kThreads = 256;
 
-// sin and cos of an angle in [0, 512 rad]: Cody-Waite reduction by 2*pi (W. J. Cody
-// and W. Waite, "Software Manual for the Elementary Functions", 1980) with 2*pi
-// split into a short head (8 significant bits, so k * head is exact for k < 2^15)
-// and a tail, then the hardware approximation on |r| <= pi.  Error stays near
-// 1e-6 rad, far below one bf16 step of the rotated values.
-__device__ __forceinline__ void sincos_reduced(float a, float* s, float* c) {
-  constexpr float kTwoPiHead = 6.28125f;                  // 201/32
-  constexpr float kTwoPiTail = 1.935307179586232e-3f;     // 2*pi - 201/32
-  constexpr float kInvTwoPi = 0.15915494309189535f;
-  const float k = rintf(a * kInvTwoPi);
-  float r = fmaf(-k, kTwoPiHead, a);
-  r = fmaf(-k, kTwoPiTail, r);
-  __sincosf(r, s, c);
-}
-
 __global__ void __launch_bounds__(kThreads) rope_kernel(uint4* __restrict__ x, int64_t ldx_v, int64_t rows,
                                                         int n_heads, int half_v, const int64_t* __restrict__ q_off,
                                                         int n_docs, float log2_theta, float inv_half_d,
@@ -71,12 +56,11 @@ __global__ void __launch_bounds__(kThreads) rope_kernel(uint4* __restrict__ x, i
       const float2 a = __bfloat1622float2(a2[k]);
       const float2 b = __bfloat1622float2(b2[k]);
       const int p0 = g * 8 + 2 * k;  // pair index of the first element
-      float s0, c0, s1, c1;
-      // theta^(-2p/D) = 2^(-(p / (D/2)) log2 theta)
-      sincos_reduced(pos * exp2f(-static_cast<float>(p0) * inv_half_d * log2_theta), &s0, &c0);
-      sincos_reduced(pos * exp2f(-static_cast<float>(p0 + 1) * inv_half_d * log2_theta), &s1, &c1);
-      a2[k] = __floats2bfloat162_rn(a.x * c0 - b.x * s0, a.y * c1 - b.y * s1);
-      b2[k] = __floats2bfloat162_rn(b.x * c0 + a.x * s0, b.y * c1 + a.y * s1);
+      float ra0, rb0, ra1, rb1;
+      rope_pair(pos, p0, inv_half_d, log2_theta, a.x, b.x, &ra0, &rb0);
+      rope_pair(pos, p0 + 1, inv_half_d, log2_theta, a.y, b.y, &ra1, &rb1);
+      a2[k] = __floats2bfloat162_rn(ra0, ra1);
+      b2[k] = __floats2bfloat162_rn(rb0, rb1);
     }
     base[g] = va;
     base[g + half_v] = vb;

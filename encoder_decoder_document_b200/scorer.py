@@ -26,7 +26,7 @@ import torch
 
 from . import (kalm_broadcast_rows, kalm_chunk_pool, kalm_cross_kv_proj, kalm_device_check, kalm_linear,
                kalm_merged_attention, kalm_ragged_offsets, kalm_yes_no_score, kalm_attention_items,
-               kalm_attention_schedule, kalm_rope)
+               kalm_attention_schedule, kalm_linear_rope)
 
 HEAD_DIM = 256
 
@@ -154,15 +154,17 @@ class FBNLScorer:
         D, nq, nkv = self.D, self.n_q, self.n_kv
         return (self.qkv[:, : nq * D], self.qkv[:, nq * D:(nq + nkv) * D], self.qkv[:, (nq + nkv) * D:])
 
-    def rope(self, qkv: torch.Tensor, q_off: torch.Tensor) -> None:
-        if self.rope_theta is not None:
-            kalm_rope(qkv, q_off, self.n_q + self.n_kv, self.rope_theta, self.D)
-            self._mark("rope")
+    def qkv_proj(self, x: torch.Tensor, l: int, qkv: torch.Tensor, q_off: torch.Tensor) -> None:
+        """Fused Q|K|V projection; with a rotary base the self Q and K heads are
+        rotated in the projection's epilogue."""
+        if self.rope_theta is None:
+            kalm_linear(x, self.w.w_qkv[l], qkv)
+        else:
+            kalm_linear_rope(x, self.w.w_qkv[l], qkv, q_off, self.n_q + self.n_kv, self.rope_theta, self.D)
+        self._mark("qkv_proj")
 
     def layer_qkv(self, l: int) -> None:
-        kalm_linear(self.x, self.w.w_qkv[l], self.qkv)
-        self._mark("qkv_proj")
-        self.rope(self.qkv, self.q_off)
+        self.qkv_proj(self.x, l, self.qkv, self.q_off)
 
     def layer_attention(self, l: int) -> None:
         q, ks, vs = self.qkv_views()
@@ -187,9 +189,7 @@ class FBNLScorer:
         kc, vc = self.cross_views(l)
         if first:
             # every document's decoder input is the query's common input: one Q|K|V for all
-            kalm_linear(self.x0, self.w.w_qkv[l], self.qkv[:Lq])
-            self._mark("qkv_proj")
-            self.rope(self.qkv[:Lq], self.one_doc_off)
+            self.qkv_proj(self.x0, l, self.qkv[:Lq], self.one_doc_off)
             q, ks, vs = (t[:Lq] for t in self.qkv_views())
             in_off = self.zero_off
         else:

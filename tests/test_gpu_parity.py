@@ -720,3 +720,57 @@ def test_end_to_end_tiny_with_rope(kalm):
     # and the rotation matters: without it the scores differ
     y0, n0, m0, s0 = oracle.forward_query(q)
     assert np.abs(m0 - m).max() > 1e-3
+
+
+@pytest.mark.parametrize("lq,rot_heads", [([128], 5), ([1, 2, 31, 129, 512, 64, 300], 5), ([7, 250, 19], 2)])
+def test_linear_rope_fused(kalm, lq, rot_heads):
+    """The projection with the rotation in its epilogue is bit-identical to the
+    projection followed by the rotation kernel, and matches the oracle's rotation
+    of the bf16 projection (single-CTA path at 128 rows, CTA-pair path with a
+    ragged tail above)."""
+    rng = np.random.default_rng(sum(lq) + rot_heads)
+    D, n, k = 256, 6 * 256, 1024
+    lq = np.asarray(lq, np.int64)
+    q_off = np.concatenate([[0], np.cumsum(lq)])
+    m, R = int(q_off[-1]), rot_heads * D
+    x = rand_bf16(rng, (m, k))
+    w = rand_bf16(rng, (n, k), 0.02)
+    xd, wd, qd = f64_to_dev(x), f64_to_dev(w), i64(q_off)
+    fused = torch.full((m, n), float("nan"), dtype=torch.bfloat16, device="cuda")
+    kalm.kalm_linear_rope(xd, wd, fused, qd, rot_heads, 1e4)
+    plain = torch.full((m, n), float("nan"), dtype=torch.bfloat16, device="cuda")
+    kalm.kalm_linear(xd, wd, plain)
+    two = plain.clone()
+    kalm.kalm_rope(two, qd, rot_heads, 1e4)
+    kalm.kalm_check_device_errors()
+    assert torch.equal(fused.view(torch.int16), two.view(torch.int16))
+    proj = from_dev(plain)
+    _one_step(proj, oracle.linear(x, w), x, w, None)
+    got = from_dev(fused)
+    pos = np.concatenate([np.arange(v) for v in lq])
+    qk = proj[:, :R].reshape(m, rot_heads, D)
+    want = oracle.apply_rope(qk, pos, 1e4).reshape(m, -1)
+    a, b = qk[..., : D // 2], qk[..., D // 2:]
+    mag = np.concatenate([np.abs(a) + np.abs(b)] * 2, axis=-1).reshape(m, -1)
+    assert (np.abs(got[:, :R] - want) <= _bf16_ulp(want) + 1e-4 * mag).all()
+    np.testing.assert_array_equal(got[:, R:], proj[:, R:])
+
+
+def test_linear_rope_checks(kalm):
+    """Unsupported shapes are refused on the host; a row whose position is past the
+    query limit is flagged on the device."""
+    from encoder_decoder_document_b200 import KalmError
+    rng = np.random.default_rng(83)
+    x = f64_to_dev(rand_bf16(rng, (600, 256)))
+    w = f64_to_dev(rand_bf16(rng, (512, 256), 0.02))
+    y = torch.empty(600, 512, dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(KalmError):
+        kalm.kalm_linear_rope(x, w, y, i64(np.array([0, 600])), 3, 1e4)   # 3 heads > 512 columns
+    with pytest.raises(KalmError):
+        kalm.kalm_linear_rope(x, w[:384], y[:, :384], i64(np.array([0, 600])), 1, 1e4)  # n % 256
+    with pytest.raises(KalmError):
+        kalm.kalm_linear_rope(x, w, y, i64(np.array([0, 600])), 1, 0.5)   # theta <= 1
+    kalm.kalm_linear_rope(x, w, y, i64(np.array([0, 600])), 1, 1e4)      # positions up to 599
+    with pytest.raises(KalmError) as e:
+        kalm.kalm_check_device_errors()
+    assert e.value.name == "KALM_ERR_DEVICE_ARG"
