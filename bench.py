@@ -167,7 +167,7 @@ def rope_alone(sc, theta=1e4, reps=10):
     kernel (bytes read + written, GB/s), and the Q|K|V projection without and with
     the rotation fused into its epilogue."""
     import torch
-    from encoder_decoder_document_b200 import kalm_linear, kalm_linear_rope, kalm_rope
+    from encoder_decoder_document_b200 import kalm_linear, kalm_linear_rope, kalm_rope, kalm_rope_table
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device="cuda")
     heads = sc.n_q + sc.n_kv
     w = sc.w.w_qkv[1]
@@ -187,7 +187,8 @@ def rope_alone(sc, theta=1e4, reps=10):
 
     us = timed(lambda: kalm_rope(sc.qkv, sc.q_off, heads, theta, sc.D))
     plain = timed(lambda: kalm_linear(sc.x, w, sc.qkv))
-    fused = timed(lambda: kalm_linear_rope(sc.x, w, sc.qkv, sc.q_off, heads, theta, sc.D))
+    table = kalm_rope_table(theta, sc.D)
+    fused = timed(lambda: kalm_linear_rope(sc.x, w, sc.qkv, sc.q_off, heads, table, sc.D))
     byts = 2 * sc.qkv.shape[0] * heads * sc.D * 2
     return {"rows": sc.qkv.shape[0], "heads": heads, "theta": theta, "bytes": byts, "us": us,
             "gbs": byts / (us * 1e-6) / 1e9, "qkv_proj_us": plain, "qkv_proj_rope_us": fused,

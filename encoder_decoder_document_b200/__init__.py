@@ -18,10 +18,11 @@ __all__ = [
     "KalmError", "load", "library_path", "kalm_version", "kalm_device_check", "kalm_check_device_errors",
     "kalm_ragged_offsets", "kalm_chunk_pool", "kalm_linear", "kalm_cross_kv_proj", "kalm_merged_attention",
     "kalm_yes_no_score", "kalm_broadcast_rows", "kalm_selftest_wait_timeout", "kalm_attention_items",
-    "kalm_attention_schedule", "kalm_rope", "kalm_linear_rope",
+    "kalm_attention_schedule", "kalm_rope", "kalm_rope_table", "kalm_linear_rope",
 ]
 
 HEAD_DIM = 256
+MAX_QUERY_TOKENS = 512  # KALM_MAX_QUERY_TOKENS
 
 
 def _stream(stream: Optional[torch.cuda.Stream]) -> int:
@@ -153,17 +154,27 @@ def kalm_rope(x: torch.Tensor, q_off: torch.Tensor, n_heads: int, theta: float, 
          q_off.numel() - 1, float(theta), _stream(stream))
 
 
+def kalm_rope_table(theta: float, head_dim: int = HEAD_DIM, stream=None) -> torch.Tensor:
+    """(cos, sin) of every rotary angle: float32 [head_dim/4][KALM_MAX_QUERY_TOKENS][4],
+    entry [q][pos] = (cos, sin) of pair 2q then of pair 2q + 1."""
+    table = torch.empty(head_dim // 4, MAX_QUERY_TOKENS, 4, dtype=torch.float32, device="cuda")
+    call("kalm_rope_table", float(theta), head_dim, _p(table, torch.float32), _stream(stream))
+    return table
+
+
 def kalm_linear_rope(x: torch.Tensor, w: torch.Tensor, y: torch.Tensor, q_off: torch.Tensor, rot_heads: int,
-                     theta: float, head_dim: int = HEAD_DIM, stream=None) -> None:
+                     table: torch.Tensor, head_dim: int = HEAD_DIM, stream=None) -> None:
     """y = x . w^T with the first rot_heads head vectors of every row rotated by the
-    row's decoder position, in the projection's epilogue."""
+    row's decoder position, in the projection's epilogue (angles from kalm_rope_table)."""
     m, k = x.shape
     n = w.shape[0]
     if w.shape[1] != k or y.shape[0] != m or y.shape[1] != n:
         raise KalmError(1, "kalm_linear_rope", f"shapes x{tuple(x.shape)} w{tuple(w.shape)} y{tuple(y.shape)}")
+    if table.numel() != MAX_QUERY_TOKENS * head_dim or not table.is_contiguous():
+        raise KalmError(1, "kalm_linear_rope", "table must be a contiguous kalm_rope_table output")
     call("kalm_linear_rope", _p(x, torch.bfloat16), _ld(x), _p(w, torch.bfloat16), _ld(w), _p(y, torch.bfloat16),
-         _ld(y), m, n, k, rot_heads * head_dim, head_dim, _p(q_off, torch.int64), q_off.numel() - 1, float(theta),
-         _stream(stream))
+         _ld(y), m, n, k, rot_heads * head_dim, head_dim, _p(q_off, torch.int64), q_off.numel() - 1,
+         _p(table, torch.float32), _stream(stream))
 
 
 def kalm_selftest_wait_timeout(wait_ns: int, stream=None) -> None:

@@ -40,7 +40,8 @@ SIGNATURES = {
     "kalm_selftest_wait_timeout": [c_u64, c_vp],
     "kalm_rope": [c_vp, c_i64, c_i64, c_i32, c_i32, c_vp, c_i32, c_f32, c_vp],
     "kalm_linear_rope": [c_vp, c_i64, c_vp, c_i64, c_vp, c_i64, c_i64, c_i32, c_i32, c_i32, c_i32, c_vp, c_i32,
-                         c_f32, c_vp],
+                         c_vp, c_vp],
+    "kalm_rope_table": [c_f32, c_i32, c_vp, c_vp],
 }
 _RESTYPE = {"kalm_version": c_i32, "kalm_attention_items": c_i64, "kalm_status_string": ctypes.c_char_p, "kalm_last_error": ctypes.c_char_p}
 

@@ -372,12 +372,21 @@ __device__ __forceinline__ void sincos_reduced(float a, float* s, float* c) {
 // pos: angle pos * theta^(-2p/head_dim), computed as 2^(-p * (2/head_dim) *
 // log2(theta)); (a, b) -> (a cos - b sin, b cos + a sin) with fixed rounding
 // steps, so every kernel that rotates gets the same bits.
+__device__ __forceinline__ void rope_angle(float pos, int pair, float inv_half_d, float log2_theta, float* sn,
+                                           float* cs) {
+  sincos_reduced(pos * exp2f(-static_cast<float>(pair) * inv_half_d * log2_theta), sn, cs);
+}
+
+__device__ __forceinline__ void rope_turn(float a, float b, float cs, float sn, float* ra, float* rb) {
+  *ra = fmaf(a, cs, __fmul_rn(-b, sn));
+  *rb = fmaf(b, cs, __fmul_rn(a, sn));
+}
+
 __device__ __forceinline__ void rope_pair(float pos, int pair, float inv_half_d, float log2_theta, float a, float b,
                                           float* ra, float* rb) {
   float sn, cs;
-  sincos_reduced(pos * exp2f(-static_cast<float>(pair) * inv_half_d * log2_theta), &sn, &cs);
-  *ra = fmaf(a, cs, __fmul_rn(-b, sn));
-  *rb = fmaf(b, cs, __fmul_rn(a, sn));
+  rope_angle(pos, pair, inv_half_d, log2_theta, &sn, &cs);
+  rope_turn(a, b, cs, sn, ra, rb);
 }
 
 // Pack two fp32 into a bf16x2 word (round to nearest even), low half = a.

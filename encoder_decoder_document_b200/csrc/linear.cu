@@ -6,15 +6,12 @@
 // output projections.
 //
 // Design (sm_100a): a persistent, warp-specialised kernel, one CTA per SM.
-//   warps 0-3   TMA producers: 128 x 64 tiles of x and BN x 64 tiles of w (128-byte
-//               swizzle) into a STAGES-deep shared-memory ring.  A warp's tile
-//               copies are served one after another, so the copies are spread
-//               over four warps (x or w, even or odd k-block) to keep enough of
-//               them in flight;
-//   warp 4      allocates tensor memory and issues tcgen05.mma (M=128, N=BN,
+//   warps 0-1   TMA producers: 128 x 64 tiles of x (warp 0) and BN x 64 tiles of w
+//               (warp 1, 128-byte swizzle) into a STAGES-deep shared-memory ring;
+//   warp 2      allocates tensor memory and issues tcgen05.mma (M=128, N=BN,
 //               K=16 per instruction) from one thread; tcgen05.commit frees a
 //               ring slot once the tensor core has read it;
-//   warps 5..8  epilogue: tcgen05.ld of the fp32 accumulator (one TMEM lane =
+//   warps 3..6  epilogue: tcgen05.ld of the fp32 accumulator (one TMEM lane =
 //               one output row per thread) in 32-column chunks, optional bf16
 //               residual add (the residual chunk is fetched by TMA ahead of
 //               time), one rounding to bf16, then the 32 x 32 chunk is staged in
@@ -23,6 +20,10 @@
 // The accumulator is double-buffered in TMEM (2 x BN columns) so the epilogue
 // of tile i overlaps the main loop of tile i+1.  Out-of-range rows/columns of
 // x and w are zero-filled by TMA; the epilogue masks their stores.
+// With a rotary table (Q|K|V projection) a 256-column tile is one head: the
+// epilogue pairs chunk c with chunk c + 4 and turns them by the row's angles,
+// read from a position-minor table (coalesced across a warp's consecutive rows)
+// one chunk ahead of their use.  Seven warps leave 224 registers a thread for that.
 #include <cmath>
 
 #include "kalm.h"
@@ -34,9 +35,9 @@ namespace {
 
 constexpr int kBM = 128;
 constexpr int kBK = 64;  // one 128-byte swizzle row of bf16
-constexpr int kProdWarps = 4;
-constexpr int kMmaWarp = 4;
-constexpr int kEpiWarp0 = 5;
+constexpr int kProdWarps = 2;  // warp 0 copies x tiles, warp 1 w tiles
+constexpr int kMmaWarp = 2;
+constexpr int kEpiWarp0 = 3;
 constexpr int kThreads = 32 * (kEpiWarp0 + 4);
 
 constexpr int kChunkBytes = 32 * 32 * 2;  // one 32-row x 32-column bf16 epilogue chunk
@@ -69,11 +70,10 @@ __device__ __forceinline__ void epi_prefetch_residual(const CUtensorMap* tm_r, u
 struct RopeArgs {
   const int64_t* q_off;
   int n_docs;
-  int rot_cols;  // 0: no rotation
-  float log2_theta;
-  float inv_half_d;  // 2 / head_dim
-  int64_t rows;      // M: rows past it are clipped by the store
-  uint32_t* err;     // device error word: a stored row whose position is out of range
+  int rot_cols;          // 0: no rotation
+  const float4* table;   // angles: [64][KALM_MAX_QUERY_TOKENS], entry [q][pos] = (cos, sin) of pairs 2q, 2q+1
+  int64_t rows;          // M: rows past it are clipped by the store
+  uint32_t* err;         // device error word: a stored row whose position is out of range
 };
 
 // One 32-column chunk of one warp's 32 rows: bf16 into a 64-byte-swizzled staging
@@ -104,6 +104,34 @@ __device__ __forceinline__ void epi_emit(const float (&v)[32], int col, int row0
   out_slot ^= 1;
 }
 
+// Row of the angle table for this lane's row of a tile whose columns are rotated
+// heads, or -1 when the tile is not rotated.  Called before the accumulator wait,
+// so the offsets search overlaps the tile's MMAs.  A row past the last document
+// (clipped by the store) reads position 0; a stored row whose position is out of
+// range is flagged.
+__device__ __forceinline__ int rope_row(const RopeArgs& rope, int n0, int nch, int row0, int lane) {
+  if (!(n0 < rope.rot_cols && nch == 8)) return -1;
+  const int64_t m = row0 + lane;
+  int lo = 0, hi = rope.n_docs - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (__ldg(rope.q_off + mid) <= m) lo = mid; else hi = mid - 1;
+  }
+  const int64_t pos64 = m - __ldg(rope.q_off + lo);
+  const bool in_range = pos64 >= 0 && pos64 < KALM_MAX_QUERY_TOKENS;
+  if (m < rope.rows && !in_range) record_error(rope.err, kErrDeviceArg | kSiteRope);
+  return in_range ? static_cast<int>(pos64) : 0;
+}
+
+// The first 32 pairs' angles of a rotated tile's row, loaded before the
+// accumulator wait so that their latency hides behind the tile's MMAs.
+__device__ __forceinline__ void rope_prefetch(const RopeArgs& rope, int rope_pos, float4 (&cs)[16]) {
+  if (rope_pos >= 0) {
+#pragma unroll
+    for (int j = 0; j < 16; ++j) cs[j] = __ldg(rope.table + j * KALM_MAX_QUERY_TOKENS + rope_pos);
+  }
+}
+
 // Epilogue of one tile for one warp: 32 rows (TMEM lanes of this warp) x nch
 // 32-column chunks.  fp32 accumulator (+ residual) -> bf16 -> swizzled staging
 // chunk -> TMA tile store.  A tile of rotated heads pairs chunk c with chunk c + 4
@@ -113,34 +141,34 @@ __device__ __forceinline__ void epi_emit(const float (&v)[32], int col, int row0
 __device__ __forceinline__ bool epi_tile(uint32_t t_row, int nch, int n0, int row0, bool has_residual,
                                          const CUtensorMap* tm_y, const CUtensorMap* tm_r, uint8_t* obuf,
                                          uint8_t* rbuf, uint64_t* rbar, uint32_t& rphase, int& out_slot, int lane,
-                                         uint64_t wait_ns, const RopeArgs& rope) {
-  if (n0 < rope.rot_cols && nch == 8) {
-    // decoder position of this lane's row
-    const int64_t m = row0 + lane;
-    int lo = 0, hi = rope.n_docs - 1;
-    while (lo < hi) {
-      const int mid = (lo + hi + 1) >> 1;
-      if (__ldg(rope.q_off + mid) <= m) lo = mid; else hi = mid - 1;
-    }
-    const int64_t pos64 = m - __ldg(rope.q_off + lo);
-    if (m < rope.rows && (pos64 < 0 || pos64 >= KALM_MAX_QUERY_TOKENS))
-      record_error(rope.err, kErrDeviceArg | kSiteRope);
-    const float pos = static_cast<float>(pos64);
+                                         uint64_t wait_ns, const RopeArgs& rope, int rope_pos, float4 (&cs)[16]) {
+  if (rope_pos >= 0) {
+    const float4* tcol = rope.table + rope_pos;  // lanes at consecutive positions read consecutive entries
 #pragma unroll 1
     for (int c = 0; c < 4; ++c) {
       uint32_t ra[32], rb[32];
       tmem_ld32(t_row + c * 32, ra);
       tmem_ld32(t_row + (c + 4) * 32, rb);
+      float4 nx[16];  // the next chunk's angles, in flight while this chunk is turned
+      if (c < 3) {
+#pragma unroll
+        for (int j = 0; j < 16; ++j) nx[j] = __ldg(tcol + ((c + 1) * 16 + j) * KALM_MAX_QUERY_TOKENS);
+      }
       tmem_ld_wait();
       float va[32], vb[32];
 #pragma unroll
-      for (int j = 0; j < 32; ++j) {
-        const float a = __bfloat162float(__float2bfloat16_rn(__uint_as_float(ra[j])));
-        const float b = __bfloat162float(__float2bfloat16_rn(__uint_as_float(rb[j])));
-        rope_pair(pos, c * 32 + j, rope.inv_half_d, rope.log2_theta, a, b, &va[j], &vb[j]);
+      for (int j = 0; j < 16; ++j) {
+        const float a0 = __bfloat162float(__float2bfloat16_rn(__uint_as_float(ra[2 * j])));
+        const float b0 = __bfloat162float(__float2bfloat16_rn(__uint_as_float(rb[2 * j])));
+        const float a1 = __bfloat162float(__float2bfloat16_rn(__uint_as_float(ra[2 * j + 1])));
+        const float b1 = __bfloat162float(__float2bfloat16_rn(__uint_as_float(rb[2 * j + 1])));
+        rope_turn(a0, b0, cs[j].x, cs[j].y, &va[2 * j], &vb[2 * j]);
+        rope_turn(a1, b1, cs[j].z, cs[j].w, &va[2 * j + 1], &vb[2 * j + 1]);
       }
       epi_emit(va, n0 + c * 32, row0, tm_y, obuf, out_slot, lane);
       epi_emit(vb, n0 + (c + 4) * 32, row0, tm_y, obuf, out_slot, lane);
+#pragma unroll
+      for (int j = 0; j < 16; ++j) cs[j] = nx[j];
     }
     return true;
   }
@@ -234,29 +262,25 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp < kProdWarps) {
     if (lane == 0) {
-      const bool is_w = warp >= 2;      // which operand this warp copies
-      const uint32_t mine = warp & 1;   // which k-blocks (by parity of the running count)
+      const bool is_w = warp == 1;  // which operand this warp copies
       const CUtensorMap* tm = is_w ? &tm_w : &tm_x;
       tma_prefetch_desc(tm);
       int stage = 0;
       uint32_t phase = 0;
-      uint32_t it = 0;
       for (int t = blockIdx.x; t < tiles && !*abort_flag; t += gridDim.x) {
         const int m0 = (t / n_n) * kBM, n0 = (t % n_n) * BN;
-        for (int kb = 0; kb < kblocks; ++kb, ++it) {
-          if ((it & 1u) == mine) {
-            if (!mbar_wait(&empty[stage], phase ^ 1u, wait_ns)) {
-              record_error(err, kErrTimeout | kSiteLinear);
-              *abort_flag = 1;
-              break;
-            }
-            if (is_w) {
-              mbar_arrive_expect_tx(&full[stage], C::B_BYTES);
-              tma_load_2d(sB + stage * C::B_BYTES, tm, &full[stage], kb * kBK, n0);
-            } else {
-              mbar_arrive_expect_tx(&full[stage], C::A_BYTES);
-              tma_load_2d(sA + stage * C::A_BYTES, tm, &full[stage], kb * kBK, m0);
-            }
+        for (int kb = 0; kb < kblocks; ++kb) {
+          if (!mbar_wait(&empty[stage], phase ^ 1u, wait_ns)) {
+            record_error(err, kErrTimeout | kSiteLinear);
+            *abort_flag = 1;
+            break;
+          }
+          if (is_w) {
+            mbar_arrive_expect_tx(&full[stage], C::B_BYTES);
+            tma_load_2d(sB + stage * C::B_BYTES, tm, &full[stage], kb * kBK, n0);
+          } else {
+            mbar_arrive_expect_tx(&full[stage], C::A_BYTES);
+            tma_load_2d(sA + stage * C::A_BYTES, tm, &full[stage], kb * kBK, m0);
           }
           if (++stage == C::STAGES) {
             stage = 0;
@@ -309,7 +333,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
   } else {
-    // epilogue warps 5..8: warp w may access TMEM lanes 32*(w%4) .. 32*(w%4)+31
+    // epilogue warps 3..6: warp w may access TMEM lanes 32*(w%4) .. 32*(w%4)+31
     const int quarter = warp & 3;
     const int ew = warp - kEpiWarp0;
     uint8_t* obuf = sOut + ew * 2 * kChunkBytes;
@@ -324,6 +348,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int row0 = m0 + quarter * 32;
       const int nch = min(BN, N - n0) / 32;
       if (has_residual && lane == 0) epi_prefetch_residual(&tm_r, rbuf, rbar, nch, n0, row0);
+      const int rpos = rope_row(rope, n0, nch, row0, lane);
+      float4 cs[16];
+      rope_prefetch(rope, rpos, cs);
       bool ok = mbar_wait(&acc_full[acc], acc_phase, wait_ns);
       ok = __all_sync(0xffffffffu, ok);
       if (ok && !*abort_flag) {
@@ -331,7 +358,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t t_row =
             tmem + (static_cast<uint32_t>(quarter * 32) << 16) + static_cast<uint32_t>(acc * BN);
         ok = epi_tile(t_row, nch, n0, row0, has_residual, &tm_y, &tm_r, obuf, rbuf, rbar, rphase, out_slot, lane,
-                      wait_ns, rope);
+                      wait_ns, rope, rpos, cs);
       }
       if (!ok || *abort_flag) {
         if (lane == 0) record_error(err, kErrTimeout | kSiteLinear);
@@ -431,32 +458,28 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 
   if (warp < kProdWarps) {
     if (lane == 0) {
-      const bool is_w = warp >= 2;
-      const uint32_t mine = warp & 1;
+      const bool is_w = warp == 1;
       const CUtensorMap* tm = is_w ? &tm_w : &tm_x;
       tma_prefetch_desc(tm);
       const uint32_t full0 = map_to_rank(smem_u32(full), 0);  // the even CTA's full barriers
       int stage = 0;
       uint32_t phase = 0;
-      uint32_t it = 0;
       for (int t = pair; t < tiles && !*abort_flag; t += n_pairs) {
         const int m0 = (t / n_n) * 2 * kBM + static_cast<int>(rank) * kBM;
         const int n0 = (t % n_n) * BN + static_cast<int>(rank) * C::BNH;
-        for (int kb = 0; kb < kblocks; ++kb, ++it) {
-          if ((it & 1u) == mine) {
-            if (!mbar_wait(&empty[stage], phase ^ 1u, wait_ns)) {
-              record_error(err, kErrTimeout | kSiteLinear);
-              *abort_flag = 1;
-              break;
-            }
-            const uint32_t bar = full0 + stage * 8;
-            if (is_w) {
-              if (leader) mbar_arrive_expect_tx(&full[stage], 2 * C::B_BYTES);
-              tma_load_2d_pair(sB + stage * C::B_BYTES, tm, bar, kb * kBK, n0);
-            } else {
-              if (leader) mbar_arrive_expect_tx(&full[stage], 2 * C::A_BYTES);
-              tma_load_2d_pair(sA + stage * C::A_BYTES, tm, bar, kb * kBK, m0);
-            }
+        for (int kb = 0; kb < kblocks; ++kb) {
+          if (!mbar_wait(&empty[stage], phase ^ 1u, wait_ns)) {
+            record_error(err, kErrTimeout | kSiteLinear);
+            *abort_flag = 1;
+            break;
+          }
+          const uint32_t bar = full0 + stage * 8;
+          if (is_w) {
+            if (leader) mbar_arrive_expect_tx(&full[stage], 2 * C::B_BYTES);
+            tma_load_2d_pair(sB + stage * C::B_BYTES, tm, bar, kb * kBK, n0);
+          } else {
+            if (leader) mbar_arrive_expect_tx(&full[stage], 2 * C::A_BYTES);
+            tma_load_2d_pair(sA + stage * C::A_BYTES, tm, bar, kb * kBK, m0);
           }
           if (++stage == C::STAGES) {
             stage = 0;
@@ -525,6 +548,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       const int row0 = m0 + quarter * 32;
       const int nch = min(BN, N - n0) / 32;
       if (has_residual && lane == 0) epi_prefetch_residual(&tm_r, rbuf, rbar, nch, n0, row0);
+      const int rpos = rope_row(rope, n0, nch, row0, lane);
+      float4 cs[16];
+      rope_prefetch(rope, rpos, cs);
       bool ok = mbar_wait(&acc_full[acc], acc_phase, wait_ns);
       ok = __all_sync(0xffffffffu, ok);
       if (ok && !*abort_flag) {
@@ -532,7 +558,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         const uint32_t t_row =
             tmem + (static_cast<uint32_t>(quarter * 32) << 16) + static_cast<uint32_t>(acc) * C::ACC_STRIDE;
         ok = epi_tile(t_row, nch, n0, row0, has_residual, &tm_y, &tm_r, obuf, rbuf, rbar, rphase, out_slot, lane,
-                      wait_ns, rope);
+                      wait_ns, rope, rpos, cs);
       }
       if (!ok || *abort_flag) {
         if (lane == 0) record_error(err, kErrTimeout | kSiteLinear);
@@ -749,7 +775,7 @@ extern "C" kalm_status kalm_cross_kv_proj(const kalm_bf16* pooled, int64_t poole
 
 extern "C" kalm_status kalm_linear_rope(const kalm_bf16* x, int64_t ldx, const kalm_bf16* w, int64_t ldw, kalm_bf16* y,
                                         int64_t ldy, int64_t m, int32_t n, int32_t k, int32_t rot_cols,
-                                        int32_t head_dim, const int64_t* q_off, int32_t n_docs, float theta,
+                                        int32_t head_dim, const int64_t* q_off, int32_t n_docs, const float* table,
                                         kalm_stream_t stream) {
   kalm_status st = ensure_device(nullptr);
   if (st != KALM_OK) return st;
@@ -758,9 +784,10 @@ extern "C" kalm_status kalm_linear_rope(const kalm_bf16* x, int64_t ldx, const k
   if (rot_cols <= 0 || rot_cols % head_dim || rot_cols > n)
     return fail(KALM_ERR_INVALID_ARG, "kalm_linear_rope: rot_cols=%d must be a positive multiple of %d <= n=%d",
                 rot_cols, head_dim, n);
-  if (!(theta > 1.f) || !std::isfinite(theta)) return fail(KALM_ERR_INVALID_ARG, "kalm_linear_rope: theta must be > 1");
+  if (!table || !aligned16(table))
+    return fail(KALM_ERR_INVALID_ARG, "kalm_linear_rope: table must be non-NULL and 16-byte aligned");
   if (n_docs <= 0 || !q_off) return fail(KALM_ERR_INVALID_ARG, "kalm_linear_rope: q_off/n_docs required");
-  RopeArgs rope{q_off, n_docs, rot_cols, log2f(theta), 2.0f / static_cast<float>(head_dim), m, device_error_word()};
+  RopeArgs rope{q_off, n_docs, rot_cols, reinterpret_cast<const float4*>(table), m, device_error_word()};
   return launch_linear(x, ldx, w, ldw, nullptr, 0, y, ldy, m, n, k, static_cast<cudaStream_t>(stream),
                        "kalm_linear_rope", rope);
 }

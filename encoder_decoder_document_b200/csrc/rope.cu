@@ -67,6 +67,23 @@ __global__ void __launch_bounds__(kThreads) rope_kernel(uint4* __restrict__ x, i
   }
 }
 
+// Table of (cos, sin) for every decoder position below KALM_MAX_QUERY_TOKENS and
+// every pair of a head, the same values rope_pair computes, so a kernel that looks
+// them up rotates to the same bits.  Layout: float4 [half/2][KALM_MAX_QUERY_TOKENS],
+// entry [q][pos] = (cos, sin) of pair 2q then of pair 2q + 1: threads holding
+// consecutive positions read consecutive 16-byte entries.
+__global__ void __launch_bounds__(kThreads) rope_table_kernel(float2* __restrict__ table, int total,
+                                                              float log2_theta, float inv_half_d) {
+  pdl_launch_dependents();
+  pdl_wait_predecessor();
+  for (int i = blockIdx.x * kThreads + threadIdx.x; i < total; i += gridDim.x * kThreads) {
+    const int p = i / KALM_MAX_QUERY_TOKENS, pos = i - p * KALM_MAX_QUERY_TOKENS;
+    float sn, cs;
+    rope_angle(static_cast<float>(pos), p, inv_half_d, log2_theta, &sn, &cs);
+    table[((p >> 1) * KALM_MAX_QUERY_TOKENS + pos) * 2 + (p & 1)] = make_float2(cs, sn);
+  }
+}
+
 }  // namespace
 }  // namespace kalm
 
@@ -95,4 +112,19 @@ extern "C" kalm_status kalm_rope(kalm_bf16* x, int64_t ldx, int64_t rows, int32_
                                half_v, q_off, n_docs, log2f(theta), 2.0f / static_cast<float>(head_dim),
                                device_error_word()),
                     "launch rope_kernel");
+}
+
+extern "C" kalm_status kalm_rope_table(float theta, int32_t head_dim, float* table, kalm_stream_t stream) {
+  kalm_status st = ensure_device(nullptr);
+  if (st != KALM_OK) return st;
+  if (head_dim <= 0 || head_dim % 16) return fail(KALM_ERR_INVALID_ARG, "kalm_rope_table: head_dim=%d", head_dim);
+  if (!(theta > 1.f) || !std::isfinite(theta)) return fail(KALM_ERR_INVALID_ARG, "kalm_rope_table: theta must be > 1");
+  if (!table || !aligned16(table))
+    return fail(KALM_ERR_INVALID_ARG, "kalm_rope_table: table must be non-NULL and 16-byte aligned");
+  const int half = head_dim / 2, total = KALM_MAX_QUERY_TOKENS * half;
+  const int blocks = (total + kThreads - 1) / kThreads;
+  return check_cuda(launch_pdl(rope_table_kernel, dim3(static_cast<unsigned>(blocks)), dim3(kThreads), 0,
+                               static_cast<cudaStream_t>(stream), reinterpret_cast<float2*>(table), total,
+                               log2f(theta), 2.0f / static_cast<float>(head_dim)),
+                    "launch rope_table_kernel");
 }

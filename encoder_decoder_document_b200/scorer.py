@@ -26,7 +26,7 @@ import torch
 
 from . import (kalm_broadcast_rows, kalm_chunk_pool, kalm_cross_kv_proj, kalm_device_check, kalm_linear,
                kalm_merged_attention, kalm_ragged_offsets, kalm_yes_no_score, kalm_attention_items,
-               kalm_attention_schedule, kalm_linear_rope)
+               kalm_attention_schedule, kalm_linear_rope, kalm_rope_table)
 
 HEAD_DIM = 256
 
@@ -70,6 +70,8 @@ class FBNLScorer:
         self.scale = head_dim ** -0.5
         self.prune = prune
         self.rope_theta = rope_theta  # rotary base for the decoder's self Q/K, or None (no rotation)
+        # the rotary angles' (cos, sin), built once for this base
+        self.rope_tab = kalm_rope_table(rope_theta, head_dim) if rope_theta is not None else None
         self._shape = None
         self.graph: Optional[torch.cuda.CUDAGraph] = None
         self.graphs = None
@@ -160,7 +162,7 @@ class FBNLScorer:
         if self.rope_theta is None:
             kalm_linear(x, self.w.w_qkv[l], qkv)
         else:
-            kalm_linear_rope(x, self.w.w_qkv[l], qkv, q_off, self.n_q + self.n_kv, self.rope_theta, self.D)
+            kalm_linear_rope(x, self.w.w_qkv[l], qkv, q_off, self.n_q + self.n_kv, self.rope_tab, self.D)
         self._mark("qkv_proj")
 
     def layer_qkv(self, l: int) -> None:

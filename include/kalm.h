@@ -275,26 +275,40 @@ kalm_status kalm_broadcast_rows(const kalm_bf16* src, int64_t ld_src, int32_t ro
 kalm_status kalm_rope(kalm_bf16* x, int64_t ldx, int64_t rows, int32_t n_heads, int32_t head_dim,
                       const int64_t* q_off, int32_t n_docs, float theta, kalm_stream_t stream);
 
+/* Table of the rotary angles' cosines and sines, built once per rotary base for
+ * kalm_linear_rope.  Same passage and reading as kalm_rope: the angle of pair p
+ * at position pos is pos * theta^(-2p/head_dim), its cosine and sine computed
+ * exactly as kalm_rope computes them.
+ *
+ * table   float[head_dim/4][KALM_MAX_QUERY_TOKENS][4] device, caller-owned,
+ *         16-byte aligned; entry [q][pos] = (cos, sin) of pair 2q, then
+ *         (cos, sin) of pair 2q + 1 (position-minor, so that consecutive rows
+ *         read consecutive entries).  Written entirely.
+ * theta   rotary base (> 1); head_dim % 16 == 0. */
+kalm_status kalm_rope_table(float theta, int32_t head_dim, float* table, kalm_stream_t stream);
+
 /* The decoder's fused Q|K|V projection with the rotary embedding of its first
  * rot_cols output columns applied in the projection's epilogue: y = x . w^T,
  * then every head vector in columns [0, rot_cols) turns as kalm_rope turns it
- * (same pairing, angle and position rule).  The result is bit-identical to
- * kalm_linear followed by kalm_rope over rot_cols / head_dim heads: the
- * accumulator is rounded to bf16 first, rotated in fp32, rounded again.  Saves
- * the rotation's separate read and write of Q and K_self.  Same passages as
- * kalm_rope for the rotation, as kalm_linear for the product.
+ * (same pairing, angle and position rule), the angles read from a table that
+ * kalm_rope_table built.  The result is bit-identical to kalm_linear followed
+ * by kalm_rope over rot_cols / head_dim heads: the accumulator is rounded to
+ * bf16 first, rotated in fp32, rounded again.  Saves the rotation's separate
+ * read and write of Q and K_self.  Same passages as kalm_rope for the rotation,
+ * as kalm_linear for the product.
  *
  * x, w, y, ldx, ldw, ldy, m, n, k   as kalm_linear (no residual).
  * rot_cols  multiple of head_dim, <= n: the Q heads and self-K heads.
  * head_dim  256 (one head per 256-column output tile).
  * q_off     int64[n_docs+1] device, as kalm_rope (rows [0, m) covered).
- * theta     rotary base (> 1).
+ * table     kalm_rope_table's output for head_dim 256 and the rotary base,
+ *           16-byte aligned; read only.
  * Requirements: those of kalm_linear, and n % 256 == 0.  A row below m whose
  * position falls outside [0, KALM_MAX_QUERY_TOKENS) is flagged in the device
  * error word (its output is then unspecified). */
 kalm_status kalm_linear_rope(const kalm_bf16* x, int64_t ldx, const kalm_bf16* w, int64_t ldw, kalm_bf16* y,
                              int64_t ldy, int64_t m, int32_t n, int32_t k, int32_t rot_cols, int32_t head_dim,
-                             const int64_t* q_off, int32_t n_docs, float theta, kalm_stream_t stream);
+                             const int64_t* q_off, int32_t n_docs, const float* table, kalm_stream_t stream);
 
 /* Failure-detection self-test: one CTA waits on a shared-memory barrier that
  * nothing completes, with a bound of `wait_ns` nanoseconds; on expiry it

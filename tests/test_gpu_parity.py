@@ -722,6 +722,21 @@ def test_end_to_end_tiny_with_rope(kalm):
     assert np.abs(m0 - m).max() > 1e-3
 
 
+@pytest.mark.parametrize("theta", [1e4, 1e6])
+def test_rope_table(kalm, theta):
+    """The angle table holds cos and sin of pos * theta^(-2p/D), and rotating through
+    it equals kalm_rope bit for bit (checked by the fused projection test).  Bound:
+    the fp32 angle at position 511 carries exp2's 2-ulp error (511 * 2.4e-7 =
+    1.2e-4 rad) plus the product's and the exponent's roundings (~5e-5 rad)."""
+    raw = kalm.kalm_rope_table(theta).cpu().numpy().astype(np.float64)   # [64][512][4]
+    tab = raw.reshape(64, 512, 2, 2).transpose(1, 0, 2, 3).reshape(512, 128, 2)   # [pos][pair][cos, sin]
+    pos = np.arange(512)[:, None]
+    ang = pos * oracle.rope_inv_freq(256, theta)[None, :]
+    assert np.abs(tab[..., 0] - np.cos(ang)).max() < 2e-4
+    assert np.abs(tab[..., 1] - np.sin(ang)).max() < 2e-4
+    np.testing.assert_array_equal(tab[0], np.stack([np.ones(128), np.zeros(128)], -1))
+
+
 @pytest.mark.parametrize("lq,rot_heads", [([128], 5), ([1, 2, 31, 129, 512, 64, 300], 5), ([7, 250, 19], 2)])
 def test_linear_rope_fused(kalm, lq, rot_heads):
     """The projection with the rotation in its epilogue is bit-identical to the
@@ -737,7 +752,7 @@ def test_linear_rope_fused(kalm, lq, rot_heads):
     w = rand_bf16(rng, (n, k), 0.02)
     xd, wd, qd = f64_to_dev(x), f64_to_dev(w), i64(q_off)
     fused = torch.full((m, n), float("nan"), dtype=torch.bfloat16, device="cuda")
-    kalm.kalm_linear_rope(xd, wd, fused, qd, rot_heads, 1e4)
+    kalm.kalm_linear_rope(xd, wd, fused, qd, rot_heads, kalm.kalm_rope_table(1e4))
     plain = torch.full((m, n), float("nan"), dtype=torch.bfloat16, device="cuda")
     kalm.kalm_linear(xd, wd, plain)
     two = plain.clone()
@@ -764,13 +779,15 @@ def test_linear_rope_checks(kalm):
     x = f64_to_dev(rand_bf16(rng, (600, 256)))
     w = f64_to_dev(rand_bf16(rng, (512, 256), 0.02))
     y = torch.empty(600, 512, dtype=torch.bfloat16, device="cuda")
+    tab, off = kalm.kalm_rope_table(1e4), i64(np.array([0, 600]))
     with pytest.raises(KalmError):
-        kalm.kalm_linear_rope(x, w, y, i64(np.array([0, 600])), 3, 1e4)   # 3 heads > 512 columns
+        kalm.kalm_linear_rope(x, w, y, off, 3, tab)   # 3 heads > 512 columns
     with pytest.raises(KalmError):
-        kalm.kalm_linear_rope(x, w[:384], y[:, :384], i64(np.array([0, 600])), 1, 1e4)  # n % 256
+        kalm.kalm_linear_rope(x, w[:384], y[:, :384], off, 1, tab)  # n % 256
     with pytest.raises(KalmError):
-        kalm.kalm_linear_rope(x, w, y, i64(np.array([0, 600])), 1, 0.5)   # theta <= 1
-    kalm.kalm_linear_rope(x, w, y, i64(np.array([0, 600])), 1, 1e4)      # positions up to 599
+        kalm.kalm_rope_table(0.5)   # theta <= 1
+    kalm.kalm_check_device_errors()
+    kalm.kalm_linear_rope(x, w, y, off, 1, tab)      # positions up to 599
     with pytest.raises(KalmError) as e:
         kalm.kalm_check_device_errors()
     assert e.value.name == "KALM_ERR_DEVICE_ARG"
