@@ -349,9 +349,9 @@ def test_yes_no_score_extreme_margins(kalm):
 # ---------------------------------------------------------------------------
 # end to end
 # ---------------------------------------------------------------------------
-def _scorer(q, graph=False):
+def _scorer(q, graph=False, rope_theta=None):
     from encoder_decoder_document_b200.scorer import DeviceWeights, FBNLScorer
-    sc = FBNLScorer(DeviceWeights.from_bits(q.weights), q.n_q, q.n_kv)
+    sc = FBNLScorer(DeviceWeights.from_bits(q.weights), q.n_q, q.n_kv, rope_theta=rope_theta)
     if graph:
         doc_len = q.doc_len
         sc.prepare(q.n_docs, int(doc_len.sum()), int(oracle.pooled_counts(doc_len).sum()), q.lq)
@@ -428,6 +428,21 @@ def test_end_to_end_full_size_sampled(kalm, name, docs):
     pooled = from_dev(sc.pooled[: sc.total_pooled])
     want, _ = oracle.chunk_pool(oracle.bf16_bits_to_f64(q.enc), q.tok_off, q.doc_len)
     assert np.abs(pooled - want).max() <= POOL_TOL
+
+
+@pytest.mark.slow
+def test_end_to_end_full_size_with_rope(kalm):
+    """Nano at full size with rotated self Q/K, in the benchmark's launch configuration
+    (CUDA graph, rotation fused into the Q|K|V projection), against the oracle on
+    sampled documents."""
+    q = synthetic.make_query("nano")
+    docs = [2, 58, 93]
+    sc = _scorer(q, graph=True, rope_theta=1e4)
+    kalm.kalm_check_device_errors()
+    res = sc.scores_to_host().numpy()
+    y, n, m, s = oracle.forward_query(q, docs=docs, rope_theta=1e4)
+    assert np.all(np.isfinite(res))
+    _check_scores(res[3][docs], s, m)
 
 
 def _rows(t, q, docs):
