@@ -513,6 +513,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float l_run = (m_ref == -INFINITY) ? 0.f : l_own * ex2_approx(m_ref - m_fin);
       const float m_run = m_fin;
       // ---- epilogue of this item: O / l -> bf16, this half's 128 columns
+      // l_part holds one item: the other group must have read the previous item's sums,
+      // which it does before it loads that item's O (bar_ofree)
+      if (n_it >= 1) {
+        const bool wo = mbar_wait(bar_ofree, (n_it - 1) & 1, p.wait_ns);
+        if (!__all_sync(0xffffffffu, wo)) {
+          ok = false;
+          break;
+        }
+      }
       l_part[half * 128 + r] = l_run;
       mbar_arrive(bar_l);
       bool wt = mbar_wait(&bar_pv[Jl & 1], (Jl >> 1) & 1, p.wait_ns) && mbar_wait(bar_l, n_it & 1, p.wait_ns);
