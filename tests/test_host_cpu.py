@@ -117,3 +117,35 @@ def test_two_rank_document_sharding_gloo():
     np.testing.assert_array_equal(merged, want)
     from encoder_decoder_document_b200.scorer import rank
     assert rank(merged[:, 2], merged[:, 3]) == rank(want[:, 2], want[:, 3])
+
+
+def _bench(args, env_extra=None):
+    import json
+    import os
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    env = dict(os.environ, **(env_extra or {}))
+    res = subprocess.run([sys.executable, os.path.join(root, "bench.py"), *args], capture_output=True, text=True,
+                         cwd=root, env=env, timeout=600)
+    assert res.returncode == 0, res.stderr[-2000:]
+    lines = [l for l in res.stdout.splitlines() if l.startswith("{")]
+    return [json.loads(l) for l in lines]
+
+
+def test_bench_reference_arm_contract():
+    """`bench.py --impl reference` times the oracle on the host cores and prints one
+    JSON line with the contract's keys; ranks other than 0 print nothing."""
+    (line,) = _bench(["--impl", "reference", "--config", "tiny", "--steps", "2", "--warmup", "1"])
+    for k in ("impl", "metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
+              "scaling", "vs_baseline", "dtype", "data", "config", "cpu_baseline", "e2e"):
+        assert k in line, k
+    assert line["impl"] == "reference" and line["steps"] == 2 and line["warmup"] == 1
+    assert line["value"] > 0 and line["higher_is_better"] is True
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] >= 1
+    assert line["cpu_baseline"]["value"] == line["value"]
+    assert line["e2e"] == {"value": line["value"], "unit": line["unit"], "h2d_bytes_per_step": 0,
+                           "d2h_bytes_per_step": 0}
+    assert "workload" in line["config"]
+    assert _bench(["--impl", "reference", "--config", "tiny", "--steps", "1", "--warmup", "0"],
+                  {"RANK": "1", "WORLD_SIZE": "2"}) == []
