@@ -431,6 +431,21 @@ def test_end_to_end_full_size_sampled(kalm, name, docs):
 
 
 @pytest.mark.slow
+def test_end_to_end_sweep_4096_documents_sampled(kalm):
+    """The throughput sweep's largest point (4096 documents, log-normal lengths down to
+    1 token, the sweep's query length) in the benchmark's launch configuration, against
+    the oracle on sampled documents: the shortest, the longest, and both ends."""
+    q = synthetic.make_query("sweep", n_docs=4096, seed=4)
+    docs = sorted({0, int(np.argmin(q.doc_len)), int(np.argmax(q.doc_len)), 4095})
+    sc = _scorer(q, graph=True)
+    kalm.kalm_check_device_errors()
+    res = sc.scores_to_host().numpy()
+    assert np.all(np.isfinite(res))
+    y, n, m, s = oracle.forward_query(q, docs=docs)
+    _check_scores(res[3][docs], s, m)
+
+
+@pytest.mark.slow
 def test_end_to_end_full_size_with_rope(kalm):
     """Nano at full size with rotated self Q/K, in the benchmark's launch configuration
     (CUDA graph, rotation fused into the Q|K|V projection), against the oracle on
