@@ -386,6 +386,19 @@ def test_end_to_end_tiny(kalm):
     assert len(ranked) == 2 and ranked[0]["relevance_score"] >= ranked[1]["relevance_score"]
 
 
+@pytest.mark.parametrize("doc_len", [[0, 5, 0, 64], [0, 0, 0]])
+def test_end_to_end_with_empty_documents(kalm, doc_len):
+    """Documents of length 0 (no pooled vectors: attention over the causal self part
+    only), also when every document of the query is empty, eagerly and in the graph."""
+    q = synthetic.make_query("tiny", doc_len=np.array(doc_len))
+    y, n, m, s = oracle.forward_query(q)
+    for graph in (False, True):
+        sc = _scorer(q, graph=graph)
+        kalm.kalm_check_device_errors()
+        res = sc.scores_to_host().numpy()
+        _check_scores(res[3], s, m)
+
+
 def test_end_to_end_tiny_batch_composition(kalm):
     # a document's score is the same alone and inside the batch (bitwise)
     q = synthetic.make_query("tiny")
