@@ -124,7 +124,8 @@ def _one_step(got, want, x=None, w=None, r=None):
 
 @pytest.mark.parametrize("m,n,k,res", [
     (1, 32, 8, False), (127, 64, 40, False), (300, 640, 640, False), (257, 1536, 640, True),
-    (1000, 512, 1152, True), (129, 2560, 72, False), (4096, 256, 2560, True)])
+    (1000, 512, 1152, True), (129, 2560, 72, False), (4096, 256, 2560, True),
+    (12800, 640, 1024, True)])   # the decoder's output projection at the Nano shape: three rounds of pair tiles
 def test_linear(kalm, m, n, k, res):
     rng = np.random.default_rng(m * 7 + n + k)
     x = rand_bf16(rng, (m, k))
