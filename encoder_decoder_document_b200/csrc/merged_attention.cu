@@ -524,7 +524,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       l_part[half * 128 + r] = l_run;
       mbar_arrive(bar_l);
-      bool wt = mbar_wait(&bar_pv[Jl & 1], (Jl >> 1) & 1, p.wait_ns) && mbar_wait(bar_l, n_it & 1, p.wait_ns);
+      // the item's last P V.  A parity wait is exact only when the barrier is at most one
+      // phase behind it; the group whose own last tile is Jl - 1 never waited on P V_{Jl-2}
+      // (same barrier), so it first waits on P V_{Jl-1} (other barrier, one phase at most),
+      // after which P V_{Jl-2} has completed too (P V products complete in order)
+      bool wt = (Jl == 0 || mbar_wait(&bar_pv[(Jl - 1) & 1], ((Jl - 1) >> 1) & 1, p.wait_ns)) &&
+                mbar_wait(&bar_pv[Jl & 1], (Jl >> 1) & 1, p.wait_ns) && mbar_wait(bar_l, n_it & 1, p.wait_ns);
       if (!__all_sync(0xffffffffu, wt)) {
         ok = false;
         break;

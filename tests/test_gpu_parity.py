@@ -720,6 +720,43 @@ def test_attention_repeat_is_bit_identical(kalm):
     _check_attn(o0, want)
 
 
+@pytest.mark.slow
+def test_attention_layer_repeat_stress_nano(kalm):
+    """A Nano layer's projection, work order and attention, launched back to back 400
+    times on fixed inputs: every attention output is bit-identical to the first.  (Races
+    between the softmax groups' item ends and the in-flight P V products showed up here
+    in about one launch in a hundred before they were fixed.)"""
+    from encoder_decoder_document_b200.scorer import DeviceWeights, FBNLScorer
+    q = synthetic.make_query("nano")
+    sc = FBNLScorer(DeviceWeights.from_bits(q.weights), q.n_q, q.n_kv)
+    sc.prepare(q.n_docs, int(q.doc_len.sum()), int(oracle.pooled_counts(q.doc_len).sum()), q.lq)
+    sc.load_inputs(torch.from_numpy(q.enc.view(np.int16)).view(torch.bfloat16), torch.from_numpy(q.doc_len),
+                   torch.from_numpy(q.x0.view(np.int16)).view(torch.bfloat16))
+    sc.documents()
+    g = torch.Generator(device="cuda").manual_seed(5)
+    sc.x.copy_(torch.randn(sc.x.shape, device="cuda", generator=g).bfloat16())
+    qv, ks, vs = sc.qkv_views()
+    kc, vc = sc.cross_views(3)
+
+    def once(resched):
+        kalm.kalm_linear(sc.x, sc.w.w_qkv[3], sc.qkv)
+        if resched:
+            kalm.kalm_attention_schedule(sc.q_off, sc.pool_off, sc.lq, sc.n_q, sc.n_kv, sc.order)
+        kalm.kalm_merged_attention(qv, ks, vs, kc, vc, sc.q_off, sc.pool_off, sc.lq, sc.n_q, sc.n_kv, sc.o, sc.scale,
+                                   order=sc.order)
+    once(True)
+    torch.cuda.synchronize()
+    ref = sc.o.view(torch.int16).clone()
+    bad = []
+    for i in range(400):
+        once(i % 2 == 0)
+        d = int((sc.o.view(torch.int16) != ref).sum())
+        if d:
+            bad.append((i, d))
+    kalm.kalm_check_device_errors()
+    assert not bad, bad[:5]
+
+
 def test_attention_order_out_of_range_is_flagged(kalm):
     """Entries outside the item range are skipped (nothing written) and flagged."""
     from encoder_decoder_document_b200 import KalmError
