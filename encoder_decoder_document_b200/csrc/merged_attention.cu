@@ -174,7 +174,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* bar_ofree = bars + 13;  // O read out by the epilogue (per item)
   uint64_t* bar_m = bars + 14;   // [2] running max after a tile published (one per tile parity)
   uint64_t* bar_sdone = bars + 16;  // every S of an item done: the Q columns of tensor memory reusable
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 17);
+  uint64_t* bar_sfree = bars + 17;  // [2] S buffer loaded into registers by its softmax group (per tile parity)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 19);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   float* l_part = reinterpret_cast<float*>(sP + 2 * kPBytes + kBarBytes);  // [2][128]
   // running max after the latest tile, per row: written by the tile's group, read by the next
@@ -190,6 +191,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&bar_v[i], 1);
       mbar_init(&bar_s[i], 1);
       mbar_init(&bar_p[i], kSoftmaxThreads / 2);  // one warp group writes each tile's P
+      mbar_init(&bar_sfree[i], kSoftmaxThreads / 2);
       mbar_init(&bar_pv[i], 1);
       mbar_init(&bar_m[i], 4);                    // the four warps of that group
     }
@@ -273,8 +275,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------ S issuer: Q copy and S = Q K^T
-    // S of tile J goes out as soon as K_J has landed and the softmax has read S_{J-2}
-    // (same buffer), independently of the P V products, which warp 11 issues.
+    // S of tile J goes out as soon as K_J has landed and the softmax has loaded S_{J-2}
+    // (same buffer) into registers, independently of the P V products, which warp 11
+    // issues.
     if (lane == 0) {
       const uint32_t q_base = smem_u32(sQ), k_base = smem_u32(sK);
       uint32_t J = 0;
@@ -302,7 +305,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t Jc = J + j;
           const int s = Jc & 1;
           if (!mbar_wait(&bar_k[s], (Jc >> 1) & 1, p.wait_ns) ||
-              (Jc >= 2 && !mbar_wait(&bar_p[s], ((Jc - 2) >> 1) & 1, p.wait_ns))) {  // S_{Jc-2} read
+              (Jc >= 2 && !mbar_wait(&bar_sfree[s], ((Jc - 2) >> 1) & 1, p.wait_ns))) {  // S_{Jc-2} loaded
             ok = false;
             break;
           }
@@ -400,6 +403,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_ld32(lane_base + 256u + s * kBKV, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
         tmem_ld32(lane_base + 256u + s * kBKV + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
         tmem_ld_wait();
+        tc_fence_before();
+        mbar_arrive(&bar_sfree[s]);  // the scores are in registers: the buffer may take S_{Jc+2}
         // visible keys of this tile: self keys k <= pos, cross keys k < Nc
         int n_vis = (j < it.n_self) ? pos + 1 - j * kBKV : it.Nc - (j - it.n_self) * kBKV;
         n_vis = max(0, min(kBKV, n_vis));
