@@ -757,6 +757,30 @@ def test_attention_layer_repeat_stress_nano(kalm):
     assert not bad, bad[:5]
 
 
+@pytest.mark.slow
+def test_step_graph_replays_bit_identical(kalm):
+    """The Nano step graph (the benchmark's launch configuration: both streams,
+    programmatic dependent launches) replayed 300 times gives the same score bits every
+    time, and the same bits as the decode-only graph over the cached documents."""
+    q = synthetic.make_query("nano")
+    sc = _scorer(q, graph=True)
+    torch.cuda.synchronize()
+    ref = sc.scores_to_host().numpy().copy()
+    bad = []
+    for i in range(300):
+        sc.graph.replay()
+        if i % 25 == 24:
+            torch.cuda.synchronize()
+            got = sc.scores_to_host().numpy()
+            if not np.array_equal(got, ref):
+                bad.append(i)
+    sc.graphs_decode[sc.slot].replay()
+    torch.cuda.synchronize()
+    kalm.kalm_check_device_errors()
+    assert not bad, bad
+    np.testing.assert_array_equal(sc.scores_to_host().numpy(), ref)
+
+
 def test_attention_order_out_of_range_is_flagged(kalm):
     """Entries outside the item range are skipped (nothing written) and flagged."""
     from encoder_decoder_document_b200 import KalmError
