@@ -80,6 +80,7 @@ class FBNLScorer:
         self.marks: Optional[list] = None
         self.launches = 0  # kernel launches issued by the last forward()
         self.side: Optional[torch.cuda.Stream] = None  # second stream for work beside the pooling
+        self._side_pending = False  # the broadcast of X is on the second stream, not yet joined
 
     # ------------------------------------------------------------------ buffers
     def prepare(self, n_docs: int, total_tokens: int, total_pooled: int, lq: int, device="cuda") -> None:
@@ -186,7 +187,15 @@ class FBNLScorer:
                               self.scale, order=self.order)
         self._mark("merged_attention")
 
+    def _join_side(self) -> None:
+        """The residual stream X is first read by an output projection: wait for the
+        broadcast if it was issued on the second stream."""
+        if self._side_pending:
+            torch.cuda.current_stream().wait_stream(self.side)
+            self._side_pending = False
+
     def layer_out(self, l: int) -> None:
+        self._join_side()
         kalm_linear(self.o, self.w.w_o[l], self.x, residual=self.x)
         self._mark("o_proj")
 
@@ -215,6 +224,7 @@ class FBNLScorer:
         if last:
             # only each document's final row reaches the readout
             x_last = self.x[Lq - 1::Lq]
+            self._join_side()
             kalm_linear(self.o[Lq - 1::Lq], self.w.w_o[l], x_last, residual=x_last)
             self._mark("o_proj")
         else:
@@ -232,7 +242,17 @@ class FBNLScorer:
 
     def decode(self, broadcast: bool = True) -> None:
         """The query side: the decoder stack over the cached cross K/V, then the readout."""
-        if broadcast:
+        if broadcast and self.marks is None and self.prune:
+            # layer 0's Q|K|V and attention read only the query input: the broadcast of X
+            # runs beside them and the first output projection waits for it
+            if self.side is None:
+                self.side = torch.cuda.Stream()
+            self.side.wait_stream(torch.cuda.current_stream())
+            with torch.cuda.stream(self.side):
+                kalm_broadcast_rows(self.x0, self.q_off, self.x)
+            self.launches += 1
+            self._side_pending = True
+        elif broadcast:
             kalm_broadcast_rows(self.x0, self.q_off, self.x)
             self._mark("broadcast")
         for l in range(self.L):
