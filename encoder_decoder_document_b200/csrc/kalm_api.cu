@@ -1,6 +1,7 @@
 // Runtime plumbing of libkalm: status strings, device check, device error word,
 // tensor-map encoding, ragged offsets, row broadcast and the bounded-wait
 // self-test.
+#include <atomic>
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
@@ -20,8 +21,11 @@ thread_local char g_last_error[512] = {0};
 __device__ uint32_t g_device_error_word;
 
 constexpr int kMaxDevices = 64;
+// `ready` is published with release order after every other field of the
+// device's set-up (and the per-kernel tables written by the set-up hooks), so a
+// thread that reads it true with acquire order also sees those writes.
 struct DeviceState {
-  bool ready = false;
+  std::atomic<bool> ready{false};
   bool ok = false;
   uint32_t* err = nullptr;
 };
@@ -62,9 +66,11 @@ kalm_status ensure_device(int* device_out) {
   if (dev >= kMaxDevices) return fail(KALM_ERR_NO_DEVICE, "device index %d out of range", dev);
   if (device_out) *device_out = dev;
   DeviceState& s = g_dev[dev];
-  if (s.ready) return s.ok ? KALM_OK : fail(KALM_ERR_NO_DEVICE, "device %d is not an sm_100 device", dev);
+  if (s.ready.load(std::memory_order_acquire))
+    return s.ok ? KALM_OK : fail(KALM_ERR_NO_DEVICE, "device %d is not an sm_100 device", dev);
   std::lock_guard<std::mutex> lock(g_mutex);
-  if (s.ready) return s.ok ? KALM_OK : fail(KALM_ERR_NO_DEVICE, "device %d is not an sm_100 device", dev);
+  if (s.ready.load(std::memory_order_relaxed))
+    return s.ok ? KALM_OK : fail(KALM_ERR_NO_DEVICE, "device %d is not an sm_100 device", dev);
   int major = 0, minor = 0;
   if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
       cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess) {
@@ -72,8 +78,8 @@ kalm_status ensure_device(int* device_out) {
     return fail(KALM_ERR_NO_DEVICE, "cannot query device %d", dev);
   }
   if (major != 10 || minor != 0) {
-    s.ready = true;
     s.ok = false;
+    s.ready.store(true, std::memory_order_release);
     return fail(KALM_ERR_NO_DEVICE, "device %d is sm_%d%d; this library is built for sm_100a only", dev, major,
                 minor);
   }
@@ -96,7 +102,7 @@ kalm_status ensure_device(int* device_out) {
   if ((st = setup_linear_kernels()) != KALM_OK) return st;
   if ((st = setup_attention_kernels()) != KALM_OK) return st;
   s.ok = true;
-  s.ready = true;
+  s.ready.store(true, std::memory_order_release);
   return KALM_OK;
 }
 
