@@ -400,6 +400,25 @@ def test_end_to_end_with_empty_documents(kalm, doc_len):
         _check_scores(res[3], s, m)
 
 
+@pytest.mark.parametrize("name,kw", [
+    # the Large architecture (hidden 2560, 8 query / 4 KV heads, Lq 256) with two layers
+    ("large", dict(n_docs=3, layers=2)),
+    # the runtime limits: a 512-row decoder and documents of 1,024 and 1,023 tokens
+    ("tiny", dict(lq=512, doc_len=np.array([1024, 1, 1023, 4]))),
+])
+def test_end_to_end_large_heads_and_maximum_lengths(kalm, name, kw):
+    """Scores against the oracle at the widest head layout and at the longest inputs
+    the runtime accepts, eagerly and in the graph."""
+    q = synthetic.make_query(name, **kw)
+    y, n, m, s = oracle.forward_query(q)
+    for graph in (False, True):
+        sc = _scorer(q, graph=graph)
+        kalm.kalm_check_device_errors()
+        res = sc.scores_to_host().numpy()
+        assert np.all(np.isfinite(res))
+        _check_scores(res[3], s, m)
+
+
 def test_end_to_end_tiny_batch_composition(kalm):
     # a document's score is the same alone and inside the batch (bitwise)
     q = synthetic.make_query("tiny")
