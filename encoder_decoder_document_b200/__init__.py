@@ -128,7 +128,7 @@ def kalm_attention_items(n_docs: int, max_q: int, n_q: int, n_kv: int, last_tile
 
 def kalm_attention_schedule(q_off: torch.Tensor, pool_off: torch.Tensor, max_q: int, n_q: int, n_kv: int,
                             order: torch.Tensor, last_tile_only: bool = False, stream=None) -> None:
-    """Write a heaviest-first work order for kalm_merged_attention into ``order`` (int32)."""
+    """Write a balanced work order for kalm_merged_attention into ``order`` (int32)."""
     call("kalm_attention_schedule", _p(q_off, torch.int64), _p(pool_off, torch.int64), q_off.numel() - 1, int(max_q),
          n_q, n_kv, 1 if last_tile_only else 0, _p(order, torch.int32), order.numel(), _stream(stream))
 

@@ -123,15 +123,13 @@ __device__ __forceinline__ Item make_item(const AttnParams& p, int w) {
 constexpr int kNoMore = -2;  // item_at: this CTA has no further items
 constexpr int kSkip = -1;    // item_at: no item at this pass
 
-// Work item of this CTA's k-th pass.  Without a work order CTA c takes items
-// c, c + grid, c + 2 grid, ...  With one (items sorted heaviest first), it takes
-// positions in snake order -- c in even passes, grid - 1 - c in odd ones -- so
-// every CTA gets a similar mix of heavy and light items.
+// Work item of this CTA's k-th pass: entry k * grid + c of the work order
+// (kalm_attention_schedule lays it out so that the CTAs' total costs come out
+// even), or without one item k * grid + c itself.
 __device__ __forceinline__ int item_at(const AttnParams& p, int k) {
   const int64_t base = static_cast<int64_t>(k) * gridDim.x;
   if (base >= p.n_items) return kNoMore;
-  const int c = static_cast<int>(blockIdx.x);
-  const int64_t idx = base + ((p.order && (k & 1)) ? static_cast<int>(gridDim.x) - 1 - c : c);
+  const int64_t idx = base + static_cast<int>(blockIdx.x);
   if (idx >= p.n_items) return kSkip;
   if (!p.order) return static_cast<int>(idx);
   const int w = p.order[idx];
@@ -615,30 +613,44 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-// Work order for the persistent kernel: every item's cost (its K/V tiles plus one
-// for the per-item Q copy and epilogue) is computed from the offsets, and the
-// items are counting-sorted by cost, heaviest first.  One CTA; the order of equal
-// costs is whatever the atomics give (each item's result does not depend on
-// which CTA computes it).
+// Work order for the persistent kernel (one CTA).  An item's cost is its K/V tiles
+// plus a fixed per-item part (the Q copy, the pipeline refill and the output write
+// at the item's end, about three tiles' time); items without tiles cost nothing.
+// The items are counting-sorted by cost, heaviest first, and dealt out in rounds
+// of `grid` (the attention launch's CTA count): in each round the heaviest
+// remaining item goes to the CTA with the least total cost so far, the next to the
+// next least loaded, and so on (longest-processing-time-first, one item per CTA
+// per round).  The result is laid out so that the attention kernel's CTA c takes
+// entry k * grid + c in its k-th pass: the CTAs that receive an item in a last,
+// partial round are renumbered 0 .. cnt - 1.  The order of equal costs is whatever
+// the atomics give; each item's result does not depend on which CTA computes it.
 constexpr int kSchedThreads = 1024;
 constexpr int kSchedBins = 64;
+constexpr int kItemFixedCost = 3;
 
-__device__ __forceinline__ int item_cost_bin(const AttnParams& p, int w) {
+__device__ __forceinline__ int item_cost(const AttnParams& p, int w) {
   const Item it = make_item(p, w);
-  const int cost = it.nt > 0 ? it.nt + 1 : 0;
-  return kSchedBins - 1 - min(cost, kSchedBins - 1);  // bin 0 = heaviest
+  return it.nt > 0 ? min(it.nt + kItemFixedCost, kSchedBins - 1) : 0;
 }
 
-__global__ void __launch_bounds__(kSchedThreads) attention_schedule_kernel(const AttnParams p, int32_t* order) {
+__global__ void __launch_bounds__(kSchedThreads) attention_schedule_kernel(const AttnParams p, int32_t* order,
+                                                                          int grid) {
   __shared__ int hist[kSchedBins];
   __shared__ int next[kSchedBins];
+  __shared__ int load[kSchedThreads];      // total cost dealt to each CTA so far
+  __shared__ int seg_item[kSchedThreads];  // this round's items, heaviest first
+  __shared__ int seg_cost[kSchedThreads];
+  __shared__ int who[kSchedThreads];       // CTA that takes this round's i-th item
+  __shared__ int label[kSchedThreads];     // final CTA number of each CTA
   pdl_launch_dependents();
   pdl_wait_predecessor();
-  if (threadIdx.x < kSchedBins) hist[threadIdx.x] = 0;
+  const int tid = threadIdx.x;
+  const int n = p.n_items;
+  if (tid < kSchedBins) hist[tid] = 0;
   __syncthreads();
-  for (int w = threadIdx.x; w < p.n_items; w += kSchedThreads) atomicAdd(&hist[item_cost_bin(p, w)], 1);
+  for (int w = tid; w < n; w += kSchedThreads) atomicAdd(&hist[kSchedBins - 1 - item_cost(p, w)], 1);
   __syncthreads();
-  if (threadIdx.x == 0) {
+  if (tid == 0) {
     int run = 0;
     for (int b = 0; b < kSchedBins; ++b) {
       next[b] = run;
@@ -646,7 +658,61 @@ __global__ void __launch_bounds__(kSchedThreads) attention_schedule_kernel(const
     }
   }
   __syncthreads();
-  for (int w = threadIdx.x; w < p.n_items; w += kSchedThreads) order[atomicAdd(&next[item_cost_bin(p, w)], 1)] = w;
+  for (int w = tid; w < n; w += kSchedThreads) order[atomicAdd(&next[kSchedBins - 1 - item_cost(p, w)], 1)] = w;
+  __syncthreads();  // the sorted list is in `order`: every thread reads it back below
+
+  if (tid < grid) {
+    load[tid] = 0;
+    label[tid] = tid;
+  }
+  const int rounds = (n + grid - 1) / grid;
+  int last_cnt = grid;
+  for (int k = 0; k < rounds; ++k) {
+    const int base = k * grid;
+    const int cnt = min(grid, n - base);
+    __syncthreads();
+    if (tid < cnt) {
+      seg_item[tid] = order[base + tid];
+      seg_cost[tid] = item_cost(p, seg_item[tid]);
+    }
+    __syncthreads();
+    if (tid < grid) {  // rank of this CTA by (cost so far, number), ascending
+      const int l = load[tid];
+      int rk = 0;
+      for (int c = 0; c < grid; ++c) {
+        const int lc = load[c];
+        rk += (lc < l || (lc == l && c < tid)) ? 1 : 0;
+      }
+      if (rk < cnt) who[rk] = tid;
+    }
+    __syncthreads();
+    if (tid < cnt) {
+      const int v = who[tid];
+      load[v] += seg_cost[tid];
+      if (cnt == grid) order[base + v] = seg_item[tid];  // a full round: entry base + CTA
+    }
+    last_cnt = cnt;
+  }
+  if (last_cnt == grid) return;  // every round full: the CTA numbers stand
+  // A partial last round: the CTA that takes its i-th item becomes CTA i (so the
+  // round's entries, still in sorted order, stay where they are), the others keep
+  // their relative order after them, and every full round is renumbered.
+  __syncthreads();
+  if (tid == 0) {
+    for (int c = 0; c < grid; ++c) label[c] = -1;
+    for (int i = 0; i < last_cnt; ++i) label[who[i]] = i;
+    int nxt = last_cnt;
+    for (int c = 0; c < grid; ++c)
+      if (label[c] < 0) label[c] = nxt++;
+  }
+  __syncthreads();
+  for (int k = 0; k + 1 < rounds; ++k) {
+    const int base = k * grid;
+    if (tid < grid) seg_item[tid] = order[base + tid];
+    __syncthreads();
+    if (tid < grid) order[base + label[tid]] = seg_item[tid];
+    __syncthreads();
+  }
 }
 
 }  // namespace
@@ -788,7 +854,14 @@ extern "C" kalm_status kalm_attention_schedule(const int64_t* q_off, const int64
   prm.tiles_per_doc = (max_q + prm.P - 1) / prm.P;
   prm.n_items = static_cast<int>(items);
   prm.err = device_error_word();
+  // the attention launch's CTA count for these sizes (one CTA per SM, at most one per item)
+  int sms = 0, dev = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (sms <= 0) sms = 148;
+  int grid = items < sms ? static_cast<int>(items) : sms;
+  if (grid > kSchedThreads) grid = kSchedThreads;  // only the balance depends on it
   return check_cuda(launch_pdl(attention_schedule_kernel, dim3(1), dim3(kSchedThreads), 0,
-                               static_cast<cudaStream_t>(stream), prm, order),
+                               static_cast<cudaStream_t>(stream), prm, order, grid),
                     "launch attention_schedule_kernel");
 }

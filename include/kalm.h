@@ -190,10 +190,11 @@ kalm_status kalm_cross_kv_proj(const kalm_bf16* pooled, int64_t pooled_ld, int64
  *         rows of `out` are left untouched.  Enough when only the final
  *         position is read afterwards (the yes/no readout of the last layer).
  * order   int32[kalm_attention_items(...)] written by kalm_attention_schedule
- *         for the same offsets and sizes, or NULL.  Only the order in which the
- *         persistent CTAs take the work items changes (heaviest first, spread
- *         over the CTAs); the results are the same.  An entry outside the item
- *         range is skipped and flagged in the device error word.
+ *         for the same offsets and sizes, or NULL.  The persistent CTA c takes
+ *         entry k * grid + c in its k-th pass (grid = min(items, SMs)); without an
+ *         order it takes item k * grid + c.  Only which CTA computes which item
+ *         changes; the results are the same.  An entry outside the item range is
+ *         skipped and flagged in the device error word.
  * out     [total_q][ldo] bf16, head h at element h*head_dim
  * lse     fp32 [total_q][n_q] or NULL: natural log of each row's softmax
  *         denominator, in scaled-logit units.
@@ -218,9 +219,12 @@ kalm_status kalm_merged_attention(const kalm_bf16* q, int64_t ldq,
 int64_t kalm_attention_items(int32_t n_docs, int32_t max_q, int32_t n_q, int32_t n_kv, int32_t last_tile_only);
 
 /* Work order for kalm_merged_attention: writes order[0 .. items-1], a
- * permutation of the work items sorted by cost (the item's K/V tiles, from
- * q_off and pool_off), heaviest first.  The costs are the same for every layer
- * of a query, so one order serves all its layers.  order is caller-owned device
+ * permutation of the work items.  An item's cost is its K/V tiles (from q_off and
+ * pool_off) plus a fixed per-item part; the items, sorted heaviest first, are
+ * dealt out in rounds of one item per CTA, each to the CTA with the least total
+ * cost so far, so that every CTA's total comes out close to the mean.  The costs
+ * are the same for every layer of a query, so one order serves all its layers.
+ * Scheduling aid; the pages have no counterpart.  order is caller-owned device
  * memory of at least order_len >= kalm_attention_items(...) entries; stream-
  * ordered, one single-CTA kernel; nothing allocated.  Errors: sizes as
  * kalm_merged_attention, order_len too small -> KALM_ERR_INVALID_ARG. */

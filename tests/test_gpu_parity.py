@@ -659,8 +659,9 @@ def test_cached_documents_match_full_queries(kalm):
 
 
 def _item_costs(q_off, p_off, max_q, n_q, n_kv):
-    """Host restatement of the work items' costs (K/V tiles + 1, 0 for an empty tile),
-    in the kernel's item numbering: item w = tile t (heaviest first), KV head, document."""
+    """Host restatement of the work items' costs (K/V tiles + 3 for the per-item part,
+    0 for an empty tile), in the kernel's item numbering: item w = tile t (last tile
+    first), KV head, document."""
     G = n_q // n_kv
     P = 128 // G
     n = len(q_off) - 1
@@ -676,17 +677,36 @@ def _item_costs(q_off, p_off, max_q, n_q, n_kv):
             costs.append(0)
             continue
         pos1 = min(pos0 + P, lq)
-        costs.append(-(-pos1 // 64) + -(-nc // 64) + 1)
+        costs.append(-(-pos1 // 64) + -(-nc // 64) + 3)
     return np.array(costs)
+
+
+def _cta_loads(order, costs, grid, snake=False):
+    """Total cost per CTA when CTA c takes entry k * grid + c in its k-th pass (with
+    ``snake``: entry k * grid + grid - 1 - c in odd passes)."""
+    loads = np.zeros(grid)
+    for k in range(-(-len(order) // grid)):
+        for c in range(grid):
+            idx = k * grid + (grid - 1 - c if snake and k % 2 else c)
+            if idx < len(order):
+                loads[c] += costs[order[idx]]
+    return loads
+
+
+_BIG = np.random.default_rng(5)
 
 
 @pytest.mark.parametrize("lq,nc,n_q,n_kv", [
     ([128] * 100, list(range(16, 256, 2))[:100], 4, 1),
     ([1, 2, 31, 33, 65, 130, 512], [0, 5, 64, 65, 128, 129, 256], 4, 1),
     ([256, 100, 17], [75, 256, 3], 8, 4),
+    (_BIG.choice([1, 7, 20, 32, 33, 64, 100, 128], 600).tolist(), _BIG.integers(0, 257, 600).tolist(), 4, 1),
 ])
-def test_attention_schedule_sorted_permutation(kalm, lq, nc, n_q, n_kv):
-    """The work order is a permutation of the items, heaviest first by the host cost."""
+def test_attention_schedule_balanced_permutation(kalm, lq, nc, n_q, n_kv):
+    """The work order is a permutation of the items dealt out in rounds of one item per
+    CTA: round k holds the k-th block of the items sorted by the host cost, heaviest
+    first, and no CTA's total cost exceeds the largest total of the plain heaviest-first
+    order taken in snake order over the CTAs."""
     q_off = np.concatenate([[0], np.cumsum(lq)])
     p_off = np.concatenate([[0], np.cumsum(nc)])
     max_q = max(lq)
@@ -698,7 +718,13 @@ def test_attention_schedule_sorted_permutation(kalm, lq, nc, n_q, n_kv):
     assert sorted(got[:n_items].tolist()) == list(range(n_items))
     assert got[n_items:].tolist() == [-7, -7, -7]          # nothing written past the items
     costs = _item_costs(q_off, p_off, max_q, n_q, n_kv)
-    assert (np.diff(costs[got[:n_items]]) <= 0).all()
+    grid = min(n_items, torch.cuda.get_device_properties(0).multi_processor_count)
+    got = got[:n_items]
+    ranked = np.sort(costs)[::-1]
+    for k in range(0, n_items, grid):
+        assert sorted(costs[got[k:k + grid]].tolist()) == sorted(ranked[k:k + grid].tolist()), k
+    snake = _cta_loads(np.argsort(-costs, kind="stable"), costs, grid, snake=True)
+    assert _cta_loads(got, costs, grid).max() <= snake.max()
 
 
 def test_attention_order_gives_identical_results(kalm):
