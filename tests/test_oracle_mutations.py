@@ -57,6 +57,11 @@ MUTATIONS = [
      "out = np.concatenate([a * c + b * s, b * c - a * s], axis=-1)"),
     ("rotary frequencies with exponent i / D",
      "return float(theta) ** (-2.0 * i / head_dim)", "return float(theta) ** (-1.0 * i / head_dim)"),
+    ("default logit scale 1 / head_dim",
+     "scale = 1.0 / math.sqrt(D) if scale is None else scale", "scale = 1.0 / D if scale is None else scale"),
+    ("each document's last encoder row dropped",
+     "a, b = int(query.tok_off[d]), int(query.tok_off[d + 1])",
+     "a, b = int(query.tok_off[d]), int(query.tok_off[d + 1]) - 1"),
 ]
 
 

@@ -360,17 +360,13 @@ def test_end_to_end_zero_weights_closed_form():
     assert O.forward_doc(enc, x0b, *zero, wy, wn, 2, 1, 8, 0.35) == (y, n, m, s)
 
 
-def test_end_to_end_vs_bruteforce_chain():
-    rng = np.random.default_rng(16)
-    H, D, n_q, n_kv, Lq, L = 16, 8, 2, 1, 3, 2
-    enc, x0, w_qkv, w_o, w_kv, wy, wn = _tiny_stack(rng, H, D, n_q, n_kv, Lq, L, length=9)
-    scale = 1.0 / math.sqrt(D)
-    got = O.forward_doc(enc, x0, w_qkv, w_o, w_kv, wy, wn, n_q, n_kv, D, scale)
-    # brute-force chain with the oracle's bf16 rounding points
+def _brute_chain(enc, x0, w_qkv, w_o, w_kv, wy, wn, n_q, n_kv, D, scale):
+    """Pure-Python chain of the brute-force pieces with the oracle's bf16 rounding
+    points, for one document whose encoder rows are all valid.  Returns (yes, no)."""
     rnd = lambda a: O.bf16_round(np.array(a)).tolist()
-    pooled = rnd(brute.pool_padded(enc.tolist(), [1] * 9, 4))
+    pooled = rnd(brute.pool_padded(enc.tolist(), [1] * len(enc), 4))
     X = x0.tolist()
-    for l in range(L):
+    for l in range(len(w_qkv)):
         kv = rnd(brute.matvec_rows(pooled, w_kv[l].tolist()))
         qkv = rnd(brute.matvec_rows(X, w_qkv[l].tolist()))
         q = [[r[h * D:(h + 1) * D] for h in range(n_q)] for r in qkv]
@@ -384,8 +380,61 @@ def test_end_to_end_vs_bruteforce_chain():
         X = rnd([[a + b for a, b in zip(pr, xr)] for pr, xr in zip(proj, X)])
     by = sum(a * b for a, b in zip(X[-1], wy))
     bn = sum(a * b for a, b in zip(X[-1], wn))
+    return by, bn
+
+
+def test_end_to_end_vs_bruteforce_chain():
+    rng = np.random.default_rng(16)
+    H, D, n_q, n_kv, Lq, L = 16, 8, 2, 1, 3, 2
+    enc, x0, w_qkv, w_o, w_kv, wy, wn = _tiny_stack(rng, H, D, n_q, n_kv, Lq, L, length=9)
+    scale = 1.0 / math.sqrt(D)
+    got = O.forward_doc(enc, x0, w_qkv, w_o, w_kv, wy, wn, n_q, n_kv, D, scale)
+    by, bn = _brute_chain(enc, x0, w_qkv, w_o, w_kv, wy, wn, n_q, n_kv, D, scale)
     assert abs(got[0] - by) < 1e-12 and abs(got[1] - bn) < 1e-12
     assert abs(got[3] - brute.softmax2_first(by, bn)) < 1e-13
+
+
+def _bits(a):
+    """float values -> bf16 bit patterns (the synthetic inputs' storage form)."""
+    import synthetic
+    return synthetic.f32_to_bf16_bits(np.asarray(a, np.float32))
+
+
+def test_forward_query_slices_documents_and_uses_the_standard_scale():
+    """forward_query on a hand-built three-document query (1, 6 and 9 encoder rows,
+    every row distinct) against forward_doc on slices written out here, at the
+    standard scaled-dot-product scale 1/sqrt(256) = 1/16 ("What this is": a scaled
+    dot-product attention), and against the pure-Python chain for one document.
+    Documents are packed one after another with no padding rows between them
+    ("Frozen inference contract": right padding, so a document's valid tokens are
+    its first rows)."""
+    import synthetic
+    rng = np.random.default_rng(33)
+    H, D, n_q, n_kv, Lq, L = 16, 256, 2, 1, 3, 1
+    lens = np.array([1, 6, 9], dtype=np.int32)
+    # row t holds distinct values: a random draw plus an offset that grows with t
+    enc_f = rng.standard_normal((16, H)).astype(np.float32) + 0.5 * np.arange(16, dtype=np.float32)[:, None]
+    x0_f = rng.standard_normal((Lq, H)).astype(np.float32)
+    w = synthetic.Weights(
+        w_qkv=_bits(rng.standard_normal((L, (n_q + 2 * n_kv) * D, H)) * 0.2),
+        w_o=_bits(rng.standard_normal((L, H, n_q * D)) * 0.2),
+        w_kv_cross=_bits(rng.standard_normal((L, 2 * n_kv * D, H)) * 0.2),
+        w_yes=_bits(rng.standard_normal(H) * 0.2), w_no=_bits(rng.standard_normal(H) * 0.2))
+    q = synthetic.Query("pin", H, n_q, n_kv, D, L, lens, np.array([0, 1, 7, 16], dtype=np.int64), _bits(enc_f),
+                        Lq, _bits(x0_f), w)
+    got = O.forward_query(q)
+    enc = O.bf16_bits_to_f64(q.enc)
+    x0 = O.bf16_bits_to_f64(q.x0)
+    ws = [O.bf16_bits_to_f64(a) for a in (w.w_qkv, w.w_o, w.w_kv_cross, w.w_yes, w.w_no)]
+    slices = {0: enc[0:1], 1: enc[1:7], 2: enc[7:16]}
+    for d, rows in slices.items():
+        want = O.forward_doc(rows, x0, *ws, n_q, n_kv, D, 1.0 / 16)
+        assert [float(g[d]) for g in got] == list(want), d
+    # the middle document through the pure-Python chain
+    by, bn = _brute_chain(slices[1], x0, *ws, n_q, n_kv, D, 1.0 / 16)
+    assert abs(got[0][1] - by) < 1e-10 and abs(got[1][1] - bn) < 1e-10
+    # the three documents' scores are distinct, so a wrong slice cannot go unnoticed
+    assert len({float(s) for s in got[3]}) == 3
 
 
 def test_forward_query_doc_independence():
