@@ -2,6 +2,7 @@
 from __future__ import annotations
 
 import glob
+import hashlib
 import os
 import shutil
 import subprocess
@@ -37,17 +38,35 @@ def _inputs() -> list[str]:
         glob.glob(os.path.join(INCLUDE, "*.h")) + [os.path.abspath(__file__)]
 
 
+STAMP = LIB + ".srchash"
+
+
+def source_hash() -> str:
+    """SHA-256 over the compiler flags and the name and bytes of every input file."""
+    h = hashlib.sha256()
+    h.update(" ".join(NVCC_FLAGS).encode())
+    for p in sorted(_inputs()):
+        h.update(os.path.relpath(p, ROOT).encode())
+        with open(p, "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
 def up_to_date() -> bool:
-    if not os.path.exists(LIB):
+    """True when libkalm.so was built from exactly the current sources and flags (the
+    hash recorded beside it at build time matches); file times are not trusted, since a
+    copied tree can carry a library that looks newer than sources it was not built from."""
+    if not (os.path.exists(LIB) and os.path.exists(STAMP)):
         return False
-    t = os.path.getmtime(LIB)
-    return all(os.path.getmtime(p) <= t for p in _inputs())
+    with open(STAMP) as f:
+        return f.read().strip() == source_hash()
 
 
 def build(force: bool = False, verbose: bool = False) -> str:
     """Compile every kernel of the path into ``libkalm.so`` beside this file."""
     if not force and up_to_date():
         return LIB
+    digest = source_hash()
     tmp = LIB + ".tmp"
     cmd = [_nvcc(), *NVCC_FLAGS, "-I", INCLUDE, "-I", CSRC, *sources(), "-o", tmp]
     if verbose:
@@ -56,6 +75,8 @@ def build(force: bool = False, verbose: bool = False) -> str:
     if res.returncode != 0:
         raise RuntimeError(f"nvcc failed ({res.returncode}):\n{res.stdout}\n{res.stderr}")
     os.replace(tmp, LIB)
+    with open(STAMP, "w") as f:
+        f.write(digest + "\n")
     return LIB
 
 

@@ -19,6 +19,8 @@ thread_local char g_last_error[512] = {0};
 
 // One error word per device (each device that loads the module holds its own copy).
 __device__ uint32_t g_device_error_word;
+// Where the read-and-clear kernel leaves the word it took (one per device as well).
+__device__ uint32_t g_error_word_taken;
 
 constexpr int kMaxDevices = 64;
 // `ready` is published with release order after every other field of the
@@ -236,6 +238,11 @@ __global__ void broadcast_rows_kernel(const uint4* __restrict__ src, int64_t ld_
   }
 }
 
+// Reads and clears the error word in one atomic step, so a bit that another
+// stream's kernel sets at the same moment lands either in this read or in the
+// next one, never in neither.
+__global__ void take_error_word_kernel() { g_error_word_taken = atomicExch(&g_device_error_word, 0u); }
+
 // Waits on a barrier that is never completed; the bounded wait must expire.
 __global__ void selftest_wait_kernel(uint64_t wait_ns, uint32_t* err) {
   __shared__ __align__(8) uint64_t bar;
@@ -279,13 +286,17 @@ kalm_status kalm_device_check(void) { return ensure_device(nullptr); }
 kalm_status kalm_check_device_errors(kalm_stream_t stream, uint32_t* word_out) {
   kalm_status st = ensure_device(nullptr);
   if (st != KALM_OK) return st;
-  st = check_cuda(cudaStreamSynchronize(static_cast<cudaStream_t>(stream)), "cudaStreamSynchronize");
+  const cudaStream_t s = static_cast<cudaStream_t>(stream);
+  // stream-ordered after the work already queued on `stream`: take the word atomically,
+  // copy it out, wait for both
+  take_error_word_kernel<<<1, 1, 0, s>>>();
+  st = check_cuda(cudaGetLastError(), "launch take_error_word_kernel");
   if (st != KALM_OK) return st;
   uint32_t w = 0;
-  st = check_cuda(cudaMemcpyFromSymbol(&w, kalm::g_device_error_word, sizeof(w)), "read error word");
+  st = check_cuda(cudaMemcpyFromSymbolAsync(&w, kalm::g_error_word_taken, sizeof(w), 0, cudaMemcpyDeviceToHost, s),
+                  "read error word");
   if (st != KALM_OK) return st;
-  const uint32_t zero = 0;
-  st = check_cuda(cudaMemcpyToSymbol(kalm::g_device_error_word, &zero, sizeof(zero)), "clear error word");
+  st = check_cuda(cudaStreamSynchronize(s), "cudaStreamSynchronize");
   if (st != KALM_OK) return st;
   if (word_out) *word_out = w;
   if (w & kErrTimeout) return fail(KALM_ERR_TIMEOUT, "device wait expired (error word 0x%x)", w);

@@ -224,6 +224,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       int n_it = 0;
       bool ok = true;
       bool q_ready = false;  // the current item's Q was issued during the previous item
+      int64_t last_j = -1;   // last K/V tile issued (for the drain at the end)
+      int q_issued = 0;      // Q tiles issued
       int wc = item_at(p, 0);
       Item nxt = load_item(p, wc);
       for (int pass = 0; wc != kNoMore && ok && !*abort_flag; ++pass) {
@@ -241,6 +243,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           mbar_arrive_expect_tx(bar_q, kQBytes);
           tma_load_4d(sQ, &tm_q, bar_q, 0, it.g * p.G, static_cast<int32_t>(it.qi + it.pos0), 0);
+          ++q_issued;
         }
         q_ready = false;
         for (int j = 0; j < it.nt; ++j, ++J) {
@@ -256,6 +259,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           mbar_arrive_expect_tx(&bar_full[s], kKVBytes);
           tma_load_3d(ring + s * kKVBytes, m, &bar_full[s], 0, row, it.g * 4);
+          last_j = J;
           if (!is_v && j == 0 && nxt.nt > 0) {
             // next item's Q as soon as this item's Q is in tensor memory
             if (!mbar_wait(bar_qfree, n_it & 1, p.wait_ns)) {
@@ -265,11 +269,18 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             mbar_arrive_expect_tx(bar_q, kQBytes);
             tma_load_4d(sQ, &tm_q, bar_q, 0, nxt.g * p.G, static_cast<int32_t>(nxt.qi + nxt.pos0), 0);
+            ++q_issued;
             q_ready = true;
           }
         }
         ++n_it;
       }
+      // Drain (matters when a role gave up on a wait): every copy this thread issued has
+      // landed before the CTA tears down.  Each barrier waited on here is at most one
+      // phase behind the issue it waits for, so the parity waits are exact.
+      for (int64_t jj = last_j; jj >= 0 && jj >= last_j - 1; --jj)
+        mbar_wait(&bar_full[jj & 1], static_cast<uint32_t>(jj >> 1) & 1, p.wait_ns);
+      if (q_issued > 0) mbar_wait(bar_q, (q_issued - 1) & 1, p.wait_ns);
     }
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------ S issuer: Q copy and S = Q K^T
@@ -281,6 +292,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t J = 0;
       int n_it = 0;
       bool ok = true;
+      uint64_t* last_bar = nullptr;  // barrier of this thread's last commit (for the drain)
+      uint32_t last_par = 0;
       int wc = item_at(p, 0);
       Item nxt = load_item(p, wc);
       for (int pass = 0; wc != kNoMore && ok && !*abort_flag; ++pass) {
@@ -299,6 +312,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_cp_128x256b(tmem + kTmemQ + static_cast<uint32_t>(kk * 8),
                            sdesc_sw128(q_base + (kk >> 2) * kQSlab + static_cast<uint32_t>((kk & 3) * 32), 16, 1024));
         umma_commit(bar_qfree);
+        last_bar = bar_qfree;
+        last_par = n_it & 1;
         for (int j = 0; j < it.nt && ok && !*abort_flag; ++j) {
           const uint32_t Jc = J + j;
           const int s = Jc & 1;
@@ -317,12 +332,21 @@ __global__ void __launch_bounds__(kThreads, 1)
             umma_bf16_ts(d_s, tmem + kTmemQ + static_cast<uint32_t>(kk * 8), bd, kIdescS, kk != 0 ? 1u : 0u);
           }
           umma_commit(&bar_s[s]);
-          if (j + 1 == it.nt) umma_commit(bar_sdone);  // every S of this item done
+          last_bar = &bar_s[s];
+          last_par = (Jc >> 1) & 1;
+          if (j + 1 == it.nt) {
+            umma_commit(bar_sdone);  // every S of this item done
+            last_bar = bar_sdone;
+            last_par = n_it & 1;
+          }
         }
         J += it.nt;
         ++n_it;
       }
       if (!ok) fail_wait();
+      // Drain: tensor-core operations complete in issue order, so once the last commit's
+      // barrier completes nothing this thread issued still reads shared or tensor memory
+      if (last_bar) mbar_wait(last_bar, last_par, p.wait_ns);
     }
   } else if (warp == kMmaWarpPV) {
     // ------------------------------------------------------------ P V issuer
@@ -331,6 +355,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t J = 0;
       int n_it = 0;
       bool ok = true;
+      int64_t last_j = -1;  // last P V issued (for the drain)
       int wc = item_at(p, 0);
       Item nxt = load_item(p, wc);
       for (int pass = 0; wc != kNoMore && ok && !*abort_flag; ++pass) {
@@ -356,11 +381,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             umma_bf16_ss(tmem, ad, bd, kIdescPV, (j | kk) != 0 ? 1u : 0u);
           }
           umma_commit(&bar_pv[s]);
+          last_j = Jc;
         }
         J += it.nt;
         ++n_it;
       }
       if (!ok) fail_wait();
+      if (last_j >= 0) mbar_wait(&bar_pv[last_j & 1], static_cast<uint32_t>(last_j >> 1) & 1, p.wait_ns);
     }
   } else {
     // ------------------------------------------------------------ softmax warps 0..7

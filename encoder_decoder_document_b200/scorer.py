@@ -24,11 +24,16 @@ from typing import Optional
 import numpy as np
 import torch
 
-from . import (kalm_broadcast_rows, kalm_chunk_pool, kalm_cross_kv_proj, kalm_device_check, kalm_linear,
+from . import (kalm_broadcast_rows, kalm_check_device_errors, kalm_chunk_pool, kalm_cross_kv_proj,
+               kalm_device_check, kalm_linear,
                kalm_merged_attention, kalm_ragged_offsets, kalm_yes_no_score, kalm_attention_items,
                kalm_attention_schedule, kalm_linear_rope, kalm_rope_table)
 
 HEAD_DIM = 256
+# the pages' runtime limits ("Runtime boundaries"): passages of at most 1,024 encoder
+# tokens, a query budget of 512 tokens
+MAX_DOC_TOKENS = 1024
+MAX_QUERY_TOKENS = 512
 
 
 def bf16_from_bits(bits: np.ndarray, device="cuda") -> torch.Tensor:
@@ -363,6 +368,8 @@ class FBNLScorer:
         Query k+1's inputs are copied on a side stream into the other input slot
         while query k runs (one captured graph per slot); every copy and every
         result read happen inside the call, which returns without synchronising.
+        Device errors (an expired bounded wait, invalid device data) are only
+        flagged on the device: call ``check_errors()`` before trusting ``outs``.
         Requires capture() first."""
         if self.graphs is None:
             raise RuntimeError("score_stream needs capture() first")
@@ -411,7 +418,8 @@ class FBNLScorer:
         each query's decoder-input copy with the previous query's compute.
 
         x0s[k]: pinned host bf16 [lq][H] decoder input of query k; outs[k]: pinned
-        [4][n_docs] fp32 host tensor for (yes, no, margin, score).  Requires
+        [4][n_docs] fp32 host tensor for (yes, no, margin, score).  Returns without
+        synchronising; call ``check_errors()`` before trusting ``outs``.  Requires
         cache_documents() (or a full forward over the same documents) and capture()."""
         if not getattr(self, "graphs_decode", None):
             raise RuntimeError("score_cached_stream needs capture() first")
@@ -447,17 +455,42 @@ class FBNLScorer:
 
         x0: bf16 bits [lq][H] (decoder input of the query); enc: bf16 bits
         [sum(doc_len)][H] (packed encoder states); doc_len: int [n_docs]."""
-        doc_len = np.asarray(doc_len, dtype=np.int32)
+        doc_len = np.asarray(doc_len)
+        if doc_len.ndim != 1:
+            raise ValueError("rerank: doc_len must be one length per document")
+        if doc_len.size and (doc_len.min() < 0 or doc_len.max() > MAX_DOC_TOKENS):
+            raise ValueError(f"rerank: document lengths must lie in [0, {MAX_DOC_TOKENS}] "
+                             f"(got {int(doc_len.min())}..{int(doc_len.max())})")
+        lq = int(np.asarray(x0).shape[0])
+        if not 1 <= lq <= MAX_QUERY_TOKENS:
+            raise ValueError(f"rerank: the query input must have 1..{MAX_QUERY_TOKENS} rows (got {lq})")
+        doc_len = doc_len.astype(np.int32)
         n = int(doc_len.shape[0])
         total_tokens = int(doc_len.sum())
+        if np.asarray(enc).shape[0] < total_tokens:
+            raise ValueError(f"rerank: enc holds {np.asarray(enc).shape[0]} rows, doc_len sums to {total_tokens}")
         total_pooled = int(((doc_len.astype(np.int64) + self.chunk - 1) // self.chunk).sum())
-        self.prepare(n, total_tokens, total_pooled, int(x0.shape[0]))
+        self.prepare(n, total_tokens, total_pooled, lq)
         self.load_inputs(torch.from_numpy(np.ascontiguousarray(enc).view(np.int16)).view(torch.bfloat16),
                          torch.from_numpy(doc_len), torch.from_numpy(np.ascontiguousarray(x0).view(np.int16))
                          .view(torch.bfloat16))
         self.run()
         res = self.scores_to_host().numpy()
+        # a bounded wait that expired or invalid device data leaves only a flag on the
+        # device: raise instead of returning scores computed past it
+        self.check_errors()
         return rank(res[2], res[3], top_n)
+
+    def check_errors(self) -> None:
+        """Wait for this scorer's streams and raise ``KalmError`` if a kernel recorded a
+        device error (a bounded wait that expired, or invalid device data) since the
+        last check.  ``score_stream`` and ``score_cached_stream`` return without waiting;
+        call this once their results are needed."""
+        if self.side is not None:
+            torch.cuda.current_stream().wait_stream(self.side)
+        if getattr(self, "_copy_stream", None) is not None:
+            torch.cuda.current_stream().wait_stream(self._copy_stream)
+        kalm_check_device_errors()
 
 
 def rank(margin: np.ndarray, score: np.ndarray, top_n: Optional[int] = None):

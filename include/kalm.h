@@ -81,6 +81,10 @@ const char* kalm_last_error(void);
 kalm_status kalm_device_check(void);
 
 /* Synchronise `stream`, read and clear the current device's error word.
+ * The read and the clear are one atomic exchange, ordered on `stream` after the
+ * work already queued there.  Kernels still running on other streams may set
+ * bits after it; those bits are kept for the next call (to see them in this
+ * one, let every stream that runs library kernels go idle first).
  * *word_out (nullable) receives the raw word: bit 0 = a bounded wait expired,
  * bit 1 = invalid device data (e.g. a length above its limit); bits 8..15 name
  * the kernel (1 pool, 2 linear, 3 attention, 4 readout, 5 offsets, 6 self-test).
@@ -89,6 +93,12 @@ kalm_status kalm_check_device_errors(kalm_stream_t stream, uint32_t* word_out);
 
 /* Ragged offsets: tok_off[d] = sum_{e<d} len[e], pool_off[d] = sum_{e<d}
  * ceil(len[e] / chunk), for d = 0..n (both arrays hold n+1 int64 values).
+ * "KaLM-Reranker-V1-Small-Q4_K_M-GGUF", "Runtime boundaries": passages of at
+ * most 1,024 encoder tokens, pooled in groups of 4; "KaLM-Reranker-V1-Large-
+ * Q8_0-GGUF", "Frozen inference contract": right padding, so a document's
+ * valid tokens are its first len[d] rows and it yields ceil(len[d] / 4)
+ * pooled vectors.  The documents of one query are packed one after another
+ * ("KaLM-Reranker-V1-Nano - MLX", "Speed": all documents decoded in one batch).
  * len: int32 device array of n values in [0, KALM_MAX_DOC_TOKENS]; a value out
  * of range is clamped to the range and flagged in the device error word.
  * n >= 0, chunk >= 1.  Either output may be NULL. */
@@ -126,7 +136,11 @@ kalm_status kalm_chunk_pool(const kalm_bf16* enc, int64_t enc_ld, const int64_t*
 
 /* Dense projection y = x . w^T (+ residual), bf16 in, fp32 accumulate, bf16 out.
  * The tcgen05 (5th-generation tensor core) GEMM behind steps 2 and the decoder
- * projections.
+ * projections.  "KaLM-Reranker-V1-Nano - MLX", "What this is": the decoder
+ * projects its hidden states to the self-attention Q/K/V, and the cross K/V
+ * are projections of the cached passage encodings; the attention output goes
+ * back through the output projection onto the residual stream (the synthetic
+ * attention-only decoder: X <- X + Attn(X Wq, X Wk, X Wv, P Wk_c, P Wv_c) Wo).
  *
  * x        [m][ldx] bf16 (m rows of k values)
  * w        [n][ldw] bf16, the nn.Linear layout [out][in]
@@ -194,7 +208,11 @@ kalm_status kalm_cross_kv_proj(const kalm_bf16* pooled, int64_t pooled_ld, int64
  *         entry k * grid + c in its k-th pass (grid = min(items, SMs)); without an
  *         order it takes item k * grid + c.  Only which CTA computes which item
  *         changes; the results are the same.  An entry outside the item range is
- *         skipped and flagged in the device error word.
+ *         skipped and flagged in the device error word.  The order must come
+ *         from kalm_attention_schedule called with the same q_off, pool_off,
+ *         n_docs, max_q, n_q, n_kv and last_tile_only: an order made for other
+ *         sizes can repeat or leave out items while every entry is in range, and
+ *         the items it leaves out are then not written (nothing detects that).
  * out     [total_q][ldo] bf16, head h at element h*head_dim
  * lse     fp32 [total_q][n_q] or NULL: natural log of each row's softmax
  *         denominator, in scaled-logit units.
