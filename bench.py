@@ -161,6 +161,28 @@ def pool_chunks(enc, len_d, chunks=(1, 2, 4, 8), reps=10):
     return out
 
 
+def plain_copy(src, reps=10):
+    """A plain device copy (torch) of the encoder states the pooling reads, L2 flushed
+    before each call: the bandwidth a read of that size reaches without any pooling
+    (bytes = read + write of the tensor)."""
+    import torch
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device="cuda")
+    dst = torch.empty_like(src)
+    ts = []
+    for i in range(reps + 2):
+        flush.fill_(1.0)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        dst.copy_(src)
+        b.record()
+        b.synchronize()
+        if i >= 2:
+            ts.append(a.elapsed_time(b))
+    us = 1e3 * statistics.median(ts)
+    byts = 2 * src.numel() * src.element_size()
+    return {"bytes": byts, "us": us, "gbs": byts / (us * 1e-6) / 1e9}
+
+
 def rope_alone(sc, theta=1e4, reps=10):
     """Cost of the rotary embedding on one layer's Q|K|V (all documents' rows, Q and
     self-K heads), L2 flushed before each call, medians: the standalone rotation
@@ -195,11 +217,19 @@ def rope_alone(sc, theta=1e4, reps=10):
             "fused_extra_us": fused - plain}
 
 
+def sweep_queries(n_docs: int) -> int:
+    """Distinct queries timed per sweep point (the configuration names 1,000 per point;
+    a bounded number keeps the run within minutes): 8, and 2 at 4096 documents."""
+    return 8 if n_docs <= 1024 else 2
+
+
 def run_sweep(args, doc_counts=(1, 16, 100, 1024, 4096)):
     """End-to-end throughput at the sweep shapes (Nano model, log-normal lengths with
-    median 200 clipped to [1, 1024], one seeded query per point with Lq drawn from
-    [32, 512]): K steps of the captured graph per point, L2 flushed before each step,
-    plus the pooling and attention kernels' own times from the instrumented graph."""
+    median 200 clipped to [1, 1024], Lq drawn from [32, 512] per query): at each point,
+    distinct seeded queries (seed 4 + k for query k), each with its own lengths, its own
+    query length and its own captured graph; K steps per query, L2 flushed before each
+    step.  Per point: total documents / total time over its queries, plus the pooling and
+    attention kernels' own times from each query's instrumented graph."""
     import torch
     import synthetic
     from encoder_decoder_document_b200 import _build, kalm_check_device_errors
@@ -207,47 +237,56 @@ def run_sweep(args, doc_counts=(1, 16, 100, 1024, 4096)):
     _build.build()
     pk = peaks()
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device="cuda")
-    weights = None
+    weights = synthetic.make_query("sweep", n_docs=1, seed=4).weights
+    dw = DeviceWeights.from_bits(weights)
     out = []
     for n in doc_counts:
-        q = synthetic.make_query("sweep", n_docs=n, seed=4, with_weights=weights is None)
-        if weights is None:
-            weights = q.weights
-        q = dataclasses.replace(q, weights=weights)
-        w = workload(q)
-        sc = FBNLScorer(DeviceWeights.from_bits(weights), q.n_q, q.n_kv)
-        total_pooled = int(((q.doc_len.astype(np.int64) + 3) // 4).sum())
-        sc.prepare(q.n_docs, int(q.doc_len.sum()), total_pooled, q.lq)
-        sc.load_inputs(torch.from_numpy(q.enc.view(np.int16)).view(torch.bfloat16),
-                       torch.from_numpy(q.doc_len), torch.from_numpy(q.x0.view(np.int16)).view(torch.bfloat16))
-        sc.capture(instrument=True)
-        ts, per = [], {}
-        for i in range(args.warmup + args.steps):
-            for g in (sc.graph, sc.graph_inst):
-                flush.fill_(1.0)
-                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-                a.record()
-                g.replay()
-                b.record()
-                b.synchronize()
-                if i >= args.warmup:
-                    if g is sc.graph:
-                        ts.append(a.elapsed_time(b))
-                    else:
-                        for label, v in sc.kernel_times().items():
-                            per.setdefault(label, []).extend(v)
-        kalm_check_device_errors()
-        ms = statistics.median(ts)
-        attn_us = 1e3 * sum(per["merged_attention"]) / args.steps
-        pool_us = 1e3 * statistics.mean(per["chunk_pool"])
-        out.append({"docs": n, "lq": q.lq, "encoder_tokens": int(q.doc_len.sum()), "ms_per_query": ms,
-                    "pairs_per_s": n / (ms * 1e-3), "step_tflops": w["total_flops"] / (ms * 1e-3) / 1e12,
-                    "attention_us": attn_us, "attention_tflops": w["merged_attention"] / (attn_us * 1e-6) / 1e12,
-                    "pool_us": pool_us, "pool_gbs": w["pool_bytes"] / (pool_us * 1e-6) / 1e9,
-                    "pool_frac": w["pool_bytes"] / (pool_us * 1e-6) / 1e9 / pk["hbm"]})
-        print(json.dumps(out[-1]), flush=True)
-        del sc
+        nq = sweep_queries(n)
+        tot_ms, tot_docs, lqs = 0.0, 0, []
+        attn_us, attn_flops, pool_us, pool_bytes, flops = 0.0, 0, 0.0, 0, 0
+        for k in range(nq):
+            q = synthetic.make_query("sweep", n_docs=n, seed=4 + k, with_weights=False)
+            q = dataclasses.replace(q, weights=weights)
+            w = workload(q)
+            sc = FBNLScorer(dw, q.n_q, q.n_kv)
+            total_pooled = int(((q.doc_len.astype(np.int64) + 3) // 4).sum())
+            sc.prepare(q.n_docs, int(q.doc_len.sum()), total_pooled, q.lq)
+            sc.load_inputs(torch.from_numpy(q.enc.view(np.int16)).view(torch.bfloat16),
+                           torch.from_numpy(q.doc_len), torch.from_numpy(q.x0.view(np.int16)).view(torch.bfloat16))
+            sc.capture(instrument=True)
+            ts, per = [], {}
+            for i in range(args.warmup + args.steps):
+                for g in (sc.graph, sc.graph_inst):
+                    flush.fill_(1.0)
+                    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                    a.record()
+                    g.replay()
+                    b.record()
+                    b.synchronize()
+                    if i >= args.warmup:
+                        if g is sc.graph:
+                            ts.append(a.elapsed_time(b))
+                        else:
+                            for label, v in sc.kernel_times().items():
+                                per.setdefault(label, []).extend(v)
+            kalm_check_device_errors()
+            tot_ms += sum(ts)
+            tot_docs += n * len(ts)
+            lqs.append(q.lq)
+            attn_us += 1e3 * sum(per["merged_attention"]) / args.steps
+            attn_flops += w["merged_attention"]
+            pool_us += 1e3 * statistics.mean(per["chunk_pool"])
+            pool_bytes += w["pool_bytes"]
+            flops += w["total_flops"] * len(ts)
+            del sc
         torch.cuda.empty_cache()
+        out.append({"docs": n, "queries": nq, "steps_per_query": args.steps, "lq": lqs,
+                    "ms_per_query": tot_ms * n / tot_docs, "pairs_per_s": tot_docs / (tot_ms * 1e-3),
+                    "step_tflops": flops / (tot_ms * 1e-3) / 1e12,
+                    "attention_us_per_query": attn_us / nq, "attention_tflops": attn_flops / (attn_us * 1e-6) / 1e12,
+                    "pool_us_per_query": pool_us / nq, "pool_gbs": pool_bytes / (pool_us * 1e-6) / 1e9,
+                    "pool_frac": pool_bytes / (pool_us * 1e-6) / 1e9 / pk["hbm"]})
+        print(json.dumps(out[-1]), flush=True)
     return out
 
 
@@ -338,17 +377,29 @@ class Clocks:
                 "samples": len(rows)}
 
 
-def cpu_baseline(q, n_sample: int):
-    """The fp64 oracle (as it stands) on the first n_sample documents of the query."""
+def cpu_baseline(q, n_sample: int, one_thread_docs: int = 0):
+    """The fp64 oracle (as it stands: a per-document loop whose matrix products run on
+    the BLAS thread pool) on the first n_sample documents of the query.  ``cores`` is
+    the BLAS pool's thread count, the threads the oracle actually used; ``host_cores``
+    the host's logical CPUs.  With ``one_thread_docs`` the same oracle is also timed
+    with the BLAS pool limited to one thread on that many documents."""
     import oracle
-    from threadpoolctl import threadpool_info
+    from threadpoolctl import threadpool_info, threadpool_limits
     t0 = time.perf_counter()
     oracle.forward_query(q, docs=range(n_sample))
     dt = time.perf_counter() - t0
     threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
-    return {"value": n_sample / dt, "unit": UNIT, "cores": threads, "kind": "oracle",
-            "sample": f"{n_sample} of {q.n_docs} documents of one {q.name} query, all {q.layers} layers, fp64 "
-                      f"numpy (BLAS threads={threads}); {dt:.1f} s"}
+    res = {"value": n_sample / dt, "unit": UNIT, "cores": threads, "host_cores": os.cpu_count(), "kind": "oracle",
+           "sample": f"{n_sample} of {q.n_docs} documents of one {q.name} query, all {q.layers} layers, fp64 "
+                     f"numpy, documents one after another, matrix products on {threads} BLAS threads; {dt:.1f} s"}
+    if one_thread_docs:
+        with threadpool_limits(limits=1):
+            t0 = time.perf_counter()
+            oracle.forward_query(q, docs=range(one_thread_docs))
+            dt1 = time.perf_counter() - t0
+        res["one_thread"] = {"value": one_thread_docs / dt1, "unit": UNIT, "cores": 1,
+                             "sample": f"{one_thread_docs} documents, BLAS limited to 1 thread; {dt1:.1f} s"}
+    return res
 
 
 def run_reference(args):
@@ -558,6 +609,7 @@ def main():
         kern[k]["ai_flop_per_byte"] = ai_k
         kern[k]["frac_of_ai_bound"] = kern[k]["tflops"] / min(pk["bf16"], ai_k * pk["hbm"] / 1e3)
     pool_gbs = w["pool_bytes"] / (kern["chunk_pool"]["avg_us"] * 1e-6) / 1e9
+    copy_ref = plain_copy(sc.enc[: int(q.doc_len.sum())])
     attn_proj_us = sum(kern[k]["us_per_step"] for k in ("merged_attention", "cross_kv_proj") if k in kern)
     attn_proj_flops = w["cross_kv_proj"] + w["merged_attention"]
     step_flops = w["total_flops"]
@@ -573,7 +625,7 @@ def main():
         if rope is not None:
             rope["frac"] = rope["gbs"] / pk["hbm"]
         if not args.no_cpu_baseline and world == 1:
-            cb = cpu_baseline(q, args.cpu_sample_docs or q.n_docs)
+            cb = cpu_baseline(q, args.cpu_sample_docs or q.n_docs, one_thread_docs=min(10, q.n_docs))
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
@@ -591,7 +643,9 @@ def main():
             "roofline": roofline,
             "algorithmic_flops_per_step": step_flops,
             "pool": {"bytes": w["pool_bytes"], "avg_us": kern["chunk_pool"]["avg_us"], "achieved_gbs": pool_gbs,
-                     "peak_gbs": pk["hbm"], "frac": pool_gbs / pk["hbm"]},
+                     "peak_gbs": pk["hbm"], "frac": pool_gbs / pk["hbm"],
+                     "plain_copy_same_size": dict(copy_ref, frac=copy_ref["gbs"] / pk["hbm"]),
+                     "frac_of_plain_copy": pool_gbs / copy_ref["gbs"]},
             "attn_plus_cross_proj": {"flops": attn_proj_flops, "us": attn_proj_us,
                                      "tflops": attn_proj_flops / (attn_proj_us * 1e-6) / 1e12,
                                      "frac": attn_proj_flops / (attn_proj_us * 1e-6) / 1e12 / pk["bf16"]},
