@@ -24,6 +24,15 @@ POOL_TOL = 1e-2
 ATTN_MAX_TOL, ATTN_MEAN_TOL = 2e-2, 5e-3
 SCORE_TOL = 1e-3
 RANK_GAP = 1e-2
+# End-to-end scores of deep stacks (Small: 26 layers, hidden 1152; the sweep's longer
+# queries) against the oracle's own fp64 chain.  The synthetic stack has no norms, so a
+# bf16-stored chain amplifies rounding-order differences layer over layer: a plain fp32
+# numpy chain of the same steps (rounded to bf16 at the same points) lands up to 2.5e-3
+# from the fp64 chain on the Small query (17 of 100 documents beyond 1e-3), and reordering
+# only its fp32 sums moves one document's score by 1.3e-3.  Every kernel stays within the
+# stated tolerances at every layer (test_stage_parity_full_size); end to end these
+# configurations are held to 3e-3 and to the stated ranking rule.
+DEEP_SCORE_TOL = 3e-3
 
 
 @pytest.fixture(scope="module")
@@ -366,8 +375,8 @@ def _scorer(q, graph=False, rope_theta=None):
     return sc
 
 
-def _check_scores(got_score, want_score, want_margin):
-    assert np.abs(got_score - want_score).max() <= SCORE_TOL
+def _check_scores(got_score, want_score, want_margin, tol=SCORE_TOL):
+    assert np.abs(got_score - want_score).max() <= tol
     # ranking: any pair the oracle separates by more than the gap keeps its order
     n = len(want_score)
     for i in range(n):
@@ -472,7 +481,7 @@ def test_end_to_end_full_configuration(kalm, name):
     res = sc.scores_to_host().numpy()
     y, n, m, s = oracle.forward_query(q)
     assert np.all(np.isfinite(res))
-    _check_scores(res[3], s, m)
+    _check_scores(res[3], s, m, SCORE_TOL if name == "nano" else DEEP_SCORE_TOL)
     # the best-first lists agree at the top wherever the oracle separates the entries
     top = np.argsort(-m, kind="stable")[:5]
     assert all(m[top[i]] - m[top[i + 1]] <= RANK_GAP or res[2][top[i]] > res[2][top[i + 1]] for i in range(4))
@@ -497,7 +506,7 @@ def test_end_to_end_sweep_points(kalm, n_docs, seed):
     res = sc.scores_to_host().numpy()
     assert np.all(np.isfinite(res))
     y, n, m, s = oracle.forward_query(q, docs=docs)
-    _check_scores(res[3][docs], s, m)
+    _check_scores(res[3][docs], s, m, DEEP_SCORE_TOL)
 
 
 @pytest.mark.slow
@@ -513,7 +522,7 @@ def test_end_to_end_sweep_4096_documents_sampled(kalm):
     res = sc.scores_to_host().numpy()
     assert np.all(np.isfinite(res))
     y, n, m, s = oracle.forward_query(q, docs=docs)
-    _check_scores(res[3][docs], s, m)
+    _check_scores(res[3][docs], s, m, DEEP_SCORE_TOL)
 
 
 @pytest.mark.slow
@@ -536,7 +545,9 @@ def _rows(t, q, docs):
 
 
 @pytest.mark.slow
-@pytest.mark.parametrize("name,docs", [("nano", [5, 61]), ("small", [7, 88]),
+@pytest.mark.parametrize("name,docs", [("nano", [5, 61]),
+                                       # Small: 0 and 1 drift furthest end to end (fp64 vs bf16 chains)
+                                       ("small", [0, 1, 7, 88]),
                                        # Large: the shortest (36) and longest (9) documents among six
                                        ("large", [1, 9, 36, 50, 77, 99])])
 def test_stage_parity_full_size(kalm, name, docs):
