@@ -49,6 +49,7 @@ def parse():
     ap.add_argument("--cpu-sample-docs", type=int, default=0, help="documents in the oracle sample (0 = auto)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-pool-sweep", action="store_true", help="skip the pooling-only sweep at 1024/4096 docs")
+    ap.add_argument("--no-fused", action="store_true", help="skip the fused attention + output projection step")
     ap.add_argument("--rope-theta", type=float, default=None,
                     help="rotate the decoder's self Q/K with this rotary base in every layer (default: off)")
     ap.add_argument("--sweep", action="store_true",
@@ -158,6 +159,54 @@ def pool_chunks(enc, len_d, chunks=(1, 2, 4, 8), reps=10):
         us = 1e3 * statistics.median(ts)
         byts = int((lens.sum() + nc.sum()) * H * 2 + 8 * n)
         out.append({"chunk": c, "bytes": byts, "us": us, "gbs": byts / (us * 1e-6) / 1e9})
+    return out
+
+
+def fused_layers(args, q, weights_dev, w, pk):
+    """The same query through a scorer whose layers (all but the pruned last one) run as
+    one fused attention + output projection launch (kalm_merged_attention_out_proj):
+    steps of its graph timed like the main step (L2 flushed before each), and the fused
+    kernel's own launch time from its instrumented graph."""
+    import torch
+    from encoder_decoder_document_b200.scorer import FBNLScorer
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device="cuda")
+    sc = FBNLScorer(weights_dev, q.n_q, q.n_kv, rope_theta=args.rope_theta, fused_out=True)
+    total_pooled = int(((q.doc_len.astype(np.int64) + 3) // 4).sum())
+    sc.prepare(q.n_docs, int(q.doc_len.sum()), total_pooled, q.lq)
+    sc.load_inputs(torch.from_numpy(q.enc.view(np.int16)).view(torch.bfloat16), torch.from_numpy(q.doc_len),
+                   torch.from_numpy(q.x0.view(np.int16)).view(torch.bfloat16))
+    sc.capture(instrument=True)
+    step_ms, per = [], {}
+    for i in range(max(args.warmup, 3) + args.steps):
+        for g in (sc.graph, sc.graph_inst):
+            flush.fill_(1.0)
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            g.replay()
+            b.record()
+            b.synchronize()
+            if i >= max(args.warmup, 3):
+                if g is sc.graph:
+                    step_ms.append(a.elapsed_time(b))
+                else:
+                    for label, v in sc.kernel_times().items():
+                        per.setdefault(label, []).extend(v)
+    from encoder_decoder_document_b200 import kalm_check_device_errors
+    kalm_check_device_errors()
+    ms = sum(step_ms) / len(step_ms)
+    fused_us = 1e3 * statistics.mean(per["attention_out_proj"])
+    n_fused = len(per["attention_out_proj"]) / args.steps
+    # algorithmic FLOPs of one fused launch: a full layer's attention and output projection
+    H, D, nq, lq, n = q.hidden, q.head_dim, q.n_q, q.lq, q.n_docs
+    nc = int(((q.doc_len.astype(np.int64) + 3) // 4).sum())
+    flops = 4 * nq * D * (n * lq * (lq + 1) // 2 + lq * nc) + 2 * nq * D * H * n * lq
+    out = {"value": q.n_docs / (ms * 1e-3), "unit": UNIT, "ms_per_step": ms, "launches_per_step": n_fused,
+           "fused_avg_us": fused_us, "fused_tflops": flops / (fused_us * 1e-6) / 1e12,
+           "fused_frac": flops / (fused_us * 1e-6) / 1e12 / pk["bf16"],
+           "how": "FBNLScorer(fused_out=True): merged attention and output projection + residual of every layer "
+                  "but the last in one persistent launch; projection tiles claimed as CTAs finish their attention "
+                  "items, each waiting only for its own document"}
+    del sc
     return out
 
 
@@ -622,6 +671,7 @@ def main():
         chunks = None if args.no_pool_sweep else [dict(x, frac=x["gbs"] / pk["hbm"])
                                                   for x in pool_chunks(sc.enc[: int(q.doc_len.sum())], sc.doc_len)]
         rope = None if args.no_pool_sweep else dict(rope_alone(sc), frac=None)
+        fused = None if (args.no_fused or world > 1) else fused_layers(args, q, sc.w, w, pk)
         if rope is not None:
             rope["frac"] = rope["gbs"] / pk["hbm"]
         if not args.no_cpu_baseline and world == 1:
@@ -668,6 +718,7 @@ def main():
                                    "the decoder-only graph (L2 flushed before each step); e2e through "
                                    "FBNLScorer.score_cached_stream with the query input copied in and scores read "
                                    "back"},
+            "fused_layer": fused,
             "pool_sweep": sweep,
             "pool_chunks": chunks,
             "rope": rope,

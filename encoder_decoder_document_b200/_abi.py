@@ -33,6 +33,10 @@ SIGNATURES = {
     "kalm_merged_attention": [c_vp, c_i64, c_vp, c_vp, c_i64, c_vp, c_vp, c_i64, c_vp, c_vp, c_i64, c_vp, c_i32,
                               c_i32, c_i64, c_i64, c_i32, c_i32, c_i32, c_f32, c_i32, c_vp, c_vp, c_i64, c_vp,
                               c_vp],
+    "kalm_merged_attention_out_proj": [c_vp, c_i64, c_vp, c_vp, c_i64, c_vp, c_vp, c_i64, c_vp, c_vp, c_i64, c_vp,
+                                       c_i32, c_i32, c_i64, c_i64, c_i32, c_i32, c_i32, c_f32, c_vp, c_vp, c_i64,
+                                       c_vp, c_i64, c_vp, c_i64, c_i32, c_vp, c_i64, c_vp],
+    "kalm_attention_out_proj_sync_len": [c_i32],
     "kalm_attention_items": [c_i32, c_i32, c_i32, c_i32, c_i32],
     "kalm_attention_schedule": [c_vp, c_vp, c_i32, c_i32, c_i32, c_i32, c_i32, c_vp, c_i64, c_vp],
     "kalm_yes_no_score": [c_vp, c_i64, c_vp, c_i32, c_i32, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp],
@@ -43,7 +47,7 @@ SIGNATURES = {
                          c_vp, c_vp],
     "kalm_rope_table": [c_f32, c_i32, c_vp, c_vp],
 }
-_RESTYPE = {"kalm_version": c_i32, "kalm_attention_items": c_i64, "kalm_status_string": ctypes.c_char_p, "kalm_last_error": ctypes.c_char_p}
+_RESTYPE = {"kalm_version": c_i32, "kalm_attention_items": c_i64, "kalm_attention_out_proj_sync_len": c_i64, "kalm_status_string": ctypes.c_char_p, "kalm_last_error": ctypes.c_char_p}
 
 
 class KalmError(RuntimeError):

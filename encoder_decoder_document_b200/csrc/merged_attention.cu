@@ -65,7 +65,7 @@ constexpr int kKVBytes = kBKV * kD * 2;        // 4 slabs of 64 rows x 128 B
 constexpr int kQSlab = kBM * 128;              // 16 KB
 constexpr int kKVSlab = kBKV * 128;            // 8 KB
 constexpr int kPBytes = kBM * kBKV * 2;        // 1 slab of 128 rows x 128 B
-constexpr int kBarBytes = 256;
+constexpr int kBarBytes = 512;
 constexpr int kSmem = 1024 + kQBytes + 2 * kKVBytes + 2 * kKVBytes + 2 * kPBytes + kBarBytes + 2 * 128 * 4 + 128 * 4;
 static_assert(kSmem <= 227 * 1024, "attention shared memory");
 constexpr uint32_t kTmemCols = 512;            // O: [0,256), S0: [256,320), S1: [320,384), Q: [384,512)
@@ -93,6 +93,18 @@ struct AttnParams {
   float scale_log2;  // scale * log2(e)
   uint64_t wait_ns;
   uint32_t* err;
+};
+
+// The fused launch's output projection (X += O . Wo^T over each document's rows).
+struct ProjParams {
+  __nv_bfloat16* x;   // residual stream [total_q][ldx], updated in place
+  int64_t ldx;
+  int hidden;         // N of the projection (multiple of 64)
+  int kdim;           // K of the projection = n_q * 256
+  int n_chunks;       // 256-column chunks of hidden
+  int m_tiles;        // 128-row tiles of max_q
+  int n_otiles;       // n_docs * m_tiles * n_chunks (tiles of rows past a document's end are skipped)
+  int* sync;          // [n_docs] per-document counters, [n_docs] tile-claim counter; zero between launches
 };
 
 // One work item: query tile t of KV head g of document d, with its extents.
@@ -147,10 +159,256 @@ __device__ __forceinline__ Item load_item(const AttnParams& p, int w) {
   return it;
 }
 
+// ------------------------------------------------------------------------------
+// Output projection phase of the fused decoder layer: X[rows of d] += O[rows of d] . Wo^T.
+// Tiles are (document, 128-row block, 256-column chunk); a CTA claims them from a
+// counter once its attention items are done and waits, per tile, for that document's
+// attention items (counted by the CTAs that computed them).  1-CTA tcgen05 GEMM:
+// warp 8 lane 0 claims tiles and loads A (O rows) and B (Wo rows) by TMA into a 4-deep
+// ring, warp 9 lane 0 issues M=128 x N=256 products into one of two TMEM
+// accumulators, warps 0-7 add the residual and write X (warp w: rows 32 (w % 4) ..,
+// columns 128 (w / 4) .. of the tile).
+constexpr int kGStages = 4;
+constexpr int kGABytes = kBM * 64 * 2;   // 128 rows x 64 k
+constexpr int kGBBytes = 256 * 64 * 2;   // 256 rows x 64 k
+constexpr int kGStageBytes = kGABytes + kGBBytes;
+constexpr uint32_t kIdescG = idesc_bf16_f32(kBM, 256, false, false);
+static_assert(kGStages * kGStageBytes + 8 * 4096 <= kQBytes + 4 * kKVBytes + 2 * kPBytes,
+              "projection ring and staging fit in the attention buffers");
+
+struct GemmBars {
+  uint64_t* full;       // [kGStages]
+  uint64_t* empty;      // [kGStages]
+  uint64_t* acc_full;   // [2]
+  uint64_t* acc_empty;  // [2] one arrival per epilogue warp
+  uint64_t* tq_full;    // [2] tile id published
+  uint64_t* tq_empty;   // [2] tile id slot free (one arrival per epilogue warp)
+  volatile int* tq;     // [2] tile ids (-1: no more)
+};
+
+__device__ __forceinline__ GemmBars gemm_bars(uint64_t* bars) {
+  return GemmBars{bars + 22, bars + 26, bars + 30, bars + 32, bars + 34, bars + 36,
+                  reinterpret_cast<volatile int*>(bars + 38)};
+}
+
+__device__ __forceinline__ void decode_otile(const ProjParams& f, int t, int& d, int& mi, int& ni) {
+  const int per_doc = f.m_tiles * f.n_chunks;
+  d = t / per_doc;
+  const int rem = t - d * per_doc;
+  mi = rem / f.n_chunks;
+  ni = rem - mi * f.n_chunks;
+}
+
+__device__ __forceinline__ void out_proj_phase(const AttnParams& p, const ProjParams& f, const CUtensorMap* tm_oa,
+                                               const CUtensorMap* tm_wo, uint8_t* smem, const GemmBars& gb,
+                                               uint32_t tmem, int warp, int lane, volatile int* abort_flag) {
+  int* claim = f.sync + p.n_docs;
+  const int kblocks = f.kdim / 64;
+  if (warp == kTmaWarp) {
+    if (lane != 0) return;
+    // ---------------------------------------------------- tile claims and A/B loads
+    tma_prefetch_desc(tm_oa);
+    tma_prefetch_desc(tm_wo);
+    int published = 0, stage = 0;
+    uint32_t phase = 0;
+    bool ok = true;
+    while (true) {
+      const int t = atomicAdd(claim, 1);
+      if (t == f.n_otiles + static_cast<int>(gridDim.x) - 1) atomicExch(claim, 0);  // the launch's last claim
+      int d = 0, mi = 0, ni = 0, lq = 0;
+      int id = -1;
+      if (t < f.n_otiles && ok && !*abort_flag) {
+        decode_otile(f, t, d, mi, ni);
+        lq = static_cast<int>(p.q_off[d + 1] - p.q_off[d]);
+        if (mi * kBM >= lq) continue;  // no rows of this document in the block
+        id = t;
+      }
+      // publish the tile (or the end) to the MMA and epilogue warps
+      const int k = published & 1;
+      if (published >= 2 && !mbar_wait(&gb.tq_empty[k], ((published - 2) >> 1) & 1, p.wait_ns)) {
+        record_error(p.err, kErrTimeout | kSiteAttention);
+        *abort_flag = 1;
+        ok = false;
+      }
+      gb.tq[k] = id;
+      mbar_arrive(&gb.tq_full[k]);
+      ++published;
+      if (id < 0) break;
+      if (!ok) continue;
+      // this document's attention items, computed by any CTA of the launch
+      const int items = p.n_kv * ((lq + p.P - 1) / p.P);
+      const int tiles_d = ((lq + kBM - 1) / kBM) * f.n_chunks;
+      const uint64_t t0 = globaltimer_ns();
+      while (ld_acquire_gpu(f.sync + d) < items) {
+        if (*abort_flag || globaltimer_ns() - t0 > p.wait_ns) {
+          record_error(p.err, kErrTimeout | kSiteAttention);
+          *abort_flag = 1;
+          ok = false;
+          break;
+        }
+      }
+      if (ok) {
+        // the document's last consumer puts its counter back to zero for the next launch
+        if (atomicAdd(f.sync + d, 1) == items + tiles_d - 1) atomicExch(f.sync + d, 0);
+      }
+      fence_proxy_async_global();  // O rows written by other CTAs, read below by TMA
+      const int32_t row0 = static_cast<int32_t>(p.q_off[d] + mi * kBM);
+      for (int kb = 0; kb < kblocks && ok; ++kb) {
+        if (!mbar_wait(&gb.empty[stage], phase ^ 1u, p.wait_ns)) {
+          record_error(p.err, kErrTimeout | kSiteAttention);
+          *abort_flag = 1;
+          ok = false;
+          break;
+        }
+        uint8_t* sa = smem + stage * kGStageBytes;
+        mbar_arrive_expect_tx(&gb.full[stage], kGStageBytes);
+        tma_load_2d(sa, tm_oa, &gb.full[stage], kb * 64, row0);
+        tma_load_2d(sa + kGABytes, tm_wo, &gb.full[stage], kb * 64, ni * 256);
+        if (++stage == kGStages) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+    }
+  } else if (warp == kMmaWarp) {
+    if (lane != 0) return;
+    // ---------------------------------------------------- products into TMEM
+    int k = 0, stage = 0, acc = 0;
+    uint32_t phase = 0, acc_phase = 0;
+    const uint32_t base = smem_u32(smem);
+    while (true) {
+      if (!mbar_wait(&gb.tq_full[k & 1], (k >> 1) & 1, p.wait_ns)) {
+        record_error(p.err, kErrTimeout | kSiteAttention);
+        *abort_flag = 1;
+        break;
+      }
+      const int id = gb.tq[k & 1];
+      ++k;
+      if (id < 0) break;
+      if (!mbar_wait(&gb.acc_empty[acc], acc_phase ^ 1u, p.wait_ns)) {
+        record_error(p.err, kErrTimeout | kSiteAttention);
+        *abort_flag = 1;
+        break;
+      }
+      tc_fence_after();
+      const uint32_t d_tmem = tmem + static_cast<uint32_t>(acc) * 256u;
+      bool ok = true;
+      for (int kb = 0; kb < kblocks; ++kb) {
+        if (!mbar_wait(&gb.full[stage], phase, p.wait_ns)) {
+          record_error(p.err, kErrTimeout | kSiteAttention);
+          *abort_flag = 1;
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint64_t ad0 = sdesc_sw128(base + stage * kGStageBytes, 16, 1024);
+        const uint64_t bd0 = sdesc_sw128(base + stage * kGStageBytes + kGABytes, 16, 1024);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          umma_bf16_ss(d_tmem, ad0 + static_cast<uint64_t>(kk * 2), bd0 + static_cast<uint64_t>(kk * 2), kIdescG,
+                       (kb | kk) != 0 ? 1u : 0u);
+        umma_commit(&gb.empty[stage]);
+        if (++stage == kGStages) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+      if (!ok) break;
+      umma_commit(&gb.acc_full[acc]);
+      acc ^= 1;
+      if (acc == 0) acc_phase ^= 1u;
+    }
+  } else if (warp < kSoftmaxThreads / 32) {
+    // ---------------------------------------------------- epilogue: + residual, bf16, X
+    const int quarter = warp & 3, half = warp >> 2;
+    uint8_t* stage_buf = smem + kGStages * kGStageBytes + warp * 4096;
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
+    int k = 0, acc = 0;
+    uint32_t acc_phase = 0;
+    while (true) {
+      bool wt = mbar_wait(&gb.tq_full[k & 1], (k >> 1) & 1, p.wait_ns);
+      if (!__all_sync(0xffffffffu, wt)) {
+        if (lane == 0) record_error(p.err, kErrTimeout | kSiteAttention);
+        *abort_flag = 1;
+        break;
+      }
+      const int id = gb.tq[k & 1];
+      const int kslot = k & 1;
+      ++k;
+      if (id < 0) break;
+      int d, mi, ni;
+      decode_otile(f, id, d, mi, ni);
+      const int64_t q0 = p.q_off[d];
+      const int lq = static_cast<int>(p.q_off[d + 1] - q0);
+      wt = mbar_wait(&gb.acc_full[acc], acc_phase, p.wait_ns);
+      if (!__all_sync(0xffffffffu, wt) || *abort_flag) {
+        if (lane == 0) record_error(p.err, kErrTimeout | kSiteAttention);
+        *abort_flag = 1;
+        break;
+      }
+      tc_fence_after();
+      const int rloc = mi * kBM + quarter * 32;  // first row of this warp, within the document
+#pragma unroll 1
+      for (int c = 0; c < 2; ++c) {
+        const int col0 = ni * 256 + half * 128 + c * 64;
+        uint32_t o[2][32];
+        tmem_ld32(lane_base + static_cast<uint32_t>(acc * 256 + half * 128 + c * 64), o[0]);
+        tmem_ld32(lane_base + static_cast<uint32_t>(acc * 256 + half * 128 + c * 64 + 32), o[1]);
+        tmem_ld_wait();
+        const bool row_ok = rloc + lane < lq && col0 < f.hidden;
+        uint4 vv[8];
+        const __nv_bfloat16* xr = f.x + (q0 + rloc + lane) * f.ldx + col0;
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          uint4 rv = make_uint4(0u, 0u, 0u, 0u);
+          if (row_ok) rv = *reinterpret_cast<const uint4*>(xr + u * 8);
+          const __nv_bfloat162* rh = reinterpret_cast<const __nv_bfloat162*>(&rv);
+          const uint32_t* oc = o[u >> 2] + (u & 3) * 8;
+          float f[8];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float2 r2 = __bfloat1622float2(rh[e]);
+            f[2 * e] = __uint_as_float(oc[2 * e]) + r2.x;
+            f[2 * e + 1] = __uint_as_float(oc[2 * e + 1]) + r2.y;
+          }
+          vv[u].x = pack_bf16x2(f[0], f[1]);
+          vv[u].y = pack_bf16x2(f[2], f[3]);
+          vv[u].z = pack_bf16x2(f[4], f[5]);
+          vv[u].w = pack_bf16x2(f[6], f[7]);
+        }
+        // staged (swizzled) and written row-major, 8 lanes per 128-byte row
+        uint8_t* row = stage_buf + lane * 128;
+#pragma unroll
+        for (int u = 0; u < 8; ++u) *reinterpret_cast<uint4*>(row + ((u ^ (lane & 7)) << 4)) = vv[u];
+        __syncwarp();
+        const int cu = lane & 7;
+#pragma unroll
+        for (int kq = 0; kq < 8; ++kq) {
+          const int rr = (lane >> 3) + 4 * kq;
+          const uint4 val = *reinterpret_cast<const uint4*>(stage_buf + rr * 128 + ((cu ^ (rr & 7)) << 4));
+          if (rloc + rr < lq && col0 < f.hidden)
+            *reinterpret_cast<uint4*>(f.x + (q0 + rloc + rr) * f.ldx + col0 + cu * 8) = val;
+        }
+        __syncwarp();
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(&gb.acc_empty[acc]);
+        mbar_arrive(&gb.tq_empty[kslot]);
+      }
+      acc ^= 1;
+      if (acc == 0) acc_phase ^= 1u;
+    }
+  }
+}
+
+template <bool FUSED>
 __global__ void __launch_bounds__(kThreads, 1)
     merged_attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_ks,
                             const __grid_constant__ CUtensorMap tm_vs, const __grid_constant__ CUtensorMap tm_kc,
-                            const __grid_constant__ CUtensorMap tm_vc, const AttnParams p) {
+                            const __grid_constant__ CUtensorMap tm_vc, const __grid_constant__ CUtensorMap tm_oa,
+                            const __grid_constant__ CUtensorMap tm_wo, const AttnParams p, const ProjParams f) {
   pdl_launch_dependents();
   pdl_wait_predecessor();  // q/K/V come from the previous kernel; offsets are read by every role
 
@@ -175,6 +433,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* bar_sfree = bars + 17;  // [2] S buffer loaded into registers by its softmax group (per tile parity)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 19);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  // fused output projection only: an item's O stores done (softmax warps) / counted (signaller)
+  uint64_t* bar_ostored = bars + 20;
+  uint64_t* bar_osig = bars + 21;
   float* l_part = reinterpret_cast<float*>(sP + 2 * kPBytes + kBarBytes);  // [2][128]
   // running max after the latest tile, per row: written by the tile's group, read by the next
   // tile's group after bar_m; the bar_m waits order every write after the previous read
@@ -196,6 +457,21 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(bar_l, kSoftmaxThreads);
     mbar_init(bar_ofree, kSoftmaxThreads);
     mbar_init(bar_sdone, 1);
+    if constexpr (FUSED) {
+      const GemmBars gb = gemm_bars(bars);
+      mbar_init(bar_ostored, kSoftmaxThreads / 32);
+      mbar_init(bar_osig, 1);
+      for (int i = 0; i < kGStages; ++i) {
+        mbar_init(&gb.full[i], 1);
+        mbar_init(&gb.empty[i], 1);
+      }
+      for (int i = 0; i < 2; ++i) {
+        mbar_init(&gb.acc_full[i], 1);
+        mbar_init(&gb.acc_empty[i], kSoftmaxThreads / 32);
+        mbar_init(&gb.tq_full[i], 1);
+        mbar_init(&gb.tq_empty[i], kSoftmaxThreads / 32);
+      }
+    }
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -281,6 +557,26 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int64_t jj = last_j; jj >= 0 && jj >= last_j - 1; --jj)
         mbar_wait(&bar_full[jj & 1], static_cast<uint32_t>(jj >> 1) & 1, p.wait_ns);
       if (q_issued > 0) mbar_wait(bar_q, (q_issued - 1) & 1, p.wait_ns);
+    } else if (FUSED && warp == kTmaWarpV && lane == 1) {  // (compiled out when not FUSED)
+      // Fused output projection: count each finished item for its document.  The softmax
+      // warps arrive once their O stores of the item are done; the release add then makes
+      // those stores visible, at gpu scope, to the CTA that projects the document.
+      int n_it = 0;
+      int wc = item_at(p, 0);
+      Item nxt = load_item(p, wc);
+      for (int pass = 0; wc != kNoMore; ++pass) {
+        const Item it = nxt;
+        wc = item_at(p, pass + 1);
+        nxt = load_item(p, wc);
+        if (it.nt == 0) continue;
+        if (!mbar_wait(bar_ostored, n_it & 1, p.wait_ns) || *abort_flag) {
+          fail_wait();
+          break;
+        }
+        red_release_gpu_add(f.sync + it.d, 1);
+        mbar_arrive(bar_osig);
+        ++n_it;
+      }
     }
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------ S issuer: Q copy and S = Q K^T
@@ -624,6 +920,20 @@ __global__ void __launch_bounds__(kThreads, 1)
         // natural-log softmax denominator in scaled-logit units
         p.lse[(it.q0 + pos) * p.n_q + head] = (m_run + log2f(l_tot)) * 0.69314718055994531f;
       }
+      if constexpr (FUSED) {
+        // this warp's O stores of the item are done; the signaller counts the item once all
+        // eight warps have arrived (and only after it counted the previous one: at most one
+        // item in flight on the barrier)
+        __syncwarp();
+        if (lane == 0) {
+          const bool ws = n_it == 0 || mbar_wait(bar_osig, (n_it - 1) & 1, p.wait_ns);
+          if (!ws) {
+            record_error(p.err, kErrTimeout | kSiteAttention);
+            *abort_flag = 1;
+          }
+          mbar_arrive(bar_ostored);
+        }
+      }
       J += it.nt;
       ++n_it;
     }
@@ -634,6 +944,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   tc_fence_before();
   __syncthreads();
+  if constexpr (FUSED) {
+    // every attention product, read and store of this CTA is done: the buffers and the
+    // tensor memory now serve the output projection
+    tc_fence_after();
+    out_proj_phase(p, f, &tm_oa, &tm_wo, smem, gemm_bars(bars), tmem, warp, lane, abort_flag);
+    tc_fence_before();
+    __syncthreads();
+  }
   if (warp == kMmaWarp) {
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
@@ -745,22 +1063,38 @@ __global__ void __launch_bounds__(kSchedThreads) attention_schedule_kernel(const
 }  // namespace
 
 kalm_status setup_attention_kernels() {
-  return check_cuda(cudaFuncSetAttribute(merged_attention_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem),
-                    "cudaFuncSetAttribute(merged_attention_kernel)");
+  kalm_status st = check_cuda(
+      cudaFuncSetAttribute(merged_attention_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem),
+      "cudaFuncSetAttribute(merged_attention_kernel)");
+  if (st != KALM_OK) return st;
+  return check_cuda(
+      cudaFuncSetAttribute(merged_attention_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem),
+      "cudaFuncSetAttribute(merged_attention_kernel<fused>)");
 }
 
 }  // namespace kalm
 
 using namespace kalm;
 
-extern "C" kalm_status kalm_merged_attention(const kalm_bf16* q, int64_t ldq, const kalm_bf16* k_self,
-                                             const kalm_bf16* v_self, int64_t ld_self, const kalm_bf16* k_cross,
-                                             const kalm_bf16* v_cross, int64_t ld_cross, const int64_t* q_off,
-                                             const int64_t* in_off, int64_t total_in, const int64_t* pool_off,
-                                             int32_t n_docs, int32_t max_q, int64_t total_q, int64_t total_pool,
-                                             int32_t n_q, int32_t n_kv, int32_t head_dim, float scale,
-                                             int32_t last_tile_only, const int32_t* order, kalm_bf16* out,
-                                             int64_t ldo, float* lse, kalm_stream_t stream) {
+namespace {
+
+// Output projection of the fused launch (kalm_merged_attention_out_proj); null: none.
+struct OutProj {
+  const kalm_bf16* w_o;
+  int64_t ldw;
+  kalm_bf16* x;
+  int64_t ldx;
+  int32_t hidden;
+  int32_t* sync;
+};
+
+kalm_status launch_attention(const kalm_bf16* q, int64_t ldq, const kalm_bf16* k_self, const kalm_bf16* v_self,
+                             int64_t ld_self, const kalm_bf16* k_cross, const kalm_bf16* v_cross, int64_t ld_cross,
+                             const int64_t* q_off, const int64_t* in_off, int64_t total_in, const int64_t* pool_off,
+                             int32_t n_docs, int32_t max_q, int64_t total_q, int64_t total_pool, int32_t n_q,
+                             int32_t n_kv, int32_t head_dim, float scale, int32_t last_tile_only,
+                             const int32_t* order, kalm_bf16* out, int64_t ldo, float* lse, const OutProj* op,
+                             kalm_stream_t stream) {
   kalm_status st = ensure_device(nullptr);
   if (st != KALM_OK) return st;
   if (head_dim != kD) return fail(KALM_ERR_UNSUPPORTED, "kalm_merged_attention: head_dim=%d (only 256)", head_dim);
@@ -838,9 +1172,85 @@ extern "C" kalm_status kalm_merged_attention(const kalm_bf16* q, int64_t ldq, co
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   if (sms <= 0) sms = 148;
   const int64_t grid = items < sms ? items : sms;  // persistent: one CTA per SM
-  return check_cuda(launch_pdl(merged_attention_kernel, dim3(static_cast<unsigned>(grid)), dim3(kThreads), kSmem,
-                                static_cast<cudaStream_t>(stream), tq, tks, tvs, tkc, tvc, prm),
-                    "launch merged_attention_kernel");
+  if (!op) {
+    return check_cuda(launch_pdl(merged_attention_kernel<false>, dim3(static_cast<unsigned>(grid)), dim3(kThreads),
+                                 kSmem, static_cast<cudaStream_t>(stream), tq, tks, tvs, tkc, tvc, tq, tq, prm,
+                                 ProjParams{}),
+                      "launch merged_attention_kernel");
+  }
+  // fused output projection: A = O rows of a document (the `out` written above), B = Wo
+  CUtensorMap toa, two;
+  {
+    const uint64_t dims[2] = {static_cast<uint64_t>(n_q) * kD, static_cast<uint64_t>(total_q)};
+    const uint64_t strides[1] = {static_cast<uint64_t>(ldo) * 2};
+    const uint32_t box[2] = {64, kBM};
+    if ((st = make_tmap_bf16(&toa, out, 2, dims, strides, box)) != KALM_OK) return st;
+  }
+  {
+    const uint64_t dims[2] = {static_cast<uint64_t>(n_q) * kD, static_cast<uint64_t>(op->hidden)};
+    const uint64_t strides[1] = {static_cast<uint64_t>(op->ldw) * 2};
+    const uint32_t box[2] = {64, 256};
+    if ((st = make_tmap_bf16(&two, op->w_o, 2, dims, strides, box)) != KALM_OK) return st;
+  }
+  ProjParams fp{};
+  fp.x = reinterpret_cast<__nv_bfloat16*>(op->x);
+  fp.ldx = op->ldx;
+  fp.hidden = op->hidden;
+  fp.kdim = n_q * kD;
+  fp.n_chunks = (op->hidden + 255) / 256;
+  fp.m_tiles = (max_q + kBM - 1) / kBM;
+  const int64_t otiles = static_cast<int64_t>(n_docs) * fp.m_tiles * fp.n_chunks;
+  if (otiles + grid > INT32_MAX) return fail(KALM_ERR_INVALID_ARG, "kalm_merged_attention_out_proj: too many tiles");
+  fp.n_otiles = static_cast<int>(otiles);
+  fp.sync = op->sync;
+  return check_cuda(launch_pdl(merged_attention_kernel<true>, dim3(static_cast<unsigned>(grid)), dim3(kThreads), kSmem,
+                               static_cast<cudaStream_t>(stream), tq, tks, tvs, tkc, tvc, toa, two, prm, fp),
+                    "launch merged_attention_kernel<fused>");
+}
+
+}  // namespace
+
+extern "C" kalm_status kalm_merged_attention(const kalm_bf16* q, int64_t ldq, const kalm_bf16* k_self,
+                                             const kalm_bf16* v_self, int64_t ld_self, const kalm_bf16* k_cross,
+                                             const kalm_bf16* v_cross, int64_t ld_cross, const int64_t* q_off,
+                                             const int64_t* in_off, int64_t total_in, const int64_t* pool_off,
+                                             int32_t n_docs, int32_t max_q, int64_t total_q, int64_t total_pool,
+                                             int32_t n_q, int32_t n_kv, int32_t head_dim, float scale,
+                                             int32_t last_tile_only, const int32_t* order, kalm_bf16* out,
+                                             int64_t ldo, float* lse, kalm_stream_t stream) {
+  return launch_attention(q, ldq, k_self, v_self, ld_self, k_cross, v_cross, ld_cross, q_off, in_off, total_in,
+                          pool_off, n_docs, max_q, total_q, total_pool, n_q, n_kv, head_dim, scale, last_tile_only,
+                          order, out, ldo, lse, nullptr, stream);
+}
+
+extern "C" int64_t kalm_attention_out_proj_sync_len(int32_t n_docs) {
+  return n_docs < 0 ? -1 : static_cast<int64_t>(n_docs) + 1;
+}
+
+extern "C" kalm_status kalm_merged_attention_out_proj(
+    const kalm_bf16* q, int64_t ldq, const kalm_bf16* k_self, const kalm_bf16* v_self, int64_t ld_self,
+    const kalm_bf16* k_cross, const kalm_bf16* v_cross, int64_t ld_cross, const int64_t* q_off, const int64_t* in_off,
+    int64_t total_in, const int64_t* pool_off, int32_t n_docs, int32_t max_q, int64_t total_q, int64_t total_pool,
+    int32_t n_q, int32_t n_kv, int32_t head_dim, float scale, const int32_t* order, kalm_bf16* out, int64_t ldo,
+    const kalm_bf16* w_o, int64_t ldw, kalm_bf16* x, int64_t ldx, int32_t hidden, int32_t* sync, int64_t sync_len,
+    kalm_stream_t stream) {
+  kalm_status st = ensure_device(nullptr);
+  if (st != KALM_OK) return st;
+  if (n_docs < 0 || hidden <= 0 || hidden % 64)
+    return fail(KALM_ERR_INVALID_ARG, "kalm_merged_attention_out_proj: hidden=%d must be a positive multiple of 64",
+                hidden);
+  if (n_docs == 0 || max_q == 0 || total_q == 0) return KALM_OK;
+  if (!w_o || !x || !sync) return fail(KALM_ERR_INVALID_ARG, "kalm_merged_attention_out_proj: NULL pointer");
+  if (sync_len < kalm_attention_out_proj_sync_len(n_docs))
+    return fail(KALM_ERR_INVALID_ARG, "kalm_merged_attention_out_proj: sync_len=%lld < %lld", (long long)sync_len,
+                (long long)kalm_attention_out_proj_sync_len(n_docs));
+  if ((reinterpret_cast<uintptr_t>(sync) & 3u) || !aligned16(w_o) || !aligned16(x) || ldw % 8 || ldx % 8 ||
+      ldw < static_cast<int64_t>(n_q) * head_dim || ldx < hidden)
+    return fail(KALM_ERR_INVALID_ARG, "kalm_merged_attention_out_proj: bad alignment or stride");
+  const OutProj op{w_o, ldw, x, ldx, hidden, sync};
+  return launch_attention(q, ldq, k_self, v_self, ld_self, k_cross, v_cross, ld_cross, q_off, in_off, total_in,
+                          pool_off, n_docs, max_q, total_q, total_pool, n_q, n_kv, head_dim, scale, 0, order, out, ldo,
+                          nullptr, &op, stream);
 }
 
 extern "C" int64_t kalm_attention_items(int32_t n_docs, int32_t max_q, int32_t n_q, int32_t n_kv,

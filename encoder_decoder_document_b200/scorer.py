@@ -25,7 +25,7 @@ import numpy as np
 import torch
 
 from . import (kalm_broadcast_rows, kalm_check_device_errors, kalm_chunk_pool, kalm_cross_kv_proj,
-               kalm_device_check, kalm_linear,
+               kalm_device_check, kalm_linear, kalm_merged_attention_out_proj, kalm_attention_out_proj_sync_len,
                kalm_merged_attention, kalm_ragged_offsets, kalm_yes_no_score, kalm_attention_items,
                kalm_attention_schedule, kalm_linear_rope, kalm_rope_table)
 
@@ -66,7 +66,7 @@ class FBNLScorer:
     (the readout reads nothing else)."""
 
     def __init__(self, weights: DeviceWeights, n_q: int, n_kv: int, chunk: int = 4, head_dim: int = HEAD_DIM,
-                 prune: bool = True, rope_theta: Optional[float] = None):
+                 prune: bool = True, rope_theta: Optional[float] = None, fused_out: bool = False):
         kalm_device_check()
         self.w = weights
         self.L, qkv_rows, self.H = weights.w_qkv.shape
@@ -75,6 +75,9 @@ class FBNLScorer:
         self.scale = head_dim ** -0.5
         self.prune = prune
         self.rope_theta = rope_theta  # rotary base for the decoder's self Q/K, or None (no rotation)
+        # attention and output projection of every layer but the pruned last one in one
+        # launch (kalm_merged_attention_out_proj)
+        self.fused_out = fused_out
         # the rotary angles' (cos, sin), built once for this base
         self.rope_tab = kalm_rope_table(rope_theta, head_dim) if rope_theta is not None else None
         self._shape = None
@@ -121,6 +124,8 @@ class FBNLScorer:
         self.order = torch.empty(max(kalm_attention_items(n_docs, lq, self.n_q, self.n_kv), 1), dtype=torch.int32,
                                  **kw)
         self.yes, self.no, self.margin, self.score = self.result[0], self.result[1], self.result[2], self.result[3]
+        # the fused layer's per-document counters (zero before a launch, left zero by it)
+        self.sync = torch.zeros(max(kalm_attention_out_proj_sync_len(n_docs), 1), dtype=torch.int32, **kw)
         self.graphs = None
         self.graphs_decode = None
 
@@ -204,8 +209,21 @@ class FBNLScorer:
         kalm_linear(self.o, self.w.w_o[l], self.x, residual=self.x)
         self._mark("o_proj")
 
+    def attention_out(self, l: int, q, ks, vs, in_off=None) -> None:
+        """Fused attention + output projection of layer l (X updated in place)."""
+        kc, vc = self.cross_views(l)
+        self._join_side()
+        kalm_merged_attention_out_proj(q, ks, vs, kc, vc, self.q_off, self.pool_off, self.lq, self.n_q, self.n_kv,
+                                       self.o, self.w.w_o[l], self.x, self.sync, self.scale, in_off=in_off,
+                                       order=self.order)
+        self._mark("attention_out_proj")
+
     def layer(self, l: int) -> None:
         self.layer_qkv(l)
+        if self.fused_out:
+            q, ks, vs = self.qkv_views()
+            self.attention_out(l, q, ks, vs)
+            return
         self.layer_attention(l)
         self.layer_out(l)
 
@@ -223,6 +241,9 @@ class FBNLScorer:
             self.layer_qkv(l)
             q, ks, vs = self.qkv_views()
             in_off = None
+        if self.fused_out and not last:
+            self.attention_out(l, q, ks, vs, in_off)
+            return
         kalm_merged_attention(q, ks, vs, kc, vc, self.q_off, self.pool_off, Lq, self.n_q, self.n_kv, self.o,
                               self.scale, in_off=in_off, last_tile_only=last, order=None if last else self.order)
         self._mark("merged_attention")

@@ -228,6 +228,51 @@ kalm_status kalm_merged_attention(const kalm_bf16* q, int64_t ldq,
                                   int32_t last_tile_only, const int32_t* order,
                                   kalm_bf16* out, int64_t ldo, float* lse, kalm_stream_t stream);
 
+/* Step 3 followed by the decoder's output projection in one launch (a fused decoder
+ * layer).  "KaLM-Reranker-V1-Nano - MLX", "What this is": the decoder's merged
+ * self + cross attention, whose output goes back through the output projection onto
+ * the residual stream (the synthetic attention-only decoder: X <- X + Attn(...) . Wo).
+ *
+ * Computes exactly what kalm_merged_attention (last_tile_only = 0, lse = NULL) writes
+ * to `out`, and then, for every document, X[rows of d] += out[rows of d] . w_o^T with
+ * one bf16 rounding (as kalm_linear with residual = x, in place).  Inside the launch
+ * each CTA first computes its attention work items; the projection tiles (document x
+ * 128 rows x 256 columns) are then claimed by the CTAs as they finish, and a tile waits
+ * only for its own document's attention items, so the projection fills the tail of the
+ * attention.
+ *
+ * Arguments up to `ldo`: as kalm_merged_attention (q_off, in_off, pool_off, order, out
+ *          ... with the same requirements; `order` must come from kalm_attention_schedule
+ *          for the same sizes, or be NULL).
+ * w_o      [hidden][ldw] bf16, the output projection in the nn.Linear layout [out][in],
+ *          in = n_q * head_dim
+ * x        [total_q][ldx] bf16, the residual stream, updated in place
+ * hidden   multiple of 64
+ * sync     int32 device array of sync_len >= kalm_attention_out_proj_sync_len(n_docs)
+ *          entries: the launch's per-document completion counters and its tile counter.
+ *          Caller-owned; must be zero before the first call (e.g. cudaMemset), and every
+ *          call leaves it zero again.  Launches that share one array must not overlap on
+ *          the GPU.  After a call that recorded a device error, zero it again.
+ * Errors: as kalm_merged_attention; NULL w_o/x/sync, hidden not a multiple of 64, a
+ *          short sync array, misaligned pointers or strides -> KALM_ERR_INVALID_ARG.  A
+ *          wait on another CTA's items that runs out its bound is recorded in the device
+ *          error word (timeout). */
+kalm_status kalm_merged_attention_out_proj(const kalm_bf16* q, int64_t ldq,
+                                           const kalm_bf16* k_self, const kalm_bf16* v_self, int64_t ld_self,
+                                           const kalm_bf16* k_cross, const kalm_bf16* v_cross, int64_t ld_cross,
+                                           const int64_t* q_off, const int64_t* in_off, int64_t total_in,
+                                           const int64_t* pool_off, int32_t n_docs, int32_t max_q,
+                                           int64_t total_q, int64_t total_pool,
+                                           int32_t n_q, int32_t n_kv, int32_t head_dim, float scale,
+                                           const int32_t* order, kalm_bf16* out, int64_t ldo,
+                                           const kalm_bf16* w_o, int64_t ldw, kalm_bf16* x, int64_t ldx,
+                                           int32_t hidden, int32_t* sync, int64_t sync_len,
+                                           kalm_stream_t stream);
+
+/* Entries of the sync array kalm_merged_attention_out_proj needs for n_docs documents
+ * (n_docs + 1), or -1 for n_docs < 0.  Host-only arithmetic. */
+int64_t kalm_attention_out_proj_sync_len(int32_t n_docs);
+
 /* Work items of one kalm_merged_attention call (one query tile of 128/(n_q/n_kv)
  * decoder positions x one KV head x one document): ceil(max_q / (128 n_kv / n_q))
  * * n_docs * n_kv, or n_docs * n_kv with last_tile_only.  Host-only

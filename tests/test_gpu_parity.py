@@ -115,6 +115,71 @@ def test_chunk_pool_edge_lengths_padded_and_strided(kalm):
 # ---------------------------------------------------------------------------
 # step 2: projections
 # ---------------------------------------------------------------------------
+@pytest.mark.parametrize("lq,nc,n_q,n_kv,hidden", [
+    ([128] * 3, [40, 0, 256], 4, 1, 640),       # Nano shape, an empty cross segment
+    ([200, 200], [17, 90], 4, 1, 1152),         # Small hidden: a 128-column last chunk, a partial row block
+    ([256, 256], [30, 77], 8, 4, 2560),         # Large heads and hidden (K = 2048, 10 column chunks)
+    ([37, 37, 37, 37], [5, 64, 65, 1], 4, 1, 640),
+    ([512, 3], [256, 2], 4, 1, 640),            # the query budget beside a 3-row document
+])
+def test_attention_out_proj_fused(kalm, lq, nc, n_q, n_kv, hidden):
+    """The fused decoder layer: `out` equals the attention kernel's output bit for bit, and
+    X + out . Wo^T equals the oracle's projection with residual within one bf16 step; the
+    per-document counters are left at zero, so a second launch gives the same result."""
+    D = 256
+    rng = np.random.default_rng(sum(lq) + hidden)
+    a = _attn_arrays(rng, lq, nc, n_q, n_kv)
+    q_off, p_off = a["q_off"], a["p_off"]
+    R, C = int(q_off[-1]), max(int(p_off[-1]), 1)
+    kc = a["kc"] if a["kc"].shape[0] else np.zeros((1, n_kv, D))
+    vc = a["vc"] if a["vc"].shape[0] else np.zeros((1, n_kv, D))
+    qkv = torch.cat([f64_to_dev(a["q"].reshape(R, -1)), f64_to_dev(a["ks"].reshape(R, -1)),
+                     f64_to_dev(a["vs"].reshape(R, -1))], 1)
+    kvc = torch.cat([f64_to_dev(kc.reshape(C, -1)), f64_to_dev(vc.reshape(C, -1))], 1)
+    w = n_kv * D
+    views = (qkv[:, : n_q * D], qkv[:, n_q * D: n_q * D + w], qkv[:, n_q * D + w:], kvc[:, :w], kvc[:, w:])
+    max_q = int(np.diff(q_off).max())
+    w_o = rand_bf16(rng, (hidden, n_q * D), 0.02)
+    x0 = rand_bf16(rng, (R, hidden))
+    order = torch.empty(kalm.kalm_attention_items(len(lq), max_q, n_q, n_kv), dtype=torch.int32, device="cuda")
+    kalm.kalm_attention_schedule(i64(q_off), i64(p_off), max_q, n_q, n_kv, order)
+    ref = torch.full((R, n_q * D), float("nan"), dtype=torch.bfloat16, device="cuda")
+    kalm.kalm_merged_attention(*views, i64(q_off), i64(p_off), max_q, n_q, n_kv, ref, 1.0 / 16, order=order)
+    sync = torch.zeros(kalm.kalm_attention_out_proj_sync_len(len(lq)), dtype=torch.int32, device="cuda")
+    results = []
+    for rep, use_order in ((0, True), (1, True), (2, False)):
+        out = torch.full((R, n_q * D), float("nan"), dtype=torch.bfloat16, device="cuda")
+        x = f64_to_dev(x0)
+        kalm.kalm_merged_attention_out_proj(*views, i64(q_off), i64(p_off), max_q, n_q, n_kv, out, f64_to_dev(w_o), x,
+                                            sync, 1.0 / 16, order=order if use_order else None)
+        kalm.kalm_check_device_errors()
+        assert torch.equal(out.view(torch.int16), ref.view(torch.int16))
+        assert int(sync.abs().sum()) == 0  # counters back at zero
+        results.append(from_dev(x))
+    o = from_dev(ref)
+    _one_step(results[0], oracle.linear(o, w_o, residual=x0), o, w_o, x0)
+    np.testing.assert_array_equal(results[0], results[1])
+    np.testing.assert_array_equal(results[0], results[2])
+
+
+def test_attention_out_proj_rejects_bad_arguments(kalm):
+    from encoder_decoder_document_b200 import KalmError
+    a = _attn_arrays(np.random.default_rng(3), [32], [4], 4, 1)
+    t = lambda n: torch.zeros(n, 256, dtype=torch.bfloat16, device="cuda")
+    q, kv, kc = t(32 * 4).view(32, 1024), t(32), t(4)
+    x = torch.zeros(32, 640, dtype=torch.bfloat16, device="cuda")
+    w_o = torch.zeros(640, 1024, dtype=torch.bfloat16, device="cuda")
+    out = torch.zeros(32, 1024, dtype=torch.bfloat16, device="cuda")
+    ok_sync = torch.zeros(2, dtype=torch.int32, device="cuda")
+    args = (q, kv, kv, kc, kc, i64(a["q_off"]), i64(a["p_off"]), 32, 4, 1, out)
+    with pytest.raises(KalmError):  # sync array too short
+        kalm.kalm_merged_attention_out_proj(*args, w_o, x, torch.zeros(1, dtype=torch.int32, device="cuda"))
+    with pytest.raises(KalmError):  # hidden not a multiple of 64
+        kalm.kalm_merged_attention_out_proj(*args, w_o[:600], x[:, :600], ok_sync)
+    kalm.kalm_merged_attention_out_proj(*args, w_o, x, ok_sync)
+    kalm.kalm_check_device_errors()
+
+
 def _one_step(got, want, x=None, w=None, r=None):
     """GPU projection vs the oracle's bf16 value.
 
@@ -427,6 +492,33 @@ def test_end_to_end_large_heads_and_maximum_lengths(kalm, name, kw):
         res = sc.scores_to_host().numpy()
         assert np.all(np.isfinite(res))
         _check_scores(res[3], s, m)
+
+
+@pytest.mark.parametrize("name,kw,docs", [("tiny", {}, None), ("nano", dict(layers=4), [0, 31, 77, 99])])
+def test_end_to_end_fused_layers(kalm, name, kw, docs):
+    """Scores with every layer but the last run as one fused attention + output projection
+    launch, eagerly and in the graph, against the oracle (and equal to the unfused stack's
+    scores within the score tolerance)."""
+    from encoder_decoder_document_b200.scorer import DeviceWeights, FBNLScorer
+    q = synthetic.make_query(name, **kw)
+    y, n, m, s = oracle.forward_query(q, docs=docs)
+    for graph in (False, True):
+        sc = FBNLScorer(DeviceWeights.from_bits(q.weights), q.n_q, q.n_kv, fused_out=True)
+        if graph:
+            total_pooled = int(oracle.pooled_counts(q.doc_len).sum())
+            sc.prepare(q.n_docs, int(q.doc_len.sum()), total_pooled, q.lq)
+            sc.load_inputs(torch.from_numpy(q.enc.view(np.int16)).view(torch.bfloat16), torch.from_numpy(q.doc_len),
+                           torch.from_numpy(q.x0.view(np.int16)).view(torch.bfloat16))
+            sc.capture()
+            for _ in range(3):  # replays reuse the counters
+                sc.run()
+        else:
+            sc.rerank(q.x0, q.enc, q.doc_len)
+        kalm.kalm_check_device_errors()
+        res = sc.scores_to_host().numpy()
+        got = res[3] if docs is None else res[3][docs]
+        _check_scores(got, s, m)
+        assert int(sc.sync.abs().sum()) == 0
 
 
 def test_end_to_end_tiny_batch_composition(kalm):
