@@ -17,7 +17,7 @@ from ._abi import KalmError, call, load, library_path  # noqa: F401
 __all__ = [
     "KalmError", "load", "library_path", "kalm_version", "kalm_device_check", "kalm_check_device_errors",
     "kalm_ragged_offsets", "kalm_chunk_pool", "kalm_linear", "kalm_cross_kv_proj", "kalm_merged_attention",
-    "kalm_merged_attention_out_proj", "kalm_attention_out_proj_sync_len",
+    "kalm_merged_attention_out_proj", "kalm_merged_attention_out_proj_static", "kalm_attention_out_proj_sync_len",
     "kalm_yes_no_score", "kalm_broadcast_rows", "kalm_selftest_wait_timeout", "kalm_attention_items",
     "kalm_attention_schedule", "kalm_rope", "kalm_rope_table", "kalm_linear_rope",
 ]
@@ -145,6 +145,30 @@ def kalm_merged_attention_out_proj(q: torch.Tensor, k_self: torch.Tensor, v_self
          n_docs, int(max_q), int(total_q), k_cross.shape[0], n_q, n_kv, head_dim, float(scale),
          _p(order, torch.int32), _p(out, torch.bfloat16), _ld(out), _p(w_o, torch.bfloat16), _ld(w_o),
          _p(x, torch.bfloat16), _ld(x), x.shape[1], _p(sync, torch.int32), sync.numel(), _stream(stream))
+
+
+def kalm_merged_attention_out_proj_static(q: torch.Tensor, k_self: torch.Tensor, v_self: torch.Tensor,
+                                          k_cross: torch.Tensor, v_cross: torch.Tensor, q_off: torch.Tensor,
+                                          pool_off: torch.Tensor, max_q: int, n_q: int, n_kv: int,
+                                          out: torch.Tensor, w_o: torch.Tensor, x: torch.Tensor,
+                                          scale: Optional[float] = None, head_dim: int = HEAD_DIM,
+                                          in_off: Optional[torch.Tensor] = None, total_q: Optional[int] = None,
+                                          order: Optional[torch.Tensor] = None, stream=None) -> None:
+    """kalm_merged_attention_out_proj with the library's built-in counters (no counter
+    array from the caller): for callers that cannot allocate device memory.  At most
+    KALM_OUT_PROJ_STATIC_MAX_DOCS (4096) documents; calls that overlap on the GPU race."""
+    if scale is None:
+        scale = head_dim ** -0.5
+    if _ld(k_self) != _ld(v_self) or _ld(k_cross) != _ld(v_cross):
+        raise KalmError(1, "kalm_merged_attention_out_proj_static", "K and V views must share a row stride")
+    n_docs = q_off.numel() - 1
+    total_q = out.shape[0] if total_q is None else total_q
+    call("kalm_merged_attention_out_proj_static", _p(q, torch.bfloat16), _ld(q), _p(k_self, torch.bfloat16),
+         _p(v_self, torch.bfloat16), _ld(k_self), _p(k_cross, torch.bfloat16), _p(v_cross, torch.bfloat16),
+         _ld(k_cross), _p(q_off, torch.int64), _p(in_off, torch.int64), q.shape[0], _p(pool_off, torch.int64),
+         n_docs, int(max_q), int(total_q), k_cross.shape[0], n_q, n_kv, head_dim, float(scale),
+         _p(order, torch.int32), _p(out, torch.bfloat16), _ld(out), _p(w_o, torch.bfloat16), _ld(w_o),
+         _p(x, torch.bfloat16), _ld(x), x.shape[1], _stream(stream))
 
 
 def kalm_attention_out_proj_sync_len(n_docs: int) -> int:

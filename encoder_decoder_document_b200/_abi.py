@@ -37,6 +37,9 @@ SIGNATURES = {
                                        c_i32, c_i32, c_i64, c_i64, c_i32, c_i32, c_i32, c_f32, c_vp, c_vp, c_i64,
                                        c_vp, c_i64, c_vp, c_i64, c_i32, c_vp, c_i64, c_vp],
     "kalm_attention_out_proj_sync_len": [c_i32],
+    "kalm_merged_attention_out_proj_static": [c_vp, c_i64, c_vp, c_vp, c_i64, c_vp, c_vp, c_i64, c_vp, c_vp, c_i64,
+                                              c_vp, c_i32, c_i32, c_i64, c_i64, c_i32, c_i32, c_i32, c_f32, c_vp, c_vp,
+                                              c_i64, c_vp, c_i64, c_vp, c_i64, c_i32, c_vp],
     "kalm_attention_items": [c_i32, c_i32, c_i32, c_i32, c_i32],
     "kalm_attention_schedule": [c_vp, c_vp, c_i32, c_i32, c_i32, c_i32, c_i32, c_vp, c_i64, c_vp],
     "kalm_yes_no_score": [c_vp, c_i64, c_vp, c_i32, c_i32, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp],

@@ -43,6 +43,7 @@
 //     next tiles goes out while P V waits for the softmax, so the tensor pipe does
 //     not idle behind one thread's waits.
 #include <cmath>
+#include <mutex>
 
 #include "kalm.h"
 #include "kalm_internal.h"
@@ -1251,6 +1252,64 @@ extern "C" kalm_status kalm_merged_attention_out_proj(
   return launch_attention(q, ldq, k_self, v_self, ld_self, k_cross, v_cross, ld_cross, q_off, in_off, total_in,
                           pool_off, n_docs, max_q, total_q, total_pool, n_q, n_kv, head_dim, scale, 0, order, out, ldo,
                           nullptr, &op, stream);
+}
+
+// ----------------------------------------------------------------------------------
+// The fused layer for callers that cannot allocate device memory.  Its counters live in a
+// fixed array in the library's own device memory instead of a caller-provided buffer:
+// every device that loads the library holds the array (16 KB) until the process exits.
+namespace {
+
+constexpr int kStaticSyncDocs = KALM_OUT_PROJ_STATIC_MAX_DOCS;  // documents per call the built-in counters hold
+static __device__ __align__(256) int32_t g_out_proj_sync[kStaticSyncDocs + 1];
+
+// Device address of g_out_proj_sync, looked up once per device (host code only sees a
+// stand-in symbol, not a device address).
+std::mutex g_static_sync_mutex;
+int32_t* g_static_sync_ptr[64] = {};
+
+kalm_status static_sync_ptr(int dev, int32_t** out) {
+  if (dev < 0 || dev >= 64) return fail(KALM_ERR_NO_DEVICE, "device index %d out of range", dev);
+  std::lock_guard<std::mutex> lock(g_static_sync_mutex);
+  if (!g_static_sync_ptr[dev]) {
+    void* ptr = nullptr;
+    kalm_status st = check_cuda(cudaGetSymbolAddress(&ptr, g_out_proj_sync), "cudaGetSymbolAddress(out-proj counters)");
+    if (st != KALM_OK) return st;
+    g_static_sync_ptr[dev] = static_cast<int32_t*>(ptr);
+  }
+  *out = g_static_sync_ptr[dev];
+  return KALM_OK;
+}
+
+}  // namespace
+
+extern "C" kalm_status kalm_merged_attention_out_proj_static(
+    const kalm_bf16* q, int64_t ldq, const kalm_bf16* k_self, const kalm_bf16* v_self, int64_t ld_self,
+    const kalm_bf16* k_cross, const kalm_bf16* v_cross, int64_t ld_cross, const int64_t* q_off, const int64_t* in_off,
+    int64_t total_in, const int64_t* pool_off, int32_t n_docs, int32_t max_q, int64_t total_q, int64_t total_pool,
+    int32_t n_q, int32_t n_kv, int32_t head_dim, float scale, const int32_t* order, kalm_bf16* out, int64_t ldo,
+    const kalm_bf16* w_o, int64_t ldw, kalm_bf16* x, int64_t ldx, int32_t hidden, kalm_stream_t stream) {
+  int dev = -1;
+  kalm_status st = ensure_device(&dev);
+  if (st != KALM_OK) return st;
+  if (n_docs > kStaticSyncDocs)
+    return fail(KALM_ERR_INVALID_ARG,
+                "kalm_merged_attention_out_proj_static: n_docs=%d is above the %d documents its built-in counters "
+                "hold (pass a counter array to kalm_merged_attention_out_proj instead)",
+                n_docs, kStaticSyncDocs);
+  if (n_docs < 0) return fail(KALM_ERR_INVALID_ARG, "kalm_merged_attention_out_proj_static: n_docs=%d", n_docs);
+  int32_t* sync = nullptr;
+  if ((st = static_sync_ptr(dev, &sync)) != KALM_OK) return st;
+  // the counters must start at zero: clear the part this call uses (a call cut short by a
+  // device error may have left values behind)
+  const int64_t len = kalm_attention_out_proj_sync_len(n_docs);
+  st = check_cuda(cudaMemsetAsync(sync, 0, static_cast<size_t>(len) * sizeof(int32_t),
+                                  static_cast<cudaStream_t>(stream)),
+                  "clear out-proj counters");
+  if (st != KALM_OK) return st;
+  return kalm_merged_attention_out_proj(q, ldq, k_self, v_self, ld_self, k_cross, v_cross, ld_cross, q_off, in_off,
+                                        total_in, pool_off, n_docs, max_q, total_q, total_pool, n_q, n_kv, head_dim,
+                                        scale, order, out, ldo, w_o, ldw, x, ldx, hidden, sync, len, stream);
 }
 
 extern "C" int64_t kalm_attention_items(int32_t n_docs, int32_t max_q, int32_t n_q, int32_t n_kv,

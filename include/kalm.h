@@ -269,6 +269,35 @@ kalm_status kalm_merged_attention_out_proj(const kalm_bf16* q, int64_t ldq,
                                            int32_t hidden, int32_t* sync, int64_t sync_len,
                                            kalm_stream_t stream);
 
+/* kalm_merged_attention_out_proj without the caller's counter array, for callers that
+ * cannot allocate device memory: code that only receives tensors from a host program
+ * that owns every allocation (an inference server with its own pooled allocator, or an
+ * embedding that forbids allocation while it serves), and C callers with no allocator
+ * of their own.  The pages have no counterpart; this is an interface convenience.
+ *
+ * Same arguments, results and errors as kalm_merged_attention_out_proj, minus sync and
+ * sync_len.  The counters live in a fixed array inside the library's device memory,
+ * sized for KALM_OUT_PROJ_STATIC_MAX_DOCS documents: every device that loads the library
+ * holds it (16 KB) until the process exits.  More documents -> KALM_ERR_INVALID_ARG.
+ * Nothing is allocated: the call clears the counters it uses with an asynchronous
+ * memset on `stream` and launches the fused kernel.
+ * - The first call on a device looks up the array's device address (a runtime query);
+ *   make that first call before any stream capture.
+ * - Every call on a device shares the one array, and it keeps the last call's contents:
+ *   calls whose work overlaps on the GPU (other streams, other host threads) race on it;
+ *   order them on one stream. */
+#define KALM_OUT_PROJ_STATIC_MAX_DOCS 4096
+kalm_status kalm_merged_attention_out_proj_static(const kalm_bf16* q, int64_t ldq,
+                                                  const kalm_bf16* k_self, const kalm_bf16* v_self, int64_t ld_self,
+                                                  const kalm_bf16* k_cross, const kalm_bf16* v_cross, int64_t ld_cross,
+                                                  const int64_t* q_off, const int64_t* in_off, int64_t total_in,
+                                                  const int64_t* pool_off, int32_t n_docs, int32_t max_q,
+                                                  int64_t total_q, int64_t total_pool,
+                                                  int32_t n_q, int32_t n_kv, int32_t head_dim, float scale,
+                                                  const int32_t* order, kalm_bf16* out, int64_t ldo,
+                                                  const kalm_bf16* w_o, int64_t ldw, kalm_bf16* x, int64_t ldx,
+                                                  int32_t hidden, kalm_stream_t stream);
+
 /* Entries of the sync array kalm_merged_attention_out_proj needs for n_docs documents
  * (n_docs + 1), or -1 for n_docs < 0.  Host-only arithmetic. */
 int64_t kalm_attention_out_proj_sync_len(int32_t n_docs);

@@ -1,0 +1,75 @@
+"""The fused decoder layer's entry point that allocates nothing.
+
+kalm_merged_attention_out_proj_static serves callers that cannot allocate device memory
+(a host program that owns every allocation, a C caller with no allocator): it keeps its
+per-document counters in a fixed array inside the library instead of a caller-provided
+one.  This checks, through the C ABI, that two calls in a row give what the entry point
+with a caller-provided counter array gives, within the tolerances of the other GPU tests.
+The file is named so that pytest collects it last; it also passes alone.
+"""
+import numpy as np
+import pytest
+import torch
+
+pytestmark = pytest.mark.gpu
+
+D = 256
+
+
+def _inputs(seed=7, lq=(128, 128, 100, 128), nc=(40, 0, 97, 256), n_q=4, n_kv=1, hidden=640):
+    g = torch.Generator(device="cuda").manual_seed(seed)
+    q_off = np.concatenate([[0], np.cumsum(lq)])
+    p_off = np.concatenate([[0], np.cumsum(nc)])
+    R, C = int(q_off[-1]), max(int(p_off[-1]), 1)
+    rnd = lambda *shape, std=1.0: (torch.randn(*shape, device="cuda", generator=g) * std).to(torch.bfloat16)
+    qkv = rnd(R, (n_q + 2 * n_kv) * D, std=0.5)
+    kvc = rnd(C, 2 * n_kv * D, std=0.5)
+    w = n_kv * D
+    views = (qkv[:, : n_q * D], qkv[:, n_q * D: n_q * D + w], qkv[:, n_q * D + w:], kvc[:, :w], kvc[:, w:])
+    dev = lambda a: torch.as_tensor(np.asarray(a, dtype=np.int64)).cuda()
+    return dict(views=views, q_off=dev(q_off), p_off=dev(p_off), max_q=max(lq), n_q=n_q, n_kv=n_kv, R=R,
+                w_o=rnd(hidden, n_q * D, std=0.02), x0=rnd(R, hidden), n_docs=len(lq))
+
+
+def _bf16_step_bound(want):
+    """One bf16 rounding step of each value (the projections' tolerance in the parity tests)."""
+    return torch.abs(want.float()) * 2.0 ** -7 + 1e-30
+
+
+def test_no_alloc_entry_point_matches_caller_counters():
+    import encoder_decoder_document_b200 as k
+    from encoder_decoder_document_b200 import _build
+    _build.build()
+    k.kalm_device_check()
+    a = _inputs()
+    args = (*a["views"], a["q_off"], a["p_off"], a["max_q"], a["n_q"], a["n_kv"])
+    # reference: the entry point with a counter array from the caller
+    sync = torch.zeros(k.kalm_attention_out_proj_sync_len(a["n_docs"]), dtype=torch.int32, device="cuda")
+    ref_out = torch.empty(a["R"], a["n_q"] * D, dtype=torch.bfloat16, device="cuda")
+    ref_x = a["x0"].clone()
+    k.kalm_merged_attention_out_proj(*args, ref_out, a["w_o"], ref_x, sync, 1.0 / 16)
+    k.kalm_check_device_errors()
+    for _ in range(2):  # two calls in a row share the built-in counters
+        out = torch.full_like(ref_out, float("nan"))
+        x = a["x0"].clone()
+        k.kalm_merged_attention_out_proj_static(*args, out, a["w_o"], x, 1.0 / 16)
+        k.kalm_check_device_errors()
+        # attention output: the same kernel on the same inputs (within the attention tolerance, in fact equal)
+        assert torch.abs(out.float() - ref_out.float()).max().item() <= 2e-2
+        # projected residual stream: within one bf16 step of the reference
+        assert bool((torch.abs(x.float() - ref_x.float()) <= _bf16_step_bound(ref_x)).all())
+
+
+def test_no_alloc_entry_point_rejects_too_many_documents():
+    import encoder_decoder_document_b200 as k
+    from encoder_decoder_document_b200 import KalmError
+    n = 4097  # one more document than the built-in counters hold
+    t = torch.zeros(n, D, dtype=torch.bfloat16, device="cuda")
+    q = torch.zeros(n, 4 * D, dtype=torch.bfloat16, device="cuda")
+    offs = torch.arange(n + 1, dtype=torch.int64, device="cuda")
+    x = torch.zeros(n, 640, dtype=torch.bfloat16, device="cuda")
+    w_o = torch.zeros(640, 4 * D, dtype=torch.bfloat16, device="cuda")
+    out = torch.zeros(n, 4 * D, dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(KalmError) as e:
+        k.kalm_merged_attention_out_proj_static(q, t, t, t, t, offs, offs, 1, 4, 1, out, w_o, x)
+    assert e.value.name == "KALM_ERR_INVALID_ARG"
