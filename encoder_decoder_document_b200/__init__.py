@@ -131,7 +131,7 @@ def kalm_merged_attention_out_proj(q: torch.Tensor, k_self: torch.Tensor, v_self
                                    order: Optional[torch.Tensor] = None, stream=None) -> None:
     """Merged attention into ``out`` and then ``x[rows of d] += out[rows of d] . w_o^T`` for
     every document, in one launch.  ``sync``: int32 device tensor of at least
-    ``kalm_attention_out_proj_sync_len(n_docs)`` entries, zero before the first call
+    ``kalm_attention_out_proj_sync_len(n_docs, max_q, hidden)`` entries, zero before the first call
     (every call leaves it zero)."""
     if scale is None:
         scale = head_dim ** -0.5
@@ -156,7 +156,8 @@ def kalm_merged_attention_out_proj_static(q: torch.Tensor, k_self: torch.Tensor,
                                           order: Optional[torch.Tensor] = None, stream=None) -> None:
     """kalm_merged_attention_out_proj with the library's built-in counters (no counter
     array from the caller): for callers that cannot allocate device memory.  At most
-    KALM_OUT_PROJ_STATIC_MAX_DOCS (4096) documents; calls that overlap on the GPU race."""
+    KALM_OUT_PROJ_STATIC_MAX_DOCS (4096) documents and KALM_OUT_PROJ_STATIC_MAX_TILES (49152)
+    projection tiles; calls that overlap on the GPU race."""
     if scale is None:
         scale = head_dim ** -0.5
     if _ld(k_self) != _ld(v_self) or _ld(k_cross) != _ld(v_cross):
@@ -171,9 +172,9 @@ def kalm_merged_attention_out_proj_static(q: torch.Tensor, k_self: torch.Tensor,
          _p(x, torch.bfloat16), _ld(x), x.shape[1], _stream(stream))
 
 
-def kalm_attention_out_proj_sync_len(n_docs: int) -> int:
-    """Entries of the sync array kalm_merged_attention_out_proj needs for n_docs documents."""
-    return int(load().kalm_attention_out_proj_sync_len(n_docs))
+def kalm_attention_out_proj_sync_len(n_docs: int, max_q: int, hidden: int) -> int:
+    """Entries of the sync array kalm_merged_attention_out_proj needs (-1 for bad sizes)."""
+    return int(load().kalm_attention_out_proj_sync_len(n_docs, max_q, hidden))
 
 
 def kalm_attention_items(n_docs: int, max_q: int, n_q: int, n_kv: int, last_tile_only: bool = False) -> int:

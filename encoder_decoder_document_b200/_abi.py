@@ -36,7 +36,7 @@ SIGNATURES = {
     "kalm_merged_attention_out_proj": [c_vp, c_i64, c_vp, c_vp, c_i64, c_vp, c_vp, c_i64, c_vp, c_vp, c_i64, c_vp,
                                        c_i32, c_i32, c_i64, c_i64, c_i32, c_i32, c_i32, c_f32, c_vp, c_vp, c_i64,
                                        c_vp, c_i64, c_vp, c_i64, c_i32, c_vp, c_i64, c_vp],
-    "kalm_attention_out_proj_sync_len": [c_i32],
+    "kalm_attention_out_proj_sync_len": [c_i32, c_i32, c_i32],
     "kalm_merged_attention_out_proj_static": [c_vp, c_i64, c_vp, c_vp, c_i64, c_vp, c_vp, c_i64, c_vp, c_vp, c_i64,
                                               c_vp, c_i32, c_i32, c_i64, c_i64, c_i32, c_i32, c_i32, c_f32, c_vp, c_vp,
                                               c_i64, c_vp, c_i64, c_vp, c_i64, c_i32, c_vp],

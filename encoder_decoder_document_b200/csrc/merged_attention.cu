@@ -105,7 +105,9 @@ struct ProjParams {
   int n_chunks;       // 256-column chunks of hidden
   int m_tiles;        // 128-row tiles of max_q
   int n_otiles;       // n_docs * m_tiles * n_chunks (tiles of rows past a document's end are skipped)
-  int* sync;          // [n_docs] per-document counters, [n_docs] tile-claim counter; zero between launches
+  // [n_docs] per-document item counters, [n_docs] ready-queue tail, [n_docs + 1] its head,
+  // [n_docs + 2, + n_otiles) the ready queue (tile id + 1, 0 = empty); all zero between launches
+  int* sync;
 };
 
 // One work item: query tile t of KV head g of document d, with its extents.
@@ -162,9 +164,10 @@ __device__ __forceinline__ Item load_item(const AttnParams& p, int w) {
 
 // ------------------------------------------------------------------------------
 // Output projection phase of the fused decoder layer: X[rows of d] += O[rows of d] . Wo^T.
-// Tiles are (document, 128-row block, 256-column chunk); a CTA claims them from a
-// counter once its attention items are done and waits, per tile, for that document's
-// attention items (counted by the CTAs that computed them).  1-CTA tcgen05 GEMM:
+// Tiles are (document, 128-row block, 256-column chunk).  When a document's last attention
+// item is counted (by whichever CTA computed it), its tiles go into a ready queue; CTAs
+// that have finished their own attention items pop tiles from it in that order, so no CTA
+// waits on a document that is still being computed while finished ones wait.  1-CTA tcgen05 GEMM:
 // warp 8 lane 0 claims tiles and loads A (O rows) and B (Wo rows) by TMA into a 4-deep
 // ring, warp 9 lane 0 issues M=128 x N=256 products into one of two TMEM
 // accumulators, warps 0-7 add the residual and write X (warp w: rows 32 (w % 4) ..,
@@ -203,26 +206,52 @@ __device__ __forceinline__ void decode_otile(const ProjParams& f, int t, int& d,
 __device__ __forceinline__ void out_proj_phase(const AttnParams& p, const ProjParams& f, const CUtensorMap* tm_oa,
                                                const CUtensorMap* tm_wo, uint8_t* smem, const GemmBars& gb,
                                                uint32_t tmem, int warp, int lane, volatile int* abort_flag) {
-  int* claim = f.sync + p.n_docs;
+  int* tail = f.sync + p.n_docs;      // pushes (by the CTAs that complete documents)
+  int* head = f.sync + p.n_docs + 1;  // pops
+  int* queue = f.sync + p.n_docs + 2;
   const int kblocks = f.kdim / 64;
   if (warp == kTmaWarp) {
     if (lane != 0) return;
-    // ---------------------------------------------------- tile claims and A/B loads
+    // ---------------------------------------------------- tile pops and A/B loads
     tma_prefetch_desc(tm_oa);
     tma_prefetch_desc(tm_wo);
     int published = 0, stage = 0;
     uint32_t phase = 0;
     bool ok = true;
+    int d = 0, mi = 0, ni = 0;
+    // documents without decoder rows have no attention items to complete them: this CTA
+    // queues the (empty) tiles of those in its stripe, so every queue slot gets filled
+    const int per_doc = f.m_tiles * f.n_chunks;
+    for (int e = blockIdx.x; e < p.n_docs; e += gridDim.x)
+      if (p.q_off[e + 1] == p.q_off[e])
+        for (int u = 0; u < per_doc; ++u) st_release_gpu(queue + atomicAdd(tail, 1), e * per_doc + u + 1);
     while (true) {
-      const int t = atomicAdd(claim, 1);
-      if (t == f.n_otiles + static_cast<int>(gridDim.x) - 1) atomicExch(claim, 0);  // the launch's last claim
-      int d = 0, mi = 0, ni = 0, lq = 0;
+      const int pos = atomicAdd(head, 1);
+      if (pos == f.n_otiles + static_cast<int>(gridDim.x) - 1) {
+        // the launch's last pop: every CTA is past its attention items (so every push is
+        // done) and every slot has been taken; the queue starts empty in the next launch
+        atomicExch(head, 0);
+        atomicExch(tail, 0);
+      }
       int id = -1;
-      if (t < f.n_otiles && ok && !*abort_flag) {
-        decode_otile(f, t, d, mi, ni);
-        lq = static_cast<int>(p.q_off[d + 1] - p.q_off[d]);
-        if (mi * kBM >= lq) continue;  // no rows of this document in the block
-        id = t;
+      if (pos < f.n_otiles && ok && !*abort_flag) {
+        // the slot is filled once the document it belongs to is complete
+        int v = 0;
+        const uint64_t t0 = globaltimer_ns();
+        while ((v = ld_acquire_gpu(queue + pos)) == 0) {
+          if (*abort_flag || globaltimer_ns() - t0 > p.wait_ns) {
+            record_error(p.err, kErrTimeout | kSiteAttention);
+            *abort_flag = 1;
+            ok = false;
+            break;
+          }
+        }
+        if (ok) {
+          queue[pos] = 0;
+          decode_otile(f, v - 1, d, mi, ni);
+          if (mi * kBM >= static_cast<int>(p.q_off[d + 1] - p.q_off[d])) continue;  // no rows in the block
+          id = v - 1;
+        }
       }
       // publish the tile (or the end) to the MMA and epilogue warps
       const int k = published & 1;
@@ -236,22 +265,6 @@ __device__ __forceinline__ void out_proj_phase(const AttnParams& p, const ProjPa
       ++published;
       if (id < 0) break;
       if (!ok) continue;
-      // this document's attention items, computed by any CTA of the launch
-      const int items = p.n_kv * ((lq + p.P - 1) / p.P);
-      const int tiles_d = ((lq + kBM - 1) / kBM) * f.n_chunks;
-      const uint64_t t0 = globaltimer_ns();
-      while (ld_acquire_gpu(f.sync + d) < items) {
-        if (*abort_flag || globaltimer_ns() - t0 > p.wait_ns) {
-          record_error(p.err, kErrTimeout | kSiteAttention);
-          *abort_flag = 1;
-          ok = false;
-          break;
-        }
-      }
-      if (ok) {
-        // the document's last consumer puts its counter back to zero for the next launch
-        if (atomicAdd(f.sync + d, 1) == items + tiles_d - 1) atomicExch(f.sync + d, 0);
-      }
       fence_proxy_async_global();  // O rows written by other CTAs, read below by TMA
       const int32_t row0 = static_cast<int32_t>(p.q_off[d] + mi * kBM);
       for (int kb = 0; kb < kblocks && ok; ++kb) {
@@ -574,7 +587,17 @@ __global__ void __launch_bounds__(kThreads, 1)
           fail_wait();
           break;
         }
-        red_release_gpu_add(f.sync + it.d, 1);
+        // count the item; the count that completes the document (acquiring the other
+        // counters' releases) queues its tiles, each slot written with release order
+        const int items = p.n_kv * ((it.Lq + p.P - 1) / p.P);
+        if (atom_add_acq_rel_gpu(f.sync + it.d, 1) + 1 == items) {
+          f.sync[it.d] = 0;  // no further count this launch: zero for the next one
+          const int per_doc = f.m_tiles * f.n_chunks;
+          for (int u = 0; u < per_doc; ++u) {
+            const int pos = atomicAdd(f.sync + p.n_docs, 1);
+            st_release_gpu(f.sync + p.n_docs + 2 + pos, it.d * per_doc + u + 1);
+          }
+        }
         mbar_arrive(bar_osig);
         ++n_it;
       }
@@ -1224,8 +1247,10 @@ extern "C" kalm_status kalm_merged_attention(const kalm_bf16* q, int64_t ldq, co
                           order, out, ldo, lse, nullptr, stream);
 }
 
-extern "C" int64_t kalm_attention_out_proj_sync_len(int32_t n_docs) {
-  return n_docs < 0 ? -1 : static_cast<int64_t>(n_docs) + 1;
+extern "C" int64_t kalm_attention_out_proj_sync_len(int32_t n_docs, int32_t max_q, int32_t hidden) {
+  if (n_docs < 0 || max_q < 0 || hidden <= 0) return -1;
+  const int64_t tiles = static_cast<int64_t>(n_docs) * ((max_q + kBM - 1) / kBM) * ((hidden + 255) / 256);
+  return static_cast<int64_t>(n_docs) + 2 + tiles;
 }
 
 extern "C" kalm_status kalm_merged_attention_out_proj(
@@ -1242,9 +1267,9 @@ extern "C" kalm_status kalm_merged_attention_out_proj(
                 hidden);
   if (n_docs == 0 || max_q == 0 || total_q == 0) return KALM_OK;
   if (!w_o || !x || !sync) return fail(KALM_ERR_INVALID_ARG, "kalm_merged_attention_out_proj: NULL pointer");
-  if (sync_len < kalm_attention_out_proj_sync_len(n_docs))
+  if (sync_len < kalm_attention_out_proj_sync_len(n_docs, max_q, hidden))
     return fail(KALM_ERR_INVALID_ARG, "kalm_merged_attention_out_proj: sync_len=%lld < %lld", (long long)sync_len,
-                (long long)kalm_attention_out_proj_sync_len(n_docs));
+                (long long)kalm_attention_out_proj_sync_len(n_docs, max_q, hidden));
   if ((reinterpret_cast<uintptr_t>(sync) & 3u) || !aligned16(w_o) || !aligned16(x) || ldw % 8 || ldx % 8 ||
       ldw < static_cast<int64_t>(n_q) * head_dim || ldx < hidden)
     return fail(KALM_ERR_INVALID_ARG, "kalm_merged_attention_out_proj: bad alignment or stride");
@@ -1260,8 +1285,10 @@ extern "C" kalm_status kalm_merged_attention_out_proj(
 // every device that loads the library holds the array (16 KB) until the process exits.
 namespace {
 
-constexpr int kStaticSyncDocs = KALM_OUT_PROJ_STATIC_MAX_DOCS;  // documents per call the built-in counters hold
-static __device__ __align__(256) int32_t g_out_proj_sync[kStaticSyncDocs + 1];
+constexpr int kStaticSyncDocs = KALM_OUT_PROJ_STATIC_MAX_DOCS;    // documents per call
+constexpr int kStaticSyncTiles = KALM_OUT_PROJ_STATIC_MAX_TILES;  // projection tiles per call
+constexpr int kStaticSyncLen = kStaticSyncDocs + 2 + kStaticSyncTiles;
+static __device__ __align__(256) int32_t g_out_proj_sync[kStaticSyncLen];
 
 // Device address of g_out_proj_sync, looked up once per device (host code only sees a
 // stand-in symbol, not a device address).
@@ -1292,17 +1319,20 @@ extern "C" kalm_status kalm_merged_attention_out_proj_static(
   int dev = -1;
   kalm_status st = ensure_device(&dev);
   if (st != KALM_OK) return st;
-  if (n_docs > kStaticSyncDocs)
+  if (n_docs < 0 || max_q < 0 || hidden <= 0)
+    return fail(KALM_ERR_INVALID_ARG, "kalm_merged_attention_out_proj_static: n_docs=%d max_q=%d hidden=%d", n_docs,
+                max_q, hidden);
+  const int64_t len = kalm_attention_out_proj_sync_len(n_docs, max_q, hidden);
+  if (n_docs > kStaticSyncDocs || len - n_docs - 2 > kStaticSyncTiles)
     return fail(KALM_ERR_INVALID_ARG,
-                "kalm_merged_attention_out_proj_static: n_docs=%d is above the %d documents its built-in counters "
-                "hold (pass a counter array to kalm_merged_attention_out_proj instead)",
-                n_docs, kStaticSyncDocs);
-  if (n_docs < 0) return fail(KALM_ERR_INVALID_ARG, "kalm_merged_attention_out_proj_static: n_docs=%d", n_docs);
+                "kalm_merged_attention_out_proj_static: %d documents and %lld projection tiles exceed what its "
+                "built-in counters hold (%d documents, %d tiles); pass a counter array to "
+                "kalm_merged_attention_out_proj instead",
+                n_docs, (long long)(len - n_docs - 2), kStaticSyncDocs, kStaticSyncTiles);
   int32_t* sync = nullptr;
   if ((st = static_sync_ptr(dev, &sync)) != KALM_OK) return st;
   // the counters must start at zero: clear the part this call uses (a call cut short by a
   // device error may have left values behind)
-  const int64_t len = kalm_attention_out_proj_sync_len(n_docs);
   st = check_cuda(cudaMemsetAsync(sync, 0, static_cast<size_t>(len) * sizeof(int32_t),
                                   static_cast<cudaStream_t>(stream)),
                   "clear out-proj counters");

@@ -125,7 +125,7 @@ class FBNLScorer:
                                  **kw)
         self.yes, self.no, self.margin, self.score = self.result[0], self.result[1], self.result[2], self.result[3]
         # the fused layer's per-document counters (zero before a launch, left zero by it)
-        self.sync = torch.zeros(max(kalm_attention_out_proj_sync_len(n_docs), 1), dtype=torch.int32, **kw)
+        self.sync = torch.zeros(max(kalm_attention_out_proj_sync_len(n_docs, lq, H), 1), dtype=torch.int32, **kw)
         self.graphs = None
         self.graphs_decode = None
 

@@ -236,10 +236,10 @@ kalm_status kalm_merged_attention(const kalm_bf16* q, int64_t ldq,
  * Computes exactly what kalm_merged_attention (last_tile_only = 0, lse = NULL) writes
  * to `out`, and then, for every document, X[rows of d] += out[rows of d] . w_o^T with
  * one bf16 rounding (as kalm_linear with residual = x, in place).  Inside the launch
- * each CTA first computes its attention work items; the projection tiles (document x
- * 128 rows x 256 columns) are then claimed by the CTAs as they finish, and a tile waits
- * only for its own document's attention items, so the projection fills the tail of the
- * attention.
+ * each CTA first computes its attention work items; when a document's last item is
+ * done, its projection tiles (document x 128 rows x 256 columns) are queued, and CTAs
+ * that have finished their own items take tiles from the queue in that order, so the
+ * projection fills the tail of the attention.
  *
  * Arguments up to `ldo`: as kalm_merged_attention (q_off, in_off, pool_off, order, out
  *          ... with the same requirements; `order` must come from kalm_attention_schedule
@@ -248,8 +248,9 @@ kalm_status kalm_merged_attention(const kalm_bf16* q, int64_t ldq,
  *          in = n_q * head_dim
  * x        [total_q][ldx] bf16, the residual stream, updated in place
  * hidden   multiple of 64
- * sync     int32 device array of sync_len >= kalm_attention_out_proj_sync_len(n_docs)
- *          entries: the launch's per-document completion counters and its tile counter.
+ * sync     int32 device array of sync_len >= kalm_attention_out_proj_sync_len(n_docs,
+ *          max_q, hidden) entries: the launch's per-document completion counters and a
+ *          queue of projection tiles whose documents are complete.
  *          Caller-owned; must be zero before the first call (e.g. cudaMemset), and every
  *          call leaves it zero again.  Launches that share one array must not overlap on
  *          the GPU.  After a call that recorded a device error, zero it again.
@@ -277,8 +278,10 @@ kalm_status kalm_merged_attention_out_proj(const kalm_bf16* q, int64_t ldq,
  *
  * Same arguments, results and errors as kalm_merged_attention_out_proj, minus sync and
  * sync_len.  The counters live in a fixed array inside the library's device memory,
- * sized for KALM_OUT_PROJ_STATIC_MAX_DOCS documents: every device that loads the library
- * holds it (16 KB) until the process exits.  More documents -> KALM_ERR_INVALID_ARG.
+ * sized for KALM_OUT_PROJ_STATIC_MAX_DOCS documents and KALM_OUT_PROJ_STATIC_MAX_TILES
+ * projection tiles (n_docs * ceil(max_q / 128) * ceil(hidden / 256)): every device that
+ * loads the library holds it (about 213 KB) until the process exits.  Larger sizes ->
+ * KALM_ERR_INVALID_ARG.
  * Nothing is allocated: the call clears the counters it uses with an asynchronous
  * memset on `stream` and launches the fused kernel.
  * - The first call on a device looks up the array's device address (a runtime query);
@@ -287,6 +290,7 @@ kalm_status kalm_merged_attention_out_proj(const kalm_bf16* q, int64_t ldq,
  *   calls whose work overlaps on the GPU (other streams, other host threads) race on it;
  *   order them on one stream. */
 #define KALM_OUT_PROJ_STATIC_MAX_DOCS 4096
+#define KALM_OUT_PROJ_STATIC_MAX_TILES 49152
 kalm_status kalm_merged_attention_out_proj_static(const kalm_bf16* q, int64_t ldq,
                                                   const kalm_bf16* k_self, const kalm_bf16* v_self, int64_t ld_self,
                                                   const kalm_bf16* k_cross, const kalm_bf16* v_cross, int64_t ld_cross,
@@ -298,9 +302,10 @@ kalm_status kalm_merged_attention_out_proj_static(const kalm_bf16* q, int64_t ld
                                                   const kalm_bf16* w_o, int64_t ldw, kalm_bf16* x, int64_t ldx,
                                                   int32_t hidden, kalm_stream_t stream);
 
-/* Entries of the sync array kalm_merged_attention_out_proj needs for n_docs documents
- * (n_docs + 1), or -1 for n_docs < 0.  Host-only arithmetic. */
-int64_t kalm_attention_out_proj_sync_len(int32_t n_docs);
+/* Entries of the sync array kalm_merged_attention_out_proj needs: n_docs + 2 +
+ * n_docs * ceil(max_q / 128) * ceil(hidden / 256), or -1 for negative sizes or
+ * hidden <= 0.  Host-only arithmetic. */
+int64_t kalm_attention_out_proj_sync_len(int32_t n_docs, int32_t max_q, int32_t hidden);
 
 /* Work items of one kalm_merged_attention call (one query tile of 128/(n_q/n_kv)
  * decoder positions x one KV head x one document): ceil(max_q / (128 n_kv / n_q))

@@ -121,6 +121,7 @@ def test_chunk_pool_edge_lengths_padded_and_strided(kalm):
     ([256, 256], [30, 77], 8, 4, 2560),         # Large heads and hidden (K = 2048, 10 column chunks)
     ([37, 37, 37, 37], [5, 64, 65, 1], 4, 1, 640),
     ([512, 3], [256, 2], 4, 1, 640),            # the query budget beside a 3-row document
+    ([64, 0, 64, 0], [10, 5, 0, 7], 4, 1, 640),  # documents without decoder rows
 ])
 def test_attention_out_proj_fused(kalm, lq, nc, n_q, n_kv, hidden):
     """The fused decoder layer: `out` equals the attention kernel's output bit for bit, and
@@ -145,7 +146,8 @@ def test_attention_out_proj_fused(kalm, lq, nc, n_q, n_kv, hidden):
     kalm.kalm_attention_schedule(i64(q_off), i64(p_off), max_q, n_q, n_kv, order)
     ref = torch.full((R, n_q * D), float("nan"), dtype=torch.bfloat16, device="cuda")
     kalm.kalm_merged_attention(*views, i64(q_off), i64(p_off), max_q, n_q, n_kv, ref, 1.0 / 16, order=order)
-    sync = torch.zeros(kalm.kalm_attention_out_proj_sync_len(len(lq)), dtype=torch.int32, device="cuda")
+    sync = torch.zeros(kalm.kalm_attention_out_proj_sync_len(len(lq), max_q, hidden), dtype=torch.int32,
+                       device="cuda")
     results = []
     for rep, use_order in ((0, True), (1, True), (2, False)):
         out = torch.full((R, n_q * D), float("nan"), dtype=torch.bfloat16, device="cuda")
@@ -170,10 +172,10 @@ def test_attention_out_proj_rejects_bad_arguments(kalm):
     x = torch.zeros(32, 640, dtype=torch.bfloat16, device="cuda")
     w_o = torch.zeros(640, 1024, dtype=torch.bfloat16, device="cuda")
     out = torch.zeros(32, 1024, dtype=torch.bfloat16, device="cuda")
-    ok_sync = torch.zeros(2, dtype=torch.int32, device="cuda")
+    ok_sync = torch.zeros(kalm.kalm_attention_out_proj_sync_len(1, 32, 640), dtype=torch.int32, device="cuda")
     args = (q, kv, kv, kc, kc, i64(a["q_off"]), i64(a["p_off"]), 32, 4, 1, out)
     with pytest.raises(KalmError):  # sync array too short
-        kalm.kalm_merged_attention_out_proj(*args, w_o, x, torch.zeros(1, dtype=torch.int32, device="cuda"))
+        kalm.kalm_merged_attention_out_proj(*args, w_o, x, ok_sync[:-1])
     with pytest.raises(KalmError):  # hidden not a multiple of 64
         kalm.kalm_merged_attention_out_proj(*args, w_o[:600], x[:, :600], ok_sync)
     kalm.kalm_merged_attention_out_proj(*args, w_o, x, ok_sync)

@@ -44,7 +44,8 @@ def test_no_alloc_entry_point_matches_caller_counters():
     a = _inputs()
     args = (*a["views"], a["q_off"], a["p_off"], a["max_q"], a["n_q"], a["n_kv"])
     # reference: the entry point with a counter array from the caller
-    sync = torch.zeros(k.kalm_attention_out_proj_sync_len(a["n_docs"]), dtype=torch.int32, device="cuda")
+    sync = torch.zeros(k.kalm_attention_out_proj_sync_len(a["n_docs"], a["max_q"], a["w_o"].shape[0]),
+                       dtype=torch.int32, device="cuda")
     ref_out = torch.empty(a["R"], a["n_q"] * D, dtype=torch.bfloat16, device="cuda")
     ref_x = a["x0"].clone()
     k.kalm_merged_attention_out_proj(*args, ref_out, a["w_o"], ref_x, sync, 1.0 / 16)
@@ -63,7 +64,7 @@ def test_no_alloc_entry_point_matches_caller_counters():
 def test_no_alloc_entry_point_rejects_too_many_documents():
     import encoder_decoder_document_b200 as k
     from encoder_decoder_document_b200 import KalmError
-    n = 4097  # one more document than the built-in counters hold
+    n = 4097  # one more document than the built-in counters hold (KALM_OUT_PROJ_STATIC_MAX_DOCS)
     t = torch.zeros(n, D, dtype=torch.bfloat16, device="cuda")
     q = torch.zeros(n, 4 * D, dtype=torch.bfloat16, device="cuda")
     offs = torch.arange(n + 1, dtype=torch.int64, device="cuda")
