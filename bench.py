@@ -278,7 +278,8 @@ def run_sweep(args, doc_counts=(1, 16, 100, 1024, 4096)):
     distinct seeded queries (seed 4 + k for query k), each with its own lengths, its own
     query length and its own captured graph; K steps per query, L2 flushed before each
     step.  Per point: total documents / total time over its queries, plus the pooling and
-    attention kernels' own times from each query's instrumented graph."""
+    attention kernels' own times from each query's instrumented graph, and (unless the CPU
+    baseline is switched off) the oracle timed on two documents of the point's first query."""
     import torch
     import synthetic
     from encoder_decoder_document_b200 import _build, kalm_check_device_errors
@@ -293,9 +294,12 @@ def run_sweep(args, doc_counts=(1, 16, 100, 1024, 4096)):
         nq = sweep_queries(n)
         tot_ms, tot_docs, lqs = 0.0, 0, []
         attn_us, attn_flops, pool_us, pool_bytes, flops = 0.0, 0, 0.0, 0, 0
+        oracle_cb = None
         for k in range(nq):
             q = synthetic.make_query("sweep", n_docs=n, seed=4 + k, with_weights=False)
             q = dataclasses.replace(q, weights=weights)
+            if k == 0 and not args.no_cpu_baseline:
+                oracle_cb = cpu_baseline(q, min(2, n))
             w = workload(q)
             sc = FBNLScorer(dw, q.n_q, q.n_kv)
             total_pooled = int(((q.doc_len.astype(np.int64) + 3) // 4).sum())
@@ -334,7 +338,8 @@ def run_sweep(args, doc_counts=(1, 16, 100, 1024, 4096)):
                     "step_tflops": flops / (tot_ms * 1e-3) / 1e12,
                     "attention_us_per_query": attn_us / nq, "attention_tflops": attn_flops / (attn_us * 1e-6) / 1e12,
                     "pool_us_per_query": pool_us / nq, "pool_gbs": pool_bytes / (pool_us * 1e-6) / 1e9,
-                    "pool_frac": pool_bytes / (pool_us * 1e-6) / 1e9 / pk["hbm"]})
+                    "pool_frac": pool_bytes / (pool_us * 1e-6) / 1e9 / pk["hbm"],
+                    "cpu_baseline": oracle_cb})
         print(json.dumps(out[-1]), flush=True)
     return out
 
@@ -675,7 +680,8 @@ def main():
         if rope is not None:
             rope["frac"] = rope["gbs"] / pk["hbm"]
         if not args.no_cpu_baseline and world == 1:
-            cb = cpu_baseline(q, args.cpu_sample_docs or q.n_docs, one_thread_docs=min(10, q.n_docs))
+            n_cpu = min(args.cpu_sample_docs or q.n_docs, q.n_docs)
+            cb = cpu_baseline(q, n_cpu, one_thread_docs=min(10, n_cpu))
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
