@@ -1282,7 +1282,8 @@ extern "C" kalm_status kalm_merged_attention_out_proj(
 // ----------------------------------------------------------------------------------
 // The fused layer for callers that cannot allocate device memory.  Its counters live in a
 // fixed array in the library's own device memory instead of a caller-provided buffer:
-// every device that loads the library holds the array (16 KB) until the process exits.
+// every device that loads the library holds the array (4096 documents' counters and a queue of
+// 49,152 projection tiles: 213,000 bytes) until the process exits.
 namespace {
 
 constexpr int kStaticSyncDocs = KALM_OUT_PROJ_STATIC_MAX_DOCS;    // documents per call
