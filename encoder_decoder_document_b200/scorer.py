@@ -476,6 +476,22 @@ class FBNLScorer:
 
         x0: bf16 bits [lq][H] (decoder input of the query); enc: bf16 bits
         [sum(doc_len)][H] (packed encoder states); doc_len: int [n_docs]."""
+        res = self.score_rows(x0, enc, doc_len)
+        return rank(res[:, 2], res[:, 3], top_n)
+
+    def rerank_sharded(self, x0: np.ndarray, enc: np.ndarray, doc_len: np.ndarray, top_n: Optional[int] = None,
+                       group=None):
+        """``rerank`` over the documents of one query split across the ranks of a
+        process group (one process per GPU, each with its own scorer): every rank
+        passes the whole query, scores its share of the documents (balanced by
+        length) and receives the full ranking.  The only exchange is one gather of the
+        per-document scores on the host."""
+        from .sharding import sharded_rerank
+        return sharded_rerank(self.score_rows, x0, enc, doc_len, top_n, group)
+
+    def score_rows(self, x0: np.ndarray, enc: np.ndarray, doc_len: np.ndarray) -> np.ndarray:
+        """Rows (yes, no, margin, score) of one query's documents, in input order
+        (``[n_docs][4]`` float32 on the host); arguments as for ``rerank``."""
         doc_len = np.asarray(doc_len)
         if doc_len.ndim != 1:
             raise ValueError("rerank: doc_len must be one length per document")
@@ -487,6 +503,8 @@ class FBNLScorer:
             raise ValueError(f"rerank: the query input must have 1..{MAX_QUERY_TOKENS} rows (got {lq})")
         doc_len = doc_len.astype(np.int32)
         n = int(doc_len.shape[0])
+        if n == 0:
+            return np.zeros((0, 4), dtype=np.float32)
         total_tokens = int(doc_len.sum())
         if np.asarray(enc).shape[0] < total_tokens:
             raise ValueError(f"rerank: enc holds {np.asarray(enc).shape[0]} rows, doc_len sums to {total_tokens}")
@@ -500,7 +518,7 @@ class FBNLScorer:
         # a bounded wait that expired or invalid device data leaves only a flag on the
         # device: raise instead of returning scores computed past it
         self.check_errors()
-        return rank(res[2], res[3], top_n)
+        return np.ascontiguousarray(res.T)
 
     def check_errors(self) -> None:
         """Wait for this scorer's streams and raise ``KalmError`` if a kernel recorded a

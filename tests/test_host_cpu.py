@@ -1,7 +1,9 @@
 """Host-side checks that need no GPU: the C-ABI library builds, loads and exports
 every symbol include/kalm.h declares; without a device every entry point
 refuses with KALM_ERR_NO_DEVICE (no CPU fallback); document sharding and the
-two-rank gather (gloo) reproduce the single-process scores in input order."""
+sharded scoring API over two gloo ranks reproduce the single-process scores in input
+order, and a failure on one rank raises on every rank."""
+import dataclasses
 import os
 import re
 import socket
@@ -78,45 +80,96 @@ def _free_port():
     return p
 
 
-def _rank_main(rank, world, port, out):
-    import torch.distributed as dist
-    import datetime
+def _oracle_rows(q):
+    """score_fn for the sharded API on the CPU: the oracle's (yes, no, margin, score)
+    rows of the documents it is given, as a query of their own."""
     import oracle
+
+    def fn(x0, enc, doc_len):
+        lens = np.asarray(doc_len, dtype=np.int32)
+        sub = dataclasses.replace(q, x0=x0, enc=enc, doc_len=lens,
+                                  tok_off=np.concatenate([[0], np.cumsum(lens, dtype=np.int64)]))
+        return np.stack(oracle.forward_query(sub), 1)
+    return fn
+
+
+def _rank_main(rank, world, port, out, fail_rank):
+    import datetime
+    import torch.distributed as dist
     import synthetic
-    from encoder_decoder_document_b200.sharding import merge_scores, shard_documents
+    from encoder_decoder_document_b200.sharding import sharded_rerank, sharded_scores
     dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{port}", rank=rank, world_size=world,
                             timeout=datetime.timedelta(seconds=60))
     q = synthetic.make_query("tiny", hidden=64, n_docs=5)
-    shards = shard_documents(q.doc_len, world)
-    mine = shards[rank]
-    part = np.stack(oracle.forward_query(q, docs=mine), 1) if len(mine) else np.zeros((0, 4))
-    gathered = [None] * world
-    dist.all_gather_object(gathered, part)
-    if rank == 0:
-        out.put(merge_scores(shards, gathered, q.n_docs))
+    fn = _oracle_rows(q)
+    if rank == fail_rank:
+        def fn(x0, enc, doc_len):  # noqa: F811 - this rank's scoring fails on the host
+            raise RuntimeError("planted failure")
+    try:
+        res = sharded_scores(fn, q.x0, q.enc, q.doc_len)
+        ranked = sharded_rerank(fn, q.x0, q.enc, q.doc_len, top_n=3)
+        out.put((rank, "ok", res, ranked))
+    except RuntimeError as e:
+        out.put((rank, "raised", str(e), None))
     dist.barrier()
     dist.destroy_process_group()
 
 
-def test_two_rank_document_sharding_gloo():
+def _run_ranks(world, fail_rank=-1):
     import multiprocessing as mp
-    import oracle
-    import synthetic
     ctx = mp.get_context("spawn")
     out = ctx.Queue()
     port = _free_port()
-    procs = [ctx.Process(target=_rank_main, args=(r, 2, port, out)) for r in range(2)]
+    procs = [ctx.Process(target=_rank_main, args=(r, world, port, out, fail_rank)) for r in range(world)]
     for p in procs:
         p.start()
-    merged = out.get(timeout=240)
+    got = sorted((out.get(timeout=240) for _ in range(world)), key=lambda t: t[0])
     for p in procs:
         p.join(timeout=120)
         assert p.exitcode == 0
+    return got
+
+
+def test_two_rank_document_sharding_gloo():
+    """The sharded scoring API over two gloo ranks: each rank scores its share of the
+    documents, one host gather puts the rows back in input order, and every rank gets
+    the whole result, equal to scoring all documents in one process."""
+    import oracle
+    import synthetic
+    from encoder_decoder_document_b200.scorer import rank
+    got = _run_ranks(2)
     q = synthetic.make_query("tiny", hidden=64, n_docs=5)
     want = np.stack(oracle.forward_query(q), 1)
-    np.testing.assert_array_equal(merged, want)
-    from encoder_decoder_document_b200.scorer import rank
-    assert rank(merged[:, 2], merged[:, 3]) == rank(want[:, 2], want[:, 3])
+    for r, status, res, ranked in got:
+        assert status == "ok", res
+        np.testing.assert_array_equal(res, want)
+        assert ranked == rank(want[:, 2], want[:, 3], 3)
+
+
+def test_sharded_scoring_failure_on_one_rank_raises_on_every_rank():
+    """A rank whose scoring fails still takes part in the gather; then every rank
+    raises, naming the failed rank, and no rank is left waiting in a collective."""
+    got = _run_ranks(2, fail_rank=1)
+    for r, status, msg, _ in got:
+        assert status == "raised"
+        assert "rank 1" in msg and "planted failure" in msg
+
+
+def test_sharded_scores_single_process_and_slicing():
+    """Without a process group the sharded call is the plain call; slice_documents
+    takes documents' rows out of a packed batch."""
+    import oracle
+    import synthetic
+    from encoder_decoder_document_b200.sharding import slice_documents, sharded_scores
+    q = synthetic.make_query("tiny", hidden=64, n_docs=4)
+    res = sharded_scores(_oracle_rows(q), q.x0, q.enc, q.doc_len)
+    np.testing.assert_array_equal(res, np.stack(oracle.forward_query(q), 1))
+    enc = np.arange(10 * 2).reshape(10, 2)
+    rows, lens = slice_documents(enc, [3, 0, 5, 2], [2, 0, 1])
+    np.testing.assert_array_equal(rows, np.concatenate([enc[3:8], enc[0:3]]))
+    np.testing.assert_array_equal(lens, [5, 3, 0])
+    rows, lens = slice_documents(enc, [3, 0, 5, 2], [])
+    assert rows.shape == (0, 2) and lens.shape == (0,)
 
 
 def _bench(args, env_extra=None):
