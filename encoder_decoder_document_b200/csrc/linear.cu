@@ -582,7 +582,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 }
 
 int g_num_sms[64] = {0};
-int g_pair_slots[64][3] = {};  // co-resident CTA pairs for BN = 256, 192, 160
+int g_pair_slots[64][4] = {};  // co-resident CTA pairs for BN = 256, 192, 160, 224
 
 template <int BN>
 kalm_status setup_pair(int dev, int slot) {
@@ -624,6 +624,7 @@ kalm_status setup_linear_kernels() {
   if ((st = setup_pair<256>(dev, 0)) != KALM_OK) return st;
   if ((st = setup_pair<192>(dev, 1)) != KALM_OK) return st;
   if ((st = setup_pair<160>(dev, 2)) != KALM_OK) return st;
+  if ((st = setup_pair<224>(dev, 3)) != KALM_OK) return st;
   return KALM_OK;
 }
 
@@ -713,11 +714,11 @@ kalm_status launch_linear(const kalm_bf16* x, int64_t ldx, const kalm_bf16* w, i
     // CTA-pair tiles of 256 x BN.  Time ~ rounds of co-resident pairs x (BN + fixed
     // per-tile cost); the fixed cost, measured at the Nano projection shapes, is worth
     // ~480 columns, so narrower tiles pay off only when they save a round.
-    const int bns[3] = {256, 192, 160};
+    const int bns[4] = {256, 192, 160, 224};
     const int64_t n_m = (m + 2 * kBM - 1) / (2 * kBM);
     int best = 0;
     int64_t best_cost = INT64_MAX;
-    for (int i = 0; i < 3; ++i) {
+    for (int i = 0; i < 4; ++i) {
       const int64_t tiles = n_m * ((n + bns[i] - 1) / bns[i]);
       const int64_t slots = pair_slots(i);
       const int64_t cost = ((tiles + slots - 1) / slots) * (bns[i] + 480);
@@ -729,6 +730,7 @@ kalm_status launch_linear(const kalm_bf16* x, int64_t ldx, const kalm_bf16* w, i
     const int slots = pair_slots(best);
     if (best == 0) return launch_pair<256>(x, ldx, w, ldw, residual, ldr, y, ldy, m, n, k, slots, stream, rope);
     if (best == 1) return launch_pair<192>(x, ldx, w, ldw, residual, ldr, y, ldy, m, n, k, slots, stream, rope);
+    if (best == 3) return launch_pair<224>(x, ldx, w, ldw, residual, ldr, y, ldy, m, n, k, slots, stream, rope);
     return launch_pair<160>(x, ldx, w, ldw, residual, ldr, y, ldy, m, n, k, slots, stream, rope);
   }
   const bool wide = (n % 256) == 0;
