@@ -37,7 +37,9 @@ def merge_scores(shards: Sequence[np.ndarray], parts: Sequence[np.ndarray], n_do
     """Put each rank's per-document rows (``parts[r][k]`` belongs to document
     ``shards[r][k]``) back into input order."""
     first = next((p for p in parts if len(p)), None)
-    width = () if first is None else np.asarray(first).shape[1:]
+    if first is None:  # no rows at all: keep the row shape the (empty) parts carry
+        first = next((p for p in parts if np.asarray(p).ndim > 1), np.zeros(0))
+    width = np.asarray(first).shape[1:]
     out = np.full((n_docs,) + tuple(width), np.nan)
     for idx, p in zip(shards, parts):
         out[np.asarray(idx, dtype=np.int64)] = p

@@ -170,6 +170,11 @@ def test_sharded_scores_single_process_and_slicing():
     np.testing.assert_array_equal(lens, [5, 3, 0])
     rows, lens = slice_documents(enc, [3, 0, 5, 2], [])
     assert rows.shape == (0, 2) and lens.shape == (0,)
+    # a query without documents: an empty (0, 4) result and an empty ranking
+    from encoder_decoder_document_b200.sharding import sharded_rerank
+    none = sharded_scores(_oracle_rows(q), q.x0, q.enc[:0], np.zeros(0, np.int32))
+    assert none.shape == (0, 4)
+    assert sharded_rerank(_oracle_rows(q), q.x0, q.enc[:0], np.zeros(0, np.int32)) == []
 
 
 def _bench(args, env_extra=None):
