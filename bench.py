@@ -50,6 +50,8 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-pool-sweep", action="store_true", help="skip the pooling-only sweep at 1024/4096 docs")
     ap.add_argument("--no-fused", action="store_true", help="skip the fused attention + output projection step")
+    ap.add_argument("--no-chain", action="store_true",
+                    help="run each output projection and the next Q|K|V projection as two launches")
     ap.add_argument("--rope-theta", type=float, default=None,
                     help="rotate the decoder's self Q/K with this rotary base in every layer (default: off)")
     ap.add_argument("--sweep", action="store_true",
@@ -93,11 +95,13 @@ def peaks():
 # ---------------------------------------------------------------------------
 # algorithmic work (what the method must do; padding and masked keys not counted)
 # ---------------------------------------------------------------------------
-def workload(q):
+def workload(q, chain: bool = True):
     """Algorithmic work of one step, per kernel kind (summed over its launches), for
     the pruned layer stack the scorer runs: the first layer's Q|K|V projection on
     the query's common input only, and in the last layer attention for the query
-    tile holding each document's final row and the output projection of that row."""
+    tile holding each document's final row and the output projection of that row.
+    With ``chain`` (the scorer's default) every other layer's output projection and
+    the next layer's Q|K|V projection are one launch, labelled o_proj_qkv."""
     H, D, nq, nkv, L, lq = q.hidden, q.head_dim, q.n_q, q.n_kv, q.layers, q.lq
     n = q.n_docs
     lens = q.doc_len.astype(np.int64)
@@ -127,6 +131,17 @@ def workload(q):
                             + 2 * (n * P * 2 * nq * D + rows * 2 * nkv * D + P_ * 2 * nkv * D),
         "o_proj": 2 * ((rows * (L - 1) + n) * (nq * D + 2 * H) + L * H * nq * D),
     }
+    if chain and L > 1:
+        # the chained launches: output projections of layers 0 .. L-2 (with the residual)
+        # and Q|K|V projections of layers 1 .. L-1, each operand read once and each
+        # result written once
+        w["o_proj_qkv"] = int(2 * nq * D * H * rows * (L - 1) + qkv_row * rows * (L - 1))
+        w["qkv_proj"] = int(qkv_row * lq)
+        w["o_proj"] = int(2 * nq * D * H * n)
+        w["bytes"]["o_proj_qkv"] = 2 * ((L - 1) * rows * (nq * D + 2 * H) + (L - 1) * H * nq * D
+                                        + (L - 1) * rows * (H + (nq + 2 * nkv) * D) + (L - 1) * (nq + 2 * nkv) * D * H)
+        w["bytes"]["qkv_proj"] = 2 * (lq * (H + (nq + 2 * nkv) * D) + (nq + 2 * nkv) * D * H)
+        w["bytes"]["o_proj"] = 2 * (n * (nq * D + 2 * H) + H * nq * D)
     return w
 
 
@@ -300,8 +315,8 @@ def run_sweep(args, doc_counts=(1, 16, 100, 1024, 4096)):
             q = dataclasses.replace(q, weights=weights)
             if k == 0 and not args.no_cpu_baseline:
                 oracle_cb = cpu_baseline(q, min(2, n))
-            w = workload(q)
-            sc = FBNLScorer(dw, q.n_q, q.n_kv)
+            sc = FBNLScorer(dw, q.n_q, q.n_kv, chain=not args.no_chain)
+            w = workload(q, chain=sc.chain)
             total_pooled = int(((q.doc_len.astype(np.int64) + 3) // 4).sum())
             sc.prepare(q.n_docs, int(q.doc_len.sum()), total_pooled, q.lq)
             sc.load_inputs(torch.from_numpy(q.enc.view(np.int16)).view(torch.bfloat16),
@@ -520,9 +535,10 @@ def main():
     # each rank scores its own query (its own document shard) of the configured shape
     base = synthetic.CONFIGS[args.config]["seed"]
     q = synthetic.make_query(args.config, seed=base if rank == 0 else base + 1000 * rank)
-    w = workload(q)
     pk = peaks()
-    sc = FBNLScorer(DeviceWeights.from_bits(q.weights), q.n_q, q.n_kv, rope_theta=args.rope_theta)
+    sc = FBNLScorer(DeviceWeights.from_bits(q.weights), q.n_q, q.n_kv, rope_theta=args.rope_theta,
+                    chain=not args.no_chain)
+    w = workload(q, chain=sc.chain)
     total_pooled = int(((q.doc_len.astype(np.int64) + 3) // 4).sum())
     sc.prepare(q.n_docs, int(q.doc_len.sum()), total_pooled, q.lq)
     enc_h = torch.from_numpy(q.enc.view(np.int16)).view(torch.bfloat16).pin_memory()
@@ -644,7 +660,7 @@ def main():
     for label, v in per_kernel.items():
         kern[label] = {"launches_per_step": len(v) / args.steps, "avg_us": 1e3 * statistics.mean(v),
                        "us_per_step": 1e3 * sum(v) / args.steps, "share": sum(v) / grand}
-    tensor_kernels = [k for k in kern if k in ("qkv_proj", "o_proj", "merged_attention", "cross_kv_proj")]
+    tensor_kernels = [k for k in kern if k in ("qkv_proj", "o_proj", "o_proj_qkv", "merged_attention", "cross_kv_proj")]
     for k in tensor_kernels:
         kern[k]["tflops"] = w[k] / (kern[k]["us_per_step"] * 1e-6) / 1e12
     dom = max(tensor_kernels, key=lambda k: kern[k]["share"])

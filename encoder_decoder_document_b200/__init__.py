@@ -16,7 +16,8 @@ from ._abi import KalmError, call, load, library_path  # noqa: F401
 
 __all__ = [
     "KalmError", "load", "library_path", "kalm_version", "kalm_device_check", "kalm_check_device_errors",
-    "kalm_ragged_offsets", "kalm_chunk_pool", "kalm_linear", "kalm_cross_kv_proj", "kalm_merged_attention",
+    "kalm_ragged_offsets", "kalm_chunk_pool", "kalm_linear", "kalm_linear_chain", "kalm_linear_chain_sync_len",
+    "kalm_cross_kv_proj", "kalm_merged_attention",
     "kalm_merged_attention_out_proj", "kalm_merged_attention_out_proj_static", "kalm_attention_out_proj_sync_len",
     "kalm_yes_no_score", "kalm_broadcast_rows", "kalm_selftest_wait_timeout", "kalm_attention_items",
     "kalm_attention_schedule", "kalm_rope", "kalm_rope_table", "kalm_linear_rope",
@@ -86,6 +87,25 @@ def kalm_linear(x: torch.Tensor, w: torch.Tensor, y: torch.Tensor, residual: Opt
     call("kalm_linear", _p(x, torch.bfloat16), _ld(x), _p(w, torch.bfloat16), _ld(w),
          _p(residual, torch.bfloat16), _ld(residual) if residual is not None else 0,
          _p(y, torch.bfloat16), _ld(y), m, n, k, _stream(stream))
+
+
+def kalm_linear_chain_sync_len(m: int) -> int:
+    return int(load().kalm_linear_chain_sync_len(m))
+
+
+def kalm_linear_chain(x1: torch.Tensor, w1: torch.Tensor, y1: torch.Tensor, w2: torch.Tensor, y2: torch.Tensor,
+                      sync: Optional[torch.Tensor], stream=None) -> None:
+    """y1 = x1 . w1^T + y1 (in place), then y2 = y1 . w2^T, in one launch; ``sync`` is an
+    int32 tensor of ``kalm_linear_chain_sync_len(m)`` entries, zero before the first call
+    (every call leaves it zero)."""
+    m, k1 = x1.shape
+    n1, n2 = w1.shape[0], w2.shape[0]
+    if w1.shape[1] != k1 or y1.shape != (m, n1) or w2.shape[1] != n1 or y2.shape != (m, n2):
+        raise KalmError(1, "kalm_linear_chain", f"shapes x1{tuple(x1.shape)} w1{tuple(w1.shape)} y1{tuple(y1.shape)} "
+                                                f"w2{tuple(w2.shape)} y2{tuple(y2.shape)}")
+    call("kalm_linear_chain", _p(x1, torch.bfloat16), _ld(x1), _p(w1, torch.bfloat16), _ld(w1),
+         _p(y1, torch.bfloat16), _ld(y1), _p(w2, torch.bfloat16), _ld(w2), _p(y2, torch.bfloat16), _ld(y2), m, n1, k1,
+         n2, _p(sync, torch.int32), sync.numel() if sync is not None else 0, _stream(stream))
 
 
 def kalm_cross_kv_proj(pooled: torch.Tensor, w_kv: torch.Tensor, kv_cross: torch.Tensor, n_kv: int,

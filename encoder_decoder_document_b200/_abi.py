@@ -29,6 +29,9 @@ SIGNATURES = {
     "kalm_ragged_offsets": [c_vp, c_i32, c_i32, c_vp, c_vp, c_vp],
     "kalm_chunk_pool": [c_vp, c_i64, c_vp, c_vp, c_i32, c_i32, c_i32, c_vp, c_i64, c_vp, c_i64, c_vp],
     "kalm_linear": [c_vp, c_i64, c_vp, c_i64, c_vp, c_i64, c_vp, c_i64, c_i64, c_i32, c_i32, c_vp],
+    "kalm_linear_chain": [c_vp, c_i64, c_vp, c_i64, c_vp, c_i64, c_vp, c_i64, c_vp, c_i64, c_i64, c_i32, c_i32,
+                          c_i32, c_vp, c_i64, c_vp],
+    "kalm_linear_chain_sync_len": [c_i64],
     "kalm_cross_kv_proj": [c_vp, c_i64, c_i64, c_i32, c_vp, c_i32, c_i32, c_i32, c_vp, c_vp],
     "kalm_merged_attention": [c_vp, c_i64, c_vp, c_vp, c_i64, c_vp, c_vp, c_i64, c_vp, c_vp, c_i64, c_vp, c_i32,
                               c_i32, c_i64, c_i64, c_i32, c_i32, c_i32, c_f32, c_i32, c_vp, c_vp, c_i64, c_vp,
@@ -50,7 +53,7 @@ SIGNATURES = {
                          c_vp, c_vp],
     "kalm_rope_table": [c_f32, c_i32, c_vp, c_vp],
 }
-_RESTYPE = {"kalm_version": c_i32, "kalm_attention_items": c_i64, "kalm_attention_out_proj_sync_len": c_i64, "kalm_status_string": ctypes.c_char_p, "kalm_last_error": ctypes.c_char_p}
+_RESTYPE = {"kalm_version": c_i32, "kalm_attention_items": c_i64, "kalm_attention_out_proj_sync_len": c_i64, "kalm_linear_chain_sync_len": c_i64, "kalm_status_string": ctypes.c_char_p, "kalm_last_error": ctypes.c_char_p}
 
 
 class KalmError(RuntimeError):

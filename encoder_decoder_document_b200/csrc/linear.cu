@@ -581,8 +581,265 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   }
 }
 
+// ---------------------------------------------------------------------------
+// Two chained pair GEMMs in one persistent launch: Y1 = X1 . W1^T + R1 (the output
+// projection with its residual, written in place), then Y2 = Y1 . W2^T (the next
+// layer's Q|K|V projection).  Every tile is 256 rows (one CTA pair) by its phase's
+// width (a runtime value up to 256); the launch walks the phase-1 tiles first and
+// then the phase-2 tiles in row-block order, round robin over the pairs, so each
+// pair finishes issuing its phase-1 tiles before it reaches a phase-2 tile.
+// A phase-2 tile reads its 256 rows of Y1 only once every phase-1 tile of that row
+// block has stored them: each epilogue warp of a phase-1 tile waits for its own tile
+// stores to complete and adds 1 to the row block's counter (gpu-scope release), and
+// the x producer of a phase-2 tile waits for the full count (acquire, bounded) before
+// its first load.  Every waiter of a row block then counts itself in a second counter;
+// the last one zeroes both, so each launch leaves the array at zero.  Phase-1 tiles
+// wait on nothing, so no pair can wait on work that is not already issued.
+// ---------------------------------------------------------------------------
+struct ChainCfg {
+  static constexpr int A_BYTES = kBM * kBK * 2;  // this CTA's 128 rows x 64 k
+  static constexpr int B_BYTES = 128 * kBK * 2;  // its half of a tile up to 256 columns
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int EPI_BYTES = 4 * 2 * kChunkBytes;
+  static constexpr int BAR_BYTES = 256;
+  static constexpr int STAGES = (232448 - 1024 - BAR_BYTES - 2 * EPI_BYTES) / STAGE_BYTES;
+  static constexpr int SMEM = 1024 + STAGES * STAGE_BYTES + 2 * EPI_BYTES + BAR_BYTES;
+  static constexpr uint32_t TMEM_COLS = 512;  // two accumulators at columns 0 and 256
+  static constexpr uint32_t ACC_STRIDE = 256;
+};
+
+// One phase of the chained launch.
+struct ChainPhase {
+  int N, K;        // output columns and reduction length
+  int BN;          // tile width: a multiple of 32 up to 256 whose half is whole 8-row groups
+  uint32_t idesc;  // instruction descriptor of a 256 x BN product
+  int n_n, kblocks;
+};
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+    linear_chain_kernel(const __grid_constant__ CUtensorMap tm_x1, const __grid_constant__ CUtensorMap tm_w1,
+                        const __grid_constant__ CUtensorMap tm_y1, const __grid_constant__ CUtensorMap tm_r1,
+                        const __grid_constant__ CUtensorMap tm_x2, const __grid_constant__ CUtensorMap tm_w2,
+                        const __grid_constant__ CUtensorMap tm_y2, const ChainPhase p1, const ChainPhase p2, int M,
+                        int* sync, uint64_t wait_ns, uint32_t* err) {
+  using C = ChainCfg;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + C::STAGES * C::A_BYTES;
+  uint8_t* sOut = sB + C::STAGES * C::B_BYTES;
+  uint8_t* sRes = sOut + C::EPI_BYTES;
+  uint64_t* full = reinterpret_cast<uint64_t*>(sRes + C::EPI_BYTES);  // used in the even CTA
+  uint64_t* empty = full + C::STAGES;
+  uint64_t* acc_full = empty + C::STAGES;
+  uint64_t* acc_empty = acc_full + 2;  // used in the even CTA
+  uint64_t* res_full = acc_empty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(res_full + 8);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = rank == 0;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::STAGES; ++s) {
+      mbar_init(&full[s], 2);  // the even CTA's x copy and w copy arrive with both CTAs' bytes
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&acc_full[b], 1);
+      mbar_init(&acc_empty[b], 8);  // one arrival per epilogue warp of both CTAs
+    }
+    for (int b = 0; b < 8; ++b) mbar_init(&res_full[b], 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == kMmaWarp) {
+    tmem_alloc_pair(tmem_slot, C::TMEM_COLS);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  cluster_sync_all();  // barriers of both CTAs initialised, tensor memory allocated
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  pdl_launch_dependents();
+  pdl_wait_predecessor();  // X1 (and the buffer Y2 overwrites) belong to the previous kernel until here
+
+  const int n_m = (M + 2 * kBM - 1) / (2 * kBM);
+  const int tiles1 = n_m * p1.n_n;
+  const int tiles = tiles1 + n_m * p2.n_n;
+  const int pair = blockIdx.x >> 1, n_pairs = gridDim.x >> 1;
+  int* done = sync;         // [n_m] phase-1 epilogue warps whose stores of the row block completed
+  int* seen = sync + n_m;   // [n_m] phase-2 producers past their wait on the row block
+  const int need = p1.n_n * 8;  // 4 epilogue warps in each CTA of every phase-1 tile of the row block
+
+  if (warp < kProdWarps) {
+    if (lane == 0) {
+      const bool is_w = warp == 1;
+      tma_prefetch_desc(is_w ? &tm_w1 : &tm_x1);
+      tma_prefetch_desc(is_w ? &tm_w2 : &tm_x2);
+      const uint32_t full0 = map_to_rank(smem_u32(full), 0);  // the even CTA's full barriers
+      int stage = 0;
+      uint32_t phase = 0;
+      for (int t = pair; t < tiles && !*abort_flag; t += n_pairs) {
+        const bool ph2 = t >= tiles1;
+        const ChainPhase& P = ph2 ? p2 : p1;
+        const int u = ph2 ? t - tiles1 : t;
+        const int rb = u / P.n_n;
+        const int m0 = rb * 2 * kBM + static_cast<int>(rank) * kBM;
+        const int n0 = (u % P.n_n) * P.BN + static_cast<int>(rank) * (P.BN / 2);
+        const CUtensorMap* tm = is_w ? (ph2 ? &tm_w2 : &tm_w1) : (ph2 ? &tm_x2 : &tm_x1);
+        if (ph2 && !is_w) {
+          // this row block's rows of Y1 are stored (bounded wait; the phase-1 tiles never wait)
+          const uint64_t t0 = globaltimer_ns();
+          bool ok = true;
+          while (ld_acquire_gpu(done + rb) < need) {
+            if (*abort_flag || globaltimer_ns() - t0 > wait_ns) {
+              ok = false;
+              break;
+            }
+          }
+          if (!ok) {
+            record_error(err, kErrTimeout | kSiteLinear);
+            *abort_flag = 1;
+            break;
+          }
+          fence_proxy_async_global();  // other CTAs wrote the rows through the async proxy
+          if (atomicAdd(seen + rb, 1) + 1 == 2 * P.n_n) {
+            // every producer that waits on this row block is past its wait: zero both
+            // counters for the next launch
+            done[rb] = 0;
+            seen[rb] = 0;
+          }
+        }
+        const int b_bytes = (P.BN / 2) * kBK * 2;
+        for (int kb = 0; kb < P.kblocks; ++kb) {
+          if (!mbar_wait(&empty[stage], phase ^ 1u, wait_ns)) {
+            record_error(err, kErrTimeout | kSiteLinear);
+            *abort_flag = 1;
+            break;
+          }
+          const uint32_t bar = full0 + stage * 8;
+          if (is_w) {
+            if (leader) mbar_arrive_expect_tx(&full[stage], 2 * b_bytes);
+            tma_load_2d_pair(sB + stage * C::B_BYTES, tm, bar, kb * kBK, n0);
+          } else {
+            if (leader) mbar_arrive_expect_tx(&full[stage], 2 * C::A_BYTES);
+            tma_load_2d_pair(sA + stage * C::A_BYTES, tm, bar, kb * kBK, m0);
+          }
+          if (++stage == C::STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+    }
+  } else if (warp == kMmaWarp) {
+    if (leader && lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      const uint32_t a_base = smem_u32(sA), b_base = smem_u32(sB);
+      for (int t = pair; t < tiles && !*abort_flag; t += n_pairs) {
+        const ChainPhase& P = t >= tiles1 ? p2 : p1;
+        if (!mbar_wait(&acc_empty[acc], acc_phase ^ 1u, wait_ns)) {
+          record_error(err, kErrTimeout | kSiteLinear);
+          *abort_flag = 1;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem + static_cast<uint32_t>(acc) * C::ACC_STRIDE;
+        bool ok = true;
+        for (int kb = 0; kb < P.kblocks; ++kb) {
+          if (!mbar_wait(&full[stage], phase, wait_ns)) {
+            record_error(err, kErrTimeout | kSiteLinear);
+            *abort_flag = 1;
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a0 = a_base + stage * C::A_BYTES, b0 = b_base + stage * C::B_BYTES;
+#pragma unroll
+          for (int kk = 0; kk < kBK / 16; ++kk) {
+            const uint64_t ad = sdesc_sw128(a0 + kk * 32, 16, 1024);
+            const uint64_t bd = sdesc_sw128(b0 + kk * 32, 16, 1024);
+            umma_bf16_ss_pair(d_tmem, ad, bd, P.idesc, (kb | kk) != 0 ? 1u : 0u);
+          }
+          umma_commit_pair_multicast(&empty[stage], 0x3);
+          if (++stage == C::STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        umma_commit_pair_multicast(&acc_full[acc], 0x3);
+        acc ^= 1;
+        if (acc == 0) acc_phase ^= 1u;
+      }
+    }
+  } else {
+    // epilogue warps: this CTA's 128 rows of the pair tile
+    const int quarter = warp & 3;
+    const int ew = warp - kEpiWarp0;
+    uint8_t* obuf = sOut + ew * 2 * kChunkBytes;
+    uint8_t* rbuf = sRes + ew * 2 * kChunkBytes;
+    uint64_t* rbar = res_full + ew * 2;
+    const uint32_t acc_empty0 = map_to_rank(smem_u32(acc_empty), 0);
+    const RopeArgs no_rope{};
+    uint32_t rphase = 0u;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    int out_slot = 0;
+    for (int t = pair; t < tiles; t += n_pairs) {
+      const bool ph2 = t >= tiles1;
+      const ChainPhase& P = ph2 ? p2 : p1;
+      const int u = ph2 ? t - tiles1 : t;
+      const int rb = u / P.n_n;
+      const int m0 = rb * 2 * kBM + static_cast<int>(rank) * kBM, n0 = (u % P.n_n) * P.BN;
+      const int row0 = m0 + quarter * 32;
+      const int nch = min(P.BN, P.N - n0) / 32;
+      if (!ph2 && lane == 0) epi_prefetch_residual(&tm_r1, rbuf, rbar, nch, n0, row0);
+      float4 cs[16];
+      bool ok = mbar_wait(&acc_full[acc], acc_phase, wait_ns);
+      ok = __all_sync(0xffffffffu, ok);
+      if (ok && !*abort_flag) {
+        tc_fence_after();
+        const uint32_t t_row =
+            tmem + (static_cast<uint32_t>(quarter * 32) << 16) + static_cast<uint32_t>(acc) * C::ACC_STRIDE;
+        ok = epi_tile(t_row, nch, n0, row0, !ph2, ph2 ? &tm_y2 : &tm_y1, &tm_r1, obuf, rbuf, rbar, rphase, out_slot,
+                      lane, wait_ns, no_rope, -1, cs);
+      }
+      if (!ok || *abort_flag) {
+        if (lane == 0) record_error(err, kErrTimeout | kSiteLinear);
+        *abort_flag = 1;
+        break;
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(acc_empty0 + acc * 8);
+      acc ^= 1;
+      if (acc == 0) acc_phase ^= 1u;
+      if (!ph2 && lane == 0) {
+        // this warp's rows of the tile are in global memory: publish them to the phase-2
+        // producers of the row block
+        bulk_wait_group<0>();
+        fence_proxy_async_global();
+        red_release_gpu_add(done + rb, 1);
+      }
+    }
+    if (lane == 0) bulk_wait_group<0>();
+  }
+  tc_fence_before();
+  cluster_sync_all();  // the peer's shared memory is read by the pair MMAs until here
+  if (warp == kMmaWarp) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem, C::TMEM_COLS);
+  }
+}
+
 int g_num_sms[64] = {0};
 int g_pair_slots[64][4] = {};  // co-resident CTA pairs for BN = 256, 192, 160, 224
+int g_chain_slots[64] = {};    // co-resident CTA pairs of the chained kernel
 
 template <int BN>
 kalm_status setup_pair(int dev, int slot) {
@@ -625,6 +882,20 @@ kalm_status setup_linear_kernels() {
   if ((st = setup_pair<192>(dev, 1)) != KALM_OK) return st;
   if ((st = setup_pair<160>(dev, 2)) != KALM_OK) return st;
   if ((st = setup_pair<224>(dev, 3)) != KALM_OK) return st;
+  // the chained kernel: its shared memory and how many of its CTA pairs fit at once
+  st = check_cuda(cudaFuncSetAttribute(linear_chain_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, ChainCfg::SMEM),
+                  "cudaFuncSetAttribute(linear_chain_kernel)");
+  if (st != KALM_OK) return st;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * 74, 1, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = ChainCfg::SMEM;
+  int clusters = 0;
+  if (cudaOccupancyMaxActiveClusters(&clusters, linear_chain_kernel, &cfg) != cudaSuccess || clusters <= 0) {
+    cudaGetLastError();
+    clusters = sms / 2;
+  }
+  g_chain_slots[dev] = clusters;
   return KALM_OK;
 }
 
@@ -749,6 +1020,90 @@ kalm_status launch_linear(const kalm_bf16* x, int64_t ldx, const kalm_bf16* w, i
   return check_cuda(ce, "launch linear_kernel");
 }
 
+namespace {
+
+// Tile width of one phase of the chained launch, by the same rounds x (width + fixed
+// cost) model as the separate projections (widths whose half is whole 8-row groups).
+int chain_width(int64_t n_m, int32_t n, int64_t slots) {
+  const int bns[4] = {256, 192, 160, 224};
+  int best = 256;
+  int64_t best_cost = INT64_MAX;
+  for (int bn : bns) {
+    const int64_t tiles = n_m * ((n + bn - 1) / bn);
+    const int64_t cost = ((tiles + slots - 1) / slots) * (bn + 480);
+    if (cost < best_cost) {
+      best_cost = cost;
+      best = bn;
+    }
+  }
+  return best;
+}
+
+}  // namespace
+
+int64_t linear_chain_sync_len(int64_t m) { return m < 0 ? -1 : 2 * ((m + 2 * kBM - 1) / (2 * kBM)); }
+
+// y1 <- x1 . w1^T + y1 (in place), then y2 <- y1 . w2^T, in one launch (kalm_linear_chain).
+kalm_status launch_linear_chain(const kalm_bf16* x1, int64_t ldx1, const kalm_bf16* w1, int64_t ldw1, kalm_bf16* y1,
+                                int64_t ldy1, const kalm_bf16* w2, int64_t ldw2, kalm_bf16* y2, int64_t ldy2,
+                                int64_t m, int32_t n1, int32_t k1, int32_t n2, int32_t* sync, int64_t sync_len,
+                                cudaStream_t stream) {
+  const char* who = "kalm_linear_chain";
+  if (m < 0 || n1 <= 0 || k1 <= 0 || n2 <= 0)
+    return fail(KALM_ERR_INVALID_ARG, "%s: m=%lld n1=%d k1=%d n2=%d", who, (long long)m, n1, k1, n2);
+  if (m == 0) return KALM_OK;
+  if (m > INT32_MAX - 512) return fail(KALM_ERR_INVALID_ARG, "%s: m=%lld too large", who, (long long)m);
+  if (!x1 || !w1 || !y1 || !w2 || !y2) return fail(KALM_ERR_INVALID_ARG, "%s: NULL pointer", who);
+  if (n1 % 32 || n2 % 32) return fail(KALM_ERR_UNSUPPORTED, "%s: n1=%d and n2=%d must be multiples of 32", who, n1, n2);
+  if (k1 % 8) return fail(KALM_ERR_INVALID_ARG, "%s: k1=%d must be a multiple of 8", who, k1);
+  if (ldx1 % 8 || ldw1 % 8 || ldy1 % 8 || ldw2 % 8 || ldy2 % 8 || ldx1 < k1 || ldw1 < k1 || ldy1 < n1 ||
+      ldw2 < n1 || ldy2 < n2)
+    return fail(KALM_ERR_INVALID_ARG, "%s: strides must be multiples of 8 and >= the row width", who);
+  if (!aligned16(x1) || !aligned16(w1) || !aligned16(y1) || !aligned16(w2) || !aligned16(y2))
+    return fail(KALM_ERR_INVALID_ARG, "%s: bf16 pointers must be 16-byte aligned", who);
+  if (m < 2 * kBM) {
+    // below one CTA pair's rows: the two projections one after the other
+    kalm_status st = launch_linear(x1, ldx1, w1, ldw1, y1, ldy1, y1, ldy1, m, n1, k1, stream, who);
+    if (st != KALM_OK) return st;
+    return launch_linear(y1, ldy1, w2, ldw2, nullptr, 0, y2, ldy2, m, n2, n1, stream, who);
+  }
+  if (!sync || (reinterpret_cast<uintptr_t>(sync) & 3u))
+    return fail(KALM_ERR_INVALID_ARG, "%s: sync must be a 4-byte aligned int32 array", who);
+  if (sync_len < linear_chain_sync_len(m))
+    return fail(KALM_ERR_INVALID_ARG, "%s: sync_len=%lld < %lld", who, (long long)sync_len,
+                (long long)linear_chain_sync_len(m));
+  int dev = 0;
+  cudaGetDevice(&dev);
+  const int64_t slots = (dev < 64 && g_chain_slots[dev] > 0) ? g_chain_slots[dev] : num_sms() / 2;
+  const int64_t n_m = (m + 2 * kBM - 1) / (2 * kBM);
+  ChainPhase p1{}, p2{};
+  p1.N = n1;
+  p1.K = k1;
+  p1.BN = chain_width(n_m, n1, slots);
+  p1.idesc = idesc_bf16_f32(2 * kBM, p1.BN, false, false);
+  p1.n_n = (n1 + p1.BN - 1) / p1.BN;
+  p1.kblocks = (k1 + kBK - 1) / kBK;
+  p2.N = n2;
+  p2.K = n1;
+  p2.BN = chain_width(n_m, n2, slots);
+  p2.idesc = idesc_bf16_f32(2 * kBM, p2.BN, false, false);
+  p2.n_n = (n2 + p2.BN - 1) / p2.BN;
+  p2.kblocks = (n1 + kBK - 1) / kBK;
+  CUtensorMap tx1, tw1, ty1, tr1, tx2, tw2, ty2, tr2;
+  kalm_status st = make_operand_maps(&tx1, &tw1, &ty1, &tr1, x1, ldx1, w1, ldw1, y1, ldy1, y1, ldy1, m, n1, k1,
+                                     static_cast<uint32_t>(p1.BN / 2));
+  if (st != KALM_OK) return st;
+  st = make_operand_maps(&tx2, &tw2, &ty2, &tr2, y1, ldy1, w2, ldw2, nullptr, 0, y2, ldy2, m, n2, n1,
+                         static_cast<uint32_t>(p2.BN / 2));
+  if (st != KALM_OK) return st;
+  const int64_t tiles = n_m * (p1.n_n + p2.n_n);
+  const int pairs = static_cast<int>(tiles < slots ? tiles : slots);
+  return check_cuda(launch_pdl(linear_chain_kernel, dim3(2 * pairs), dim3(kThreads), ChainCfg::SMEM, stream, tx1, tw1,
+                               ty1, tr1, tx2, tw2, ty2, p1, p2, static_cast<int>(m), sync, kWaitNs,
+                               device_error_word()),
+                    "launch linear_chain_kernel");
+}
+
 }  // namespace kalm
 
 using namespace kalm;
@@ -760,6 +1115,18 @@ extern "C" kalm_status kalm_linear(const kalm_bf16* x, int64_t ldx, const kalm_b
   if (st != KALM_OK) return st;
   return launch_linear(x, ldx, w, ldw, residual, ldr, y, ldy, m, n, k, static_cast<cudaStream_t>(stream),
                        "kalm_linear");
+}
+
+extern "C" int64_t kalm_linear_chain_sync_len(int64_t m) { return linear_chain_sync_len(m); }
+
+extern "C" kalm_status kalm_linear_chain(const kalm_bf16* x1, int64_t ldx1, const kalm_bf16* w1, int64_t ldw1,
+                                         kalm_bf16* y1, int64_t ldy1, const kalm_bf16* w2, int64_t ldw2,
+                                         kalm_bf16* y2, int64_t ldy2, int64_t m, int32_t n1, int32_t k1, int32_t n2,
+                                         int32_t* sync, int64_t sync_len, kalm_stream_t stream) {
+  kalm_status st = ensure_device(nullptr);
+  if (st != KALM_OK) return st;
+  return launch_linear_chain(x1, ldx1, w1, ldw1, y1, ldy1, w2, ldw2, y2, ldy2, m, n1, k1, n2, sync, sync_len,
+                             static_cast<cudaStream_t>(stream));
 }
 
 extern "C" kalm_status kalm_cross_kv_proj(const kalm_bf16* pooled, int64_t pooled_ld, int64_t total_pooled,

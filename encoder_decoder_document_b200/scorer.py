@@ -27,7 +27,8 @@ import torch
 from . import (kalm_broadcast_rows, kalm_check_device_errors, kalm_chunk_pool, kalm_cross_kv_proj,
                kalm_device_check, kalm_linear, kalm_merged_attention_out_proj, kalm_attention_out_proj_sync_len,
                kalm_merged_attention, kalm_ragged_offsets, kalm_yes_no_score, kalm_attention_items,
-               kalm_attention_schedule, kalm_linear_rope, kalm_rope_table)
+               kalm_attention_schedule, kalm_linear_rope, kalm_rope_table, kalm_linear_chain,
+               kalm_linear_chain_sync_len)
 
 HEAD_DIM = 256
 # the pages' runtime limits ("Runtime boundaries"): passages of at most 1,024 encoder
@@ -66,7 +67,8 @@ class FBNLScorer:
     (the readout reads nothing else)."""
 
     def __init__(self, weights: DeviceWeights, n_q: int, n_kv: int, chunk: int = 4, head_dim: int = HEAD_DIM,
-                 prune: bool = True, rope_theta: Optional[float] = None, fused_out: bool = False):
+                 prune: bool = True, rope_theta: Optional[float] = None, fused_out: bool = False,
+                 chain: bool = True):
         kalm_device_check()
         self.w = weights
         self.L, qkv_rows, self.H = weights.w_qkv.shape
@@ -78,6 +80,10 @@ class FBNLScorer:
         # attention and output projection of every layer but the pruned last one in one
         # launch (kalm_merged_attention_out_proj)
         self.fused_out = fused_out
+        # each layer's output projection and the next layer's Q|K|V projection in one launch
+        # (kalm_linear_chain), in the pruned stack without rotation and without the fused layer
+        self.chain = chain and prune and rope_theta is None and not fused_out
+        self._qkv_ready = -1  # layer whose Q|K|V the last chained launch produced
         # the rotary angles' (cos, sin), built once for this base
         self.rope_tab = kalm_rope_table(rope_theta, head_dim) if rope_theta is not None else None
         self._shape = None
@@ -126,6 +132,8 @@ class FBNLScorer:
         self.yes, self.no, self.margin, self.score = self.result[0], self.result[1], self.result[2], self.result[3]
         # the fused layer's per-document counters (zero before a launch, left zero by it)
         self.sync = torch.zeros(max(kalm_attention_out_proj_sync_len(n_docs, lq, H), 1), dtype=torch.int32, **kw)
+        # the chained projections' per-row-block counters (zero before a launch, left zero by it)
+        self.chain_sync = torch.zeros(max(kalm_linear_chain_sync_len(rows), 1), dtype=torch.int32, **kw)
         self.graphs = None
         self.graphs_decode = None
 
@@ -238,7 +246,8 @@ class FBNLScorer:
             q, ks, vs = (t[:Lq] for t in self.qkv_views())
             in_off = self.zero_off
         else:
-            self.layer_qkv(l)
+            if not (self.chain and self._qkv_ready == l):  # else the previous launch projected them
+                self.layer_qkv(l)
             q, ks, vs = self.qkv_views()
             in_off = None
         if self.fused_out and not last:
@@ -253,6 +262,12 @@ class FBNLScorer:
             self._join_side()
             kalm_linear(self.o[Lq - 1::Lq], self.w.w_o[l], x_last, residual=x_last)
             self._mark("o_proj")
+        elif self.chain:
+            # X += O Wo, then the next layer's Q|K|V from the updated X, in one launch
+            self._join_side()
+            kalm_linear_chain(self.o, self.w.w_o[l], self.x, self.w.w_qkv[l + 1], self.qkv, self.chain_sync)
+            self._mark("o_proj_qkv")
+            self._qkv_ready = l + 1
         else:
             self.layer_out(l)
 
@@ -268,6 +283,7 @@ class FBNLScorer:
 
     def decode(self, broadcast: bool = True) -> None:
         """The query side: the decoder stack over the cached cross K/V, then the readout."""
+        self._qkv_ready = -1
         if broadcast and self.marks is None and self.prune:
             # layer 0's Q|K|V and attention read only the query input: the broadcast of X
             # runs beside them and the first output projection waits for it

@@ -153,6 +153,35 @@ kalm_status kalm_linear(const kalm_bf16* x, int64_t ldx, const kalm_bf16* w, int
                         const kalm_bf16* residual, int64_t ldr, kalm_bf16* y, int64_t ldy,
                         int64_t m, int32_t n, int32_t k, kalm_stream_t stream);
 
+/* A decoder layer's output projection and the next layer's Q|K|V projection,
+ * chained in one launch (same passage as kalm_linear: the residual update
+ * X <- X + O Wo, then the next layer projects the updated X):
+ *   y1 <- x1 . w1^T + y1            (in place: y1 is also the residual)
+ *   y2 <- y1 . w2^T                  (reads the y1 just written)
+ * Each output element is computed as kalm_linear computes it (same K order, one
+ * rounding to bf16), so the results are bit for bit those of the two separate
+ * calls.  A tile of the second product starts as soon as the first product's
+ * tiles of its 256-row block are stored, instead of after the whole first product.
+ *
+ * x1 [m][ldx1], w1 [n1][ldw1] (k1 inputs), y1 [m][ldy1] (n1 columns, in/out),
+ * w2 [n2][ldw2] (n1 inputs), y2 [m][ldy2] (n2 columns); bf16, 16-byte aligned,
+ * strides multiples of 8.  y1 must not overlap x1 or w1, and y2 none of x1, w1, y1.
+ * sync: int32[sync_len], sync_len >= kalm_linear_chain_sync_len(m), caller-owned
+ *   device memory that must be zero at the call; every launch that ends without
+ *   a device error leaves it zero again.  After a device error (see
+ *   kalm_check_device_errors) zero it before the next call.  Calls that share
+ *   one array must not overlap on the GPU.  Unused (may be NULL) when m < 256,
+ *   where the two products run as two launches.
+ * Requirements: m >= 0, n1 % 32 == 0, n2 % 32 == 0, k1 % 8 == 0. */
+kalm_status kalm_linear_chain(const kalm_bf16* x1, int64_t ldx1, const kalm_bf16* w1, int64_t ldw1,
+                              kalm_bf16* y1, int64_t ldy1, const kalm_bf16* w2, int64_t ldw2,
+                              kalm_bf16* y2, int64_t ldy2, int64_t m, int32_t n1, int32_t k1,
+                              int32_t n2, int32_t* sync, int64_t sync_len, kalm_stream_t stream);
+
+/* Length in int32 of kalm_linear_chain's sync array for m rows (2 per 256-row
+ * block), or -1 for m < 0. */
+int64_t kalm_linear_chain_sync_len(int64_t m);
+
 /* Step 2 - cross-attention K/V projection of the cached pooled vectors for
  * n_layers decoder layers at once.
  * "KaLM-Reranker-V1-Nano - MLX", "What this is": the cross-attention KV is

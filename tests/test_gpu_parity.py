@@ -214,6 +214,74 @@ def test_linear(kalm, m, n, k, res):
     _one_step(from_dev(y), oracle.linear(x, w, residual=r), x, w, r)
 
 
+@pytest.mark.parametrize("m,n1,k1,n2", [
+    (12800, 640, 1024, 1536),   # Nano: output projection, then the next layer's Q|K|V
+    (12700, 640, 1024, 1536),   # a ragged last row block (rows past m are clipped)
+    (256, 640, 1024, 1536),     # exactly one CTA pair of rows
+    (200, 640, 1024, 1536),     # below one pair: two launches
+    (3000, 1152, 1024, 1536),   # Small's widths
+    (2560, 2560, 2048, 4096)])  # Large's widths
+def test_linear_chain_matches_two_projections(kalm, m, n1, k1, n2):
+    """kalm_linear_chain = kalm_linear(x1, w1, y1, residual=y1) then kalm_linear(y1, w2, y2),
+    bit for bit (each element keeps its K order and one rounding), and the counters it
+    uses are back at zero after every call, so a repeat gives the same bits."""
+    g = torch.Generator(device="cuda").manual_seed(m + n1 + k1 + n2)
+    x1 = torch.randn(m, k1, device="cuda", generator=g).bfloat16()
+    w1 = (torch.randn(n1, k1, device="cuda", generator=g) * 0.02).bfloat16()
+    r = torch.randn(m, n1, device="cuda", generator=g).bfloat16()
+    w2 = (torch.randn(n2, n1, device="cuda", generator=g) * 0.02).bfloat16()
+    y1_ref, y2_ref = r.clone(), torch.empty(m, n2, dtype=torch.bfloat16, device="cuda")
+    kalm.kalm_linear(x1, w1, y1_ref, residual=y1_ref)
+    kalm.kalm_linear(y1_ref, w2, y2_ref)
+    sync = torch.zeros(max(kalm.kalm_linear_chain_sync_len(m), 1), dtype=torch.int32, device="cuda")
+    for _ in range(2):
+        y1 = r.clone()
+        y2 = torch.full((m, n2), float("nan"), dtype=torch.bfloat16, device="cuda")
+        kalm.kalm_linear_chain(x1, w1, y1, w2, y2, sync)
+        kalm.kalm_check_device_errors()
+        assert torch.equal(y1, y1_ref)
+        assert torch.equal(y2, y2_ref)
+        assert int(sync.abs().sum()) == 0
+
+
+def test_linear_chain_against_the_oracle(kalm):
+    """The chained projections against the oracle's two products at a shape with a
+    ragged last row block: the first product within one bf16 step, the second from
+    the first's bf16 result within one bf16 step."""
+    rng = np.random.default_rng(11)
+    m, n1, k1, n2 = 700, 640, 512, 1536
+    x1 = rand_bf16(rng, (m, k1))
+    w1 = rand_bf16(rng, (n1, k1), 0.02)
+    r = rand_bf16(rng, (m, n1))
+    w2 = rand_bf16(rng, (n2, n1), 0.02)
+    y1 = f64_to_dev(r)
+    y2 = torch.empty(m, n2, dtype=torch.bfloat16, device="cuda")
+    sync = torch.zeros(kalm.kalm_linear_chain_sync_len(m), dtype=torch.int32, device="cuda")
+    kalm.kalm_linear_chain(f64_to_dev(x1), f64_to_dev(w1), y1, f64_to_dev(w2), y2, sync)
+    kalm.kalm_check_device_errors()
+    got1 = from_dev(y1)
+    _one_step(got1, oracle.linear(x1, w1, residual=r), x1, w1, r)
+    _one_step(from_dev(y2), oracle.linear(got1, w2), got1, w2, None)
+
+
+def test_linear_chain_rejects_bad_arguments(kalm):
+    m, n1, k1, n2 = 512, 640, 1024, 1536
+    x1 = torch.zeros(m, k1, dtype=torch.bfloat16, device="cuda")
+    w1 = torch.zeros(n1, k1, dtype=torch.bfloat16, device="cuda")
+    y1 = torch.zeros(m, n1, dtype=torch.bfloat16, device="cuda")
+    w2 = torch.zeros(n2, n1, dtype=torch.bfloat16, device="cuda")
+    y2 = torch.zeros(m, n2, dtype=torch.bfloat16, device="cuda")
+    short = torch.zeros(kalm.kalm_linear_chain_sync_len(m) - 1, dtype=torch.int32, device="cuda")
+    with pytest.raises(kalm.KalmError):
+        kalm.kalm_linear_chain(x1, w1, y1, w2, y2, short)
+    with pytest.raises(kalm.KalmError):
+        kalm.kalm_linear_chain(x1, w1, y1, w2, y2, None)
+    with pytest.raises(kalm.KalmError):
+        kalm.kalm_linear_chain(x1, w1, y1, w2[:, :512], y2, short)
+    assert kalm.kalm_linear_chain_sync_len(-1) == -1
+    assert kalm.kalm_linear_chain_sync_len(12800) == 100
+
+
 def test_linear_in_place_residual_and_strided(kalm):
     rng = np.random.default_rng(21)
     m, n, k = 200, 640, 1024
@@ -548,6 +616,38 @@ def test_pruned_stack_matches_full_stack(kalm, name, layers):
     assert np.abs(res[0] - res[1]).max() <= 1e-6
     y, n, m, s = oracle.forward_query(q)
     assert np.abs(res[1][3] - s).max() <= SCORE_TOL
+
+
+def test_chained_projections_match_separate_launches(kalm):
+    """The scorer's default (each output projection chained with the next layer's
+    Q|K|V projection in one launch) gives the same scores, bit for bit, as separate
+    launches: eagerly, in the step graph and in the decode-only graph (Nano, all 100
+    documents); the chained launches leave their counters at zero."""
+    from encoder_decoder_document_b200.scorer import DeviceWeights, FBNLScorer
+    q = synthetic.make_query("nano")
+    enc = torch.from_numpy(q.enc.view(np.int16)).view(torch.bfloat16)
+    dl = torch.from_numpy(q.doc_len)
+    x0 = torch.from_numpy(q.x0.view(np.int16)).view(torch.bfloat16)
+    res = []
+    for chain in (False, True):
+        sc = FBNLScorer(DeviceWeights.from_bits(q.weights), q.n_q, q.n_kv, chain=chain)
+        assert sc.chain == chain
+        sc.rerank(q.x0, q.enc, q.doc_len)
+        eager = sc.scores_to_host().numpy().copy()
+        sc.load_inputs(enc, dl, x0)
+        sc.capture()
+        sc.run()
+        graph = sc.scores_to_host().numpy().copy()
+        sc.cache_documents(enc, dl)
+        sc.graphs_decode[sc.slot].replay()
+        decode = sc.scores_to_host().numpy().copy()
+        kalm.kalm_check_device_errors()
+        res.append((eager, graph, decode))
+        if chain:
+            assert int(sc.chain_sync.abs().sum()) == 0
+    for a, b in zip(res[0], res[1]):
+        assert np.array_equal(a, b)
+    assert np.array_equal(res[1][0], res[1][1]) and np.array_equal(res[1][0], res[1][2])
 
 
 def _sample_docs(q, k=8, seed=0):
