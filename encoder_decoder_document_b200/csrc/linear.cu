@@ -704,12 +704,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             break;
           }
           fence_proxy_async_global();  // other CTAs wrote the rows through the async proxy
-          if (atomicAdd(seen + rb, 1) + 1 == 2 * P.n_n) {
-            // every producer that waits on this row block is past its wait: zero both
-            // counters for the next launch
-            done[rb] = 0;
-            seen[rb] = 0;
-          }
         }
         const int b_bytes = (P.BN / 2) * kBK * 2;
         for (int kb = 0; kb < P.kblocks; ++kb) {
@@ -730,6 +724,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             stage = 0;
             phase ^= 1u;
           }
+        }
+        if (ph2 && !is_w && atomicAdd(seen + rb, 1) + 1 == 2 * P.n_n) {
+          // (after the tile's loads, off their path) every producer that waits on this row
+          // block is past its wait: zero both counters for the next launch
+          done[rb] = 0;
+          seen[rb] = 0;
         }
       }
     }
