@@ -1022,9 +1022,14 @@ kalm_status launch_linear(const kalm_bf16* x, int64_t ldx, const kalm_bf16* w, i
 
 namespace {
 
-// Tile width of one phase of the chained launch, by the same rounds x (width + fixed
-// cost) model as the separate projections (widths whose half is whole 8-row groups).
+// Tile width of one phase of the chained launch (widths whose half is whole 8-row
+// groups).  Both phases share one tile list, so a phase need not fill whole rounds of
+// pairs: the widest width that divides n (no partial last tile, fewest operand bytes
+// per output) is taken; otherwise the same rounds x (width + fixed cost) model as the
+// separate projections.
 int chain_width(int64_t n_m, int32_t n, int64_t slots) {
+  for (int bn : {256, 224, 192, 160})
+    if (n % bn == 0) return bn;
   const int bns[4] = {256, 192, 160, 224};
   int best = 256;
   int64_t best_cost = INT64_MAX;
