@@ -54,6 +54,10 @@ def test_no_device_is_an_explicit_error(lib):
     assert lib.kalm_device_check() == 3
     assert lib.kalm_linear(None, 0, None, 0, None, 0, None, 0, 0, 32, 8, None) == 3
     assert lib.kalm_chunk_pool(None, 0, None, None, 0, 8, 4, None, 0, None, 0, None) == 3
+    assert lib.kalm_linear_chain(None, 0, None, 0, None, 0, None, 0, None, 0, 512, 640, 1024, 1536, None, 0,
+                                 None) == 3
+    # host-side size helpers need no device
+    assert lib.kalm_linear_chain_sync_len(12800) == 100 and lib.kalm_linear_chain_sync_len(-1) == -1
     with pytest.raises(k.KalmError) as e:
         k.kalm_device_check()
     assert e.value.name == "KALM_ERR_NO_DEVICE"
