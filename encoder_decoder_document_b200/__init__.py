@@ -17,6 +17,7 @@ from ._abi import KalmError, call, load, library_path  # noqa: F401
 __all__ = [
     "KalmError", "load", "library_path", "kalm_version", "kalm_device_check", "kalm_check_device_errors",
     "kalm_ragged_offsets", "kalm_chunk_pool", "kalm_linear", "kalm_linear_chain", "kalm_linear_chain_sync_len",
+    "kalm_linear_chain_rope",
     "kalm_cross_kv_proj", "kalm_merged_attention",
     "kalm_merged_attention_out_proj", "kalm_merged_attention_out_proj_static", "kalm_attention_out_proj_sync_len",
     "kalm_yes_no_score", "kalm_broadcast_rows", "kalm_selftest_wait_timeout", "kalm_attention_items",
@@ -106,6 +107,24 @@ def kalm_linear_chain(x1: torch.Tensor, w1: torch.Tensor, y1: torch.Tensor, w2: 
     call("kalm_linear_chain", _p(x1, torch.bfloat16), _ld(x1), _p(w1, torch.bfloat16), _ld(w1),
          _p(y1, torch.bfloat16), _ld(y1), _p(w2, torch.bfloat16), _ld(w2), _p(y2, torch.bfloat16), _ld(y2), m, n1, k1,
          n2, _p(sync, torch.int32), sync.numel() if sync is not None else 0, _stream(stream))
+
+
+def kalm_linear_chain_rope(x1: torch.Tensor, w1: torch.Tensor, y1: torch.Tensor, w2: torch.Tensor, y2: torch.Tensor,
+                           q_off: torch.Tensor, rot_heads: int, table: torch.Tensor, sync: Optional[torch.Tensor],
+                           head_dim: int = HEAD_DIM, stream=None) -> None:
+    """kalm_linear_chain with the first rot_heads head vectors of every row of y2 rotated
+    by the row's decoder position (angles from kalm_rope_table), as kalm_linear_rope."""
+    m, k1 = x1.shape
+    n1, n2 = w1.shape[0], w2.shape[0]
+    if w1.shape[1] != k1 or y1.shape != (m, n1) or w2.shape[1] != n1 or y2.shape != (m, n2):
+        raise KalmError(1, "kalm_linear_chain_rope", f"shapes x1{tuple(x1.shape)} w1{tuple(w1.shape)} "
+                                                     f"y1{tuple(y1.shape)} w2{tuple(w2.shape)} y2{tuple(y2.shape)}")
+    if table.numel() != MAX_QUERY_TOKENS * head_dim or not table.is_contiguous():
+        raise KalmError(1, "kalm_linear_chain_rope", "table must be a contiguous kalm_rope_table output")
+    call("kalm_linear_chain_rope", _p(x1, torch.bfloat16), _ld(x1), _p(w1, torch.bfloat16), _ld(w1),
+         _p(y1, torch.bfloat16), _ld(y1), _p(w2, torch.bfloat16), _ld(w2), _p(y2, torch.bfloat16), _ld(y2), m, n1, k1,
+         n2, rot_heads * head_dim, head_dim, _p(q_off, torch.int64), q_off.numel() - 1, _p(table, torch.float32),
+         _p(sync, torch.int32), sync.numel() if sync is not None else 0, _stream(stream))
 
 
 def kalm_cross_kv_proj(pooled: torch.Tensor, w_kv: torch.Tensor, kv_cross: torch.Tensor, n_kv: int,

@@ -32,6 +32,8 @@ SIGNATURES = {
     "kalm_linear_chain": [c_vp, c_i64, c_vp, c_i64, c_vp, c_i64, c_vp, c_i64, c_vp, c_i64, c_i64, c_i32, c_i32,
                           c_i32, c_vp, c_i64, c_vp],
     "kalm_linear_chain_sync_len": [c_i64],
+    "kalm_linear_chain_rope": [c_vp, c_i64, c_vp, c_i64, c_vp, c_i64, c_vp, c_i64, c_vp, c_i64, c_i64, c_i32, c_i32,
+                               c_i32, c_i32, c_i32, c_vp, c_i32, c_vp, c_vp, c_i64, c_vp],
     "kalm_cross_kv_proj": [c_vp, c_i64, c_i64, c_i32, c_vp, c_i32, c_i32, c_i32, c_vp, c_vp],
     "kalm_merged_attention": [c_vp, c_i64, c_vp, c_vp, c_i64, c_vp, c_vp, c_i64, c_vp, c_vp, c_i64, c_vp, c_i32,
                               c_i32, c_i64, c_i64, c_i32, c_i32, c_i32, c_f32, c_i32, c_vp, c_vp, c_i64, c_vp,

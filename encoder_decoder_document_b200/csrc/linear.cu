@@ -616,12 +616,13 @@ struct ChainPhase {
   int n_n, kblocks;
 };
 
+template <bool ROPE>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     linear_chain_kernel(const __grid_constant__ CUtensorMap tm_x1, const __grid_constant__ CUtensorMap tm_w1,
                         const __grid_constant__ CUtensorMap tm_y1, const __grid_constant__ CUtensorMap tm_r1,
                         const __grid_constant__ CUtensorMap tm_x2, const __grid_constant__ CUtensorMap tm_w2,
                         const __grid_constant__ CUtensorMap tm_y2, const ChainPhase p1, const ChainPhase p2, int M,
-                        int* sync, uint64_t wait_ns, uint32_t* err) {
+                        int* sync, uint64_t wait_ns, uint32_t* err, const RopeArgs rope) {
   using C = ChainCfg;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -799,7 +800,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       const int row0 = m0 + quarter * 32;
       const int nch = min(P.BN, P.N - n0) / 32;
       if (!ph2 && lane == 0) epi_prefetch_residual(&tm_r1, rbuf, rbar, nch, n0, row0);
+      // the second product's rotated heads (one 256-column tile is one head); compiled out
+      // without rotation
+      const RopeArgs& rp = (ROPE && ph2) ? rope : no_rope;
+      const int rpos = ROPE ? rope_row(rp, n0, nch, row0, lane) : -1;
       float4 cs[16];
+      if constexpr (ROPE) rope_prefetch(rp, rpos, cs);
       bool ok = mbar_wait(&acc_full[acc], acc_phase, wait_ns);
       ok = __all_sync(0xffffffffu, ok);
       if (ok && !*abort_flag) {
@@ -807,7 +813,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         const uint32_t t_row =
             tmem + (static_cast<uint32_t>(quarter * 32) << 16) + static_cast<uint32_t>(acc) * C::ACC_STRIDE;
         ok = epi_tile(t_row, nch, n0, row0, !ph2, ph2 ? &tm_y2 : &tm_y1, &tm_r1, obuf, rbuf, rbar, rphase, out_slot,
-                      lane, wait_ns, no_rope, -1, cs);
+                      lane, wait_ns, rp, rpos, cs);
       }
       if (!ok || *abort_flag) {
         if (lane == 0) record_error(err, kErrTimeout | kSiteLinear);
@@ -883,15 +889,20 @@ kalm_status setup_linear_kernels() {
   if ((st = setup_pair<160>(dev, 2)) != KALM_OK) return st;
   if ((st = setup_pair<224>(dev, 3)) != KALM_OK) return st;
   // the chained kernel: its shared memory and how many of its CTA pairs fit at once
-  st = check_cuda(cudaFuncSetAttribute(linear_chain_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, ChainCfg::SMEM),
+  st = check_cuda(cudaFuncSetAttribute(linear_chain_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       ChainCfg::SMEM),
                   "cudaFuncSetAttribute(linear_chain_kernel)");
+  if (st != KALM_OK) return st;
+  st = check_cuda(cudaFuncSetAttribute(linear_chain_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       ChainCfg::SMEM),
+                  "cudaFuncSetAttribute(linear_chain_kernel<rope>)");
   if (st != KALM_OK) return st;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(2 * 74, 1, 1);
   cfg.blockDim = dim3(kThreads, 1, 1);
   cfg.dynamicSmemBytes = ChainCfg::SMEM;
   int clusters = 0;
-  if (cudaOccupancyMaxActiveClusters(&clusters, linear_chain_kernel, &cfg) != cudaSuccess || clusters <= 0) {
+  if (cudaOccupancyMaxActiveClusters(&clusters, linear_chain_kernel<false>, &cfg) != cudaSuccess || clusters <= 0) {
     cudaGetLastError();
     clusters = sms / 2;
   }
@@ -1052,8 +1063,7 @@ int64_t linear_chain_sync_len(int64_t m) { return m < 0 ? -1 : 2 * ((m + 2 * kBM
 kalm_status launch_linear_chain(const kalm_bf16* x1, int64_t ldx1, const kalm_bf16* w1, int64_t ldw1, kalm_bf16* y1,
                                 int64_t ldy1, const kalm_bf16* w2, int64_t ldw2, kalm_bf16* y2, int64_t ldy2,
                                 int64_t m, int32_t n1, int32_t k1, int32_t n2, int32_t* sync, int64_t sync_len,
-                                cudaStream_t stream) {
-  const char* who = "kalm_linear_chain";
+                                cudaStream_t stream, const char* who, const RopeArgs& rope = RopeArgs{}) {
   if (m < 0 || n1 <= 0 || k1 <= 0 || n2 <= 0)
     return fail(KALM_ERR_INVALID_ARG, "%s: m=%lld n1=%d k1=%d n2=%d", who, (long long)m, n1, k1, n2);
   if (m == 0) return KALM_OK;
@@ -1070,7 +1080,7 @@ kalm_status launch_linear_chain(const kalm_bf16* x1, int64_t ldx1, const kalm_bf
     // below one CTA pair's rows: the two projections one after the other
     kalm_status st = launch_linear(x1, ldx1, w1, ldw1, y1, ldy1, y1, ldy1, m, n1, k1, stream, who);
     if (st != KALM_OK) return st;
-    return launch_linear(y1, ldy1, w2, ldw2, nullptr, 0, y2, ldy2, m, n2, n1, stream, who);
+    return launch_linear(y1, ldy1, w2, ldw2, nullptr, 0, y2, ldy2, m, n2, n1, stream, who, rope);
   }
   if (!sync || (reinterpret_cast<uintptr_t>(sync) & 3u))
     return fail(KALM_ERR_INVALID_ARG, "%s: sync must be a 4-byte aligned int32 array", who);
@@ -1090,7 +1100,7 @@ kalm_status launch_linear_chain(const kalm_bf16* x1, int64_t ldx1, const kalm_bf
   p1.kblocks = (k1 + kBK - 1) / kBK;
   p2.N = n2;
   p2.K = n1;
-  p2.BN = chain_width(n_m, n2, slots);
+  p2.BN = rope.rot_cols > 0 ? 256 : chain_width(n_m, n2, slots);  // rotated heads: one head per tile
   p2.idesc = idesc_bf16_f32(2 * kBM, p2.BN, false, false);
   p2.n_n = (n2 + p2.BN - 1) / p2.BN;
   p2.kblocks = (n1 + kBK - 1) / kBK;
@@ -1103,10 +1113,13 @@ kalm_status launch_linear_chain(const kalm_bf16* x1, int64_t ldx1, const kalm_bf
   if (st != KALM_OK) return st;
   const int64_t tiles = n_m * (p1.n_n + p2.n_n);
   const int pairs = static_cast<int>(tiles < slots ? tiles : slots);
-  return check_cuda(launch_pdl(linear_chain_kernel, dim3(2 * pairs), dim3(kThreads), ChainCfg::SMEM, stream, tx1, tw1,
-                               ty1, tr1, tx2, tw2, ty2, p1, p2, static_cast<int>(m), sync, kWaitNs,
-                               device_error_word()),
-                    "launch linear_chain_kernel");
+  const cudaError_t ce =
+      rope.rot_cols > 0
+          ? launch_pdl(linear_chain_kernel<true>, dim3(2 * pairs), dim3(kThreads), ChainCfg::SMEM, stream, tx1, tw1,
+                       ty1, tr1, tx2, tw2, ty2, p1, p2, static_cast<int>(m), sync, kWaitNs, device_error_word(), rope)
+          : launch_pdl(linear_chain_kernel<false>, dim3(2 * pairs), dim3(kThreads), ChainCfg::SMEM, stream, tx1, tw1,
+                       ty1, tr1, tx2, tw2, ty2, p1, p2, static_cast<int>(m), sync, kWaitNs, device_error_word(), rope);
+  return check_cuda(ce, "launch linear_chain_kernel");
 }
 
 }  // namespace kalm
@@ -1131,7 +1144,28 @@ extern "C" kalm_status kalm_linear_chain(const kalm_bf16* x1, int64_t ldx1, cons
   kalm_status st = ensure_device(nullptr);
   if (st != KALM_OK) return st;
   return launch_linear_chain(x1, ldx1, w1, ldw1, y1, ldy1, w2, ldw2, y2, ldy2, m, n1, k1, n2, sync, sync_len,
-                             static_cast<cudaStream_t>(stream));
+                             static_cast<cudaStream_t>(stream), "kalm_linear_chain");
+}
+
+extern "C" kalm_status kalm_linear_chain_rope(const kalm_bf16* x1, int64_t ldx1, const kalm_bf16* w1, int64_t ldw1,
+                                              kalm_bf16* y1, int64_t ldy1, const kalm_bf16* w2, int64_t ldw2,
+                                              kalm_bf16* y2, int64_t ldy2, int64_t m, int32_t n1, int32_t k1,
+                                              int32_t n2, int32_t rot_cols, int32_t head_dim, const int64_t* q_off,
+                                              int32_t n_docs, const float* table, int32_t* sync, int64_t sync_len,
+                                              kalm_stream_t stream) {
+  kalm_status st = ensure_device(nullptr);
+  if (st != KALM_OK) return st;
+  const char* who = "kalm_linear_chain_rope";
+  if (head_dim != 256) return fail(KALM_ERR_UNSUPPORTED, "%s: head_dim=%d (only 256)", who, head_dim);
+  if (n2 % 256) return fail(KALM_ERR_UNSUPPORTED, "%s: n2=%d must be a multiple of 256", who, n2);
+  if (rot_cols <= 0 || rot_cols % head_dim || rot_cols > n2)
+    return fail(KALM_ERR_INVALID_ARG, "%s: rot_cols=%d must be a positive multiple of %d <= n2=%d", who, rot_cols,
+                head_dim, n2);
+  if (!table || !aligned16(table)) return fail(KALM_ERR_INVALID_ARG, "%s: table must be non-NULL and 16-byte aligned", who);
+  if (n_docs <= 0 || !q_off) return fail(KALM_ERR_INVALID_ARG, "%s: q_off/n_docs required", who);
+  RopeArgs rope{q_off, n_docs, rot_cols, reinterpret_cast<const float4*>(table), m, device_error_word()};
+  return launch_linear_chain(x1, ldx1, w1, ldw1, y1, ldy1, w2, ldw2, y2, ldy2, m, n1, k1, n2, sync, sync_len,
+                             static_cast<cudaStream_t>(stream), who, rope);
 }
 
 extern "C" kalm_status kalm_cross_kv_proj(const kalm_bf16* pooled, int64_t pooled_ld, int64_t total_pooled,

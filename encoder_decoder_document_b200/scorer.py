@@ -28,7 +28,7 @@ from . import (kalm_broadcast_rows, kalm_check_device_errors, kalm_chunk_pool, k
                kalm_device_check, kalm_linear, kalm_merged_attention_out_proj, kalm_attention_out_proj_sync_len,
                kalm_merged_attention, kalm_ragged_offsets, kalm_yes_no_score, kalm_attention_items,
                kalm_attention_schedule, kalm_linear_rope, kalm_rope_table, kalm_linear_chain,
-               kalm_linear_chain_sync_len)
+               kalm_linear_chain_rope, kalm_linear_chain_sync_len)
 
 HEAD_DIM = 256
 # the pages' runtime limits ("Runtime boundaries"): passages of at most 1,024 encoder
@@ -81,8 +81,9 @@ class FBNLScorer:
         # launch (kalm_merged_attention_out_proj)
         self.fused_out = fused_out
         # each layer's output projection and the next layer's Q|K|V projection in one launch
-        # (kalm_linear_chain), in the pruned stack without rotation and without the fused layer
-        self.chain = chain and prune and rope_theta is None and not fused_out
+        # (kalm_linear_chain, or kalm_linear_chain_rope with rotation), in the pruned stack
+        # without the fused layer
+        self.chain = chain and prune and not fused_out
         self._qkv_ready = -1  # layer whose Q|K|V the last chained launch produced
         # the rotary angles' (cos, sin), built once for this base
         self.rope_tab = kalm_rope_table(rope_theta, head_dim) if rope_theta is not None else None
@@ -265,7 +266,11 @@ class FBNLScorer:
         elif self.chain:
             # X += O Wo, then the next layer's Q|K|V from the updated X, in one launch
             self._join_side()
-            kalm_linear_chain(self.o, self.w.w_o[l], self.x, self.w.w_qkv[l + 1], self.qkv, self.chain_sync)
+            if self.rope_theta is None:
+                kalm_linear_chain(self.o, self.w.w_o[l], self.x, self.w.w_qkv[l + 1], self.qkv, self.chain_sync)
+            else:
+                kalm_linear_chain_rope(self.o, self.w.w_o[l], self.x, self.w.w_qkv[l + 1], self.qkv, self.q_off,
+                                       self.n_q + self.n_kv, self.rope_tab, self.chain_sync, self.D)
             self._mark("o_proj_qkv")
             self._qkv_ready = l + 1
         else:

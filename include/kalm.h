@@ -182,6 +182,21 @@ kalm_status kalm_linear_chain(const kalm_bf16* x1, int64_t ldx1, const kalm_bf16
  * block), or -1 for m < 0. */
 int64_t kalm_linear_chain_sync_len(int64_t m);
 
+/* kalm_linear_chain with the rotary embedding of the second product's first
+ * rot_cols columns applied in its epilogue, as kalm_linear_rope applies it (same
+ * passages, pairing, angle table and position rule): the output projection of a
+ * layer and the next layer's rotated Q|K|V projection in one launch.  Results
+ * are bit for bit those of kalm_linear (residual in place) then kalm_linear_rope.
+ * Arguments as kalm_linear_chain, and rot_cols, head_dim, q_off, n_docs, table
+ * as kalm_linear_rope (head_dim 256, n2 % 256 == 0, rot_cols a positive multiple
+ * of head_dim <= n2). */
+kalm_status kalm_linear_chain_rope(const kalm_bf16* x1, int64_t ldx1, const kalm_bf16* w1, int64_t ldw1,
+                                   kalm_bf16* y1, int64_t ldy1, const kalm_bf16* w2, int64_t ldw2,
+                                   kalm_bf16* y2, int64_t ldy2, int64_t m, int32_t n1, int32_t k1,
+                                   int32_t n2, int32_t rot_cols, int32_t head_dim, const int64_t* q_off,
+                                   int32_t n_docs, const float* table, int32_t* sync, int64_t sync_len,
+                                   kalm_stream_t stream);
+
 /* Step 2 - cross-attention K/V projection of the cached pooled vectors for
  * n_layers decoder layers at once.
  * "KaLM-Reranker-V1-Nano - MLX", "What this is": the cross-attention KV is

@@ -244,6 +244,33 @@ def test_linear_chain_matches_two_projections(kalm, m, n1, k1, n2):
         assert int(sync.abs().sum()) == 0
 
 
+@pytest.mark.parametrize("lq,rot_heads", [([128] * 100, 5), ([1, 2, 31, 129, 512, 64, 300], 5), ([7, 250, 19], 2)])
+def test_linear_chain_rope_matches_projection_and_rope(kalm, lq, rot_heads):
+    """kalm_linear_chain_rope = kalm_linear (residual in place) then kalm_linear_rope, bit
+    for bit: the Nano layout (100 documents of 128 rows), ragged documents across a
+    ragged last row block, and fewer than 256 rows (two launches)."""
+    g = torch.Generator(device="cuda").manual_seed(sum(lq) + rot_heads)
+    lq = np.asarray(lq, np.int64)
+    q_off = i64(np.concatenate([[0], np.cumsum(lq)]))
+    m, n1, k1, n2 = int(lq.sum()), 640, 1024, 6 * 256
+    x1 = torch.randn(m, k1, device="cuda", generator=g).bfloat16()
+    w1 = (torch.randn(n1, k1, device="cuda", generator=g) * 0.02).bfloat16()
+    r = torch.randn(m, n1, device="cuda", generator=g).bfloat16()
+    w2 = (torch.randn(n2, n1, device="cuda", generator=g) * 0.02).bfloat16()
+    table = kalm.kalm_rope_table(1e4)
+    y1_ref, y2_ref = r.clone(), torch.empty(m, n2, dtype=torch.bfloat16, device="cuda")
+    kalm.kalm_linear(x1, w1, y1_ref, residual=y1_ref)
+    kalm.kalm_linear_rope(y1_ref, w2, y2_ref, q_off, rot_heads, table)
+    sync = torch.zeros(max(kalm.kalm_linear_chain_sync_len(m), 1), dtype=torch.int32, device="cuda")
+    y1 = r.clone()
+    y2 = torch.full((m, n2), float("nan"), dtype=torch.bfloat16, device="cuda")
+    kalm.kalm_linear_chain_rope(x1, w1, y1, w2, y2, q_off, rot_heads, table, sync)
+    kalm.kalm_check_device_errors()
+    assert torch.equal(y1, y1_ref)
+    assert torch.equal(y2.view(torch.int16), y2_ref.view(torch.int16))
+    assert int(sync.abs().sum()) == 0
+
+
 def test_linear_chain_against_the_oracle(kalm):
     """The chained projections against the oracle's two products at a shape with a
     ragged last row block: the first product within one bf16 step, the second from
@@ -618,11 +645,13 @@ def test_pruned_stack_matches_full_stack(kalm, name, layers):
     assert np.abs(res[1][3] - s).max() <= SCORE_TOL
 
 
-def test_chained_projections_match_separate_launches(kalm):
+@pytest.mark.parametrize("rope_theta", [None, 1e4])
+def test_chained_projections_match_separate_launches(kalm, rope_theta):
     """The scorer's default (each output projection chained with the next layer's
-    Q|K|V projection in one launch) gives the same scores, bit for bit, as separate
-    launches: eagerly, in the step graph and in the decode-only graph (Nano, all 100
-    documents); the chained launches leave their counters at zero."""
+    Q|K|V projection in one launch, with or without rotation) gives the same scores,
+    bit for bit, as separate launches: eagerly, in the step graph and in the
+    decode-only graph (Nano, all 100 documents); the chained launches leave their
+    counters at zero."""
     from encoder_decoder_document_b200.scorer import DeviceWeights, FBNLScorer
     q = synthetic.make_query("nano")
     enc = torch.from_numpy(q.enc.view(np.int16)).view(torch.bfloat16)
@@ -630,7 +659,7 @@ def test_chained_projections_match_separate_launches(kalm):
     x0 = torch.from_numpy(q.x0.view(np.int16)).view(torch.bfloat16)
     res = []
     for chain in (False, True):
-        sc = FBNLScorer(DeviceWeights.from_bits(q.weights), q.n_q, q.n_kv, chain=chain)
+        sc = FBNLScorer(DeviceWeights.from_bits(q.weights), q.n_q, q.n_kv, chain=chain, rope_theta=rope_theta)
         assert sc.chain == chain
         sc.rerank(q.x0, q.enc, q.doc_len)
         eager = sc.scores_to_host().numpy().copy()
