@@ -62,6 +62,22 @@ MUTATIONS = [
     ("each document's last encoder row dropped",
      "a, b = int(query.tok_off[d]), int(query.tok_off[d + 1])",
      "a, b = int(query.tok_off[d]), int(query.tok_off[d + 1]) - 1"),
+    ("decoder residual dropped",
+     "Xn = linear(o.reshape(Lq, n_q * D), w_o_l, residual=X)", "Xn = linear(o.reshape(Lq, n_q * D), w_o_l)"),
+    ("every layer reads the first layer's cross weights",
+     "w_o[l], w_kv_cross[l], n_q", "w_o[l], w_kv_cross[0], n_q"),
+    ("softmax left unnormalised",
+     "o[:, h, :] = (e / s) @ vals", "o[:, h, :] = e @ vals"),
+    ("cross keys masked out",
+     "np.ones((Lq, Nc), dtype=bool)], axis=1)", "np.zeros((Lq, Nc), dtype=bool)], axis=1)"),
+    ("pooled chunks overlapping by one token",
+     "hi = min(lo + chunk, n)", "hi = min(lo + chunk + 1, n)"),
+    ("batched attention reading the next document's cross rows",
+     "k_cross[c0:c1], v_cross[c0:c1], scale,", "k_cross[c0 + 1:c1 + 1], v_cross[c0 + 1:c1 + 1], scale,"),
+    ("yes logit read with the no row",
+     "yes = x @ np.asarray(w_yes, np.float64)", "yes = x @ np.asarray(w_no, np.float64)"),
+    ("cross keys and values swapped",
+     "merged_attention_doc(q, ks, vs, kv[:, 0], kv[:, 1], scale)", "merged_attention_doc(q, ks, vs, kv[:, 1], kv[:, 0], scale)"),
 ]
 
 
