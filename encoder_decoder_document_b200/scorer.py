@@ -114,10 +114,11 @@ class FBNLScorer:
                            doc_len=torch.empty(n_docs, dtype=torch.int32, **kw),
                            x0=torch.empty(lq, H, dtype=torch.bfloat16, **kw)) for _ in range(2)]
         self.use_slot(0)
-        self.q_len = torch.full((n_docs,), lq, dtype=torch.int32, **kw)
         self.tok_off = torch.empty(n_docs + 1, dtype=torch.int64, **kw)
         self.pool_off = torch.empty(n_docs + 1, dtype=torch.int64, **kw)
-        self.q_off = torch.empty(n_docs + 1, dtype=torch.int64, **kw)
+        # every document of a query has the query's Lq decoder rows, so their offsets belong
+        # to the shape and are fixed here once (document d's rows start at d * Lq)
+        self.q_off = torch.arange(n_docs + 1, dtype=torch.int64, **kw) * lq
         self.zero_off = torch.zeros(n_docs, dtype=torch.int64, **kw)
         self.one_doc_off = torch.tensor([0, lq], dtype=torch.int64, **kw)  # the query's common rows
         self.pooled = torch.empty(max(total_pooled, 1), H, dtype=torch.bfloat16, **kw)
@@ -156,8 +157,6 @@ class FBNLScorer:
         the work order and the query input broadcast (both need only the offsets) run
         there, beside the pooling and the cross projection; the caller joins it."""
         kalm_ragged_offsets(self.doc_len, self.tok_off, self.pool_off, self.chunk)
-        self._mark("offsets")
-        kalm_ragged_offsets(self.q_len, self.q_off, None, 1)
         self._mark("offsets")
         if side is not None:
             side.wait_stream(torch.cuda.current_stream())
