@@ -211,3 +211,21 @@ def test_bench_reference_arm_contract():
     assert "workload" in line["config"]
     assert _bench(["--impl", "reference", "--config", "tiny", "--steps", "1", "--warmup", "0"],
                   {"RANK": "1", "WORLD_SIZE": "2"}) == []
+
+
+def test_bench_accounting_with_chained_projections():
+    """The bench's per-kernel work with the projections chained only regroups the work
+    of the unchained stack: the same total, and the chained launches plus the first
+    layer's Q|K|V and the last layer's output projection carry the unchained
+    projections' FLOPs (Nano and a one-layer stack, where nothing chains)."""
+    import importlib.util
+    import synthetic
+    spec = importlib.util.spec_from_file_location("bench_module", os.path.join(ROOT, "bench.py"))
+    bench = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(bench)
+    for name in ("nano", "tiny"):
+        q = synthetic.make_query(name, with_weights=False)
+        a, b = bench.workload(q, chain=False), bench.workload(q, chain=True)
+        assert a["total_flops"] == b["total_flops"]
+        assert b.get("o_proj_qkv", 0) + b["qkv_proj"] + b["o_proj"] == a["qkv_proj"] + a["o_proj"]
+        assert ("o_proj_qkv" in b) == (q.layers > 1)
